@@ -1,0 +1,248 @@
+"""Plain, slow, fp64 CPU oracle for LoLA's chunkwise hybrid attention.
+
+TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and bench.py's
+cpu_baseline / reference leg may import this module.  It shares no code with
+the CUDA library (sparse_kv_caching_b200) and never imports it; the only input
+both sides share is the seeded generator in `synth`, which holds none of the
+method's arithmetic.
+
+Source: "LoLA: Low-Rank Linear Attention With Sparse Caching" (McDermott,
+Heath, Parhi; arXiv 2505.23666v3), as restated by its close-reading notes
+(cc.laoqi.cc, LoLA reading notes): §2.2 (Eqs. 3-5, linear attention state),
+§2.3 (Eq. 10, Self-Recall Error), §2.4 (Fig. 1, Eqs. 11-13, candidate set,
+top-lambda retention, fold), §2.5 (Eq. 14, shared normaliser), §2.6 (Eq. 15,
+Fig. 2, chunkwise inference) and §2.7 (App. B memory count).
+
+Readings taken where the pages leave a step open (each is listed, with its
+reason, in the design notes of this repository):
+  R1  SRE is the squared L2 residual (the summaries' form); the ranking equals
+      that of the unsquared norm of §2.3.
+  R2  eta counts the exact pairs that precede the current block; the block's
+      own causal pairs are read in addition.  After the block is appended to
+      the window, the oldest pairs beyond eta leave it (the set L).
+  R3  Read first with the state entering the block, then update (§2.6: the
+      queries of a block share the existing state; scoring follows the block).
+      The per-token decode step is the same rule with a block of one token.
+  R4  With H = 0 and s = 0 (nothing folded yet) the memory recalls the zero
+      vector, so SRE = ||v||^2.  phi > 0, hence phi(k)^T s > 0 once anything
+      has been folded; no epsilon is added anywhere.
+  R5  Ties at the lambda-th score: exact cap of lambda, order (SRE descending,
+      position ascending): the older pair is kept.
+  R6  |E| <= lambda keeps every candidate: no scoring, no fold (§2.4).
+  R7  GQA: kv head floor(h / Gq) serves query head h; W, H, s, G and the window
+      are per kv head and the selection is shared by the head group.
+  R8  The output is Eq. 14 evaluated as written (no max-stabiliser: the fp64
+      exponent stays far from overflow for these inputs; this is asserted).
+
+Parity status of every function here: pinned by the tests in
+tests/test_oracle_pins.py (closed forms, reductions to textbook softmax
+attention and to the window+linear hybrid, brute-force state, exhaustive
+pairwise check of the selection, identical-key closed form, partition
+invariant, decode == one-token blocks, split calls == one call, and the
+printed App. B / Table 10 memory counts).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+TIE_REL = 1e-5   # relative band around the lambda-th SRE inside which swaps are valid
+
+
+# ---------------------------------------------------------------------------
+# Feature map (notes §2.1 notation table: learned phi: R^{d_k} -> R^D; the
+# Hedgehog form [softmax(xW), softmax(-xW)] is the fixed choice of this build)
+# ---------------------------------------------------------------------------
+def _softmax(z: np.ndarray) -> np.ndarray:
+    e = np.exp(z - z.max(axis=-1, keepdims=True))
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def feature_map(x: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """phi(x) = [softmax(x W), softmax(-x W)] in fp64; x [..., d], W [d, Dh] -> [..., 2 Dh]."""
+    z = np.asarray(x, np.float64) @ np.asarray(W, np.float64)
+    return np.concatenate([_softmax(z), _softmax(-z)], axis=-1)
+
+
+# ---------------------------------------------------------------------------
+# Memory count of App. B (notes §2.7): elements held per head after t tokens.
+# ---------------------------------------------------------------------------
+def state_elements(t: int, eta: int, lam: int, d_k: int, d_v: int, D: int) -> int:
+    """M_LoLA(t) = min{ t (d_k + d_v), (eta + lam)(d_k + d_v) + D d_v + D }."""
+    return min(t * (d_k + d_v), (eta + lam) * (d_k + d_v) + D * d_v + D)
+
+
+def full_elements(t: int, d_k: int, d_v: int) -> int:
+    """M_full(t) = t (d_k + d_v): the softmax KV cache of the same head."""
+    return t * (d_k + d_v)
+
+
+# ---------------------------------------------------------------------------
+# Self-Recall Error (notes §2.3, Eq. 10; squared per R1; zero state per R4)
+# ---------------------------------------------------------------------------
+def self_recall_error(phik: np.ndarray, v: np.ndarray, H: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """SRE(k, v | H, s) = || H^T phi(k) / (phi(k)^T s) - v ||^2 for each row.
+
+    phik [n, D], v [n, d], H [D, d], s [D] -> [n].  Where phi(k)^T s == 0 the
+    prediction is the zero vector (R4).
+    """
+    den = phik @ s
+    num = phik @ H
+    pred = np.zeros_like(num)
+    ok = den > 0
+    pred[ok] = num[ok] / den[ok, None]
+    r = pred - v
+    return (r * r).sum(axis=1)
+
+
+def top_lambda(E: list[int], sre: np.ndarray, lam: int) -> list[int]:
+    """Top_lambda of Eq. 11 with the exact cap and tie order of R5."""
+    order = sorted(range(len(E)), key=lambda i: (-sre[i], E[i]))
+    return sorted(E[i] for i in order[:lam])
+
+
+def valid_alternative(E: list[int], sre: np.ndarray, lam: int, keep: list[int],
+                      rel: float = TIE_REL) -> bool:
+    """True if `keep` is a top-lambda set of E under scores `sre` up to ties.
+
+    A set is valid when it has lambda distinct members of E, every kept score is
+    >= tau (1 - rel) and every dropped score is <= tau (1 + rel), tau being the
+    lambda-th largest score.  Only these sets count as correct results when the
+    lambda-th score is (nearly) tied.
+    """
+    ks = set(keep)
+    if len(ks) != lam or len(keep) != lam or not ks <= set(E):
+        return False
+    tau = float(np.sort(sre)[::-1][lam - 1])
+    band = rel * abs(tau)
+    for i, e in enumerate(E):
+        if e in ks and sre[i] < tau - band:
+            return False
+        if e not in ks and sre[i] > tau + band:
+            return False
+    return True
+
+
+class LolaStream:
+    """The three memories of one LoLA head stream: window W, sparse cache G, state (H, s).
+
+    One instance serves one (sequence, kv head) pair and its group of query
+    heads.  Every token ever seen is kept in a plain history so that positions
+    index it; the memories themselves hold positions only.
+    """
+
+    def __init__(self, W: np.ndarray, eta: int, lam: int):
+        self.W = np.asarray(W, np.float64)
+        self.d, self.Dh = self.W.shape
+        self.D = 2 * self.Dh
+        self.eta, self.lam = int(eta), int(lam)
+        self.K = np.zeros((0, self.d))
+        self.V = np.zeros((0, self.d))
+        self.phiK = np.zeros((0, self.D))
+        self.t = 0
+        self.window: list[int] = []     # W: positions, oldest first
+        self.cache: list[int] = []      # G: positions (sorted)
+        self.folded: list[int] = []     # F: positions absorbed into (H, s)
+        self.H = np.zeros((self.D, self.d))
+        self.s = np.zeros(self.D)
+        self.log: list[dict] = []
+
+    # -- history ----------------------------------------------------------
+    def _append(self, k: np.ndarray, v: np.ndarray) -> list[int]:
+        k = np.asarray(k, np.float64).reshape(-1, self.d)
+        v = np.asarray(v, np.float64).reshape(-1, self.d)
+        self.K = np.concatenate([self.K, k])
+        self.V = np.concatenate([self.V, v])
+        self.phiK = np.concatenate([self.phiK, feature_map(k, self.W)])
+        P = list(range(self.t, self.t + len(k)))
+        self.t += len(k)
+        return P
+
+    # -- read (Eq. 14 with the state entering the block; R3, R8) ----------
+    def _read(self, Q: np.ndarray, P: list[int], rows: np.ndarray | None) -> np.ndarray:
+        Gq, n, d = Q.shape
+        y = np.full((Gq, n, d), np.nan)
+        exact = self.cache + self.window           # G and W entering the block
+        Ke, Ve = self.K[exact], self.V[exact]
+        Kb, Vb = self.K[P], self.V[P]
+        causal = np.tril(np.ones((n, n)))          # block key j visible to query i iff j <= i
+        scale = 1.0 / np.sqrt(d)
+        for h in range(Gq):
+            sel = np.arange(n) if rows is None else np.nonzero(rows[h])[0]
+            if len(sel) == 0:
+                continue
+            q = np.asarray(Q[h, sel], np.float64)
+            le = (q @ Ke.T) * scale
+            lb = (q @ Kb.T) * scale
+            assert le.size == 0 or le.max() < 700.0
+            assert lb.max() < 700.0
+            ae = np.exp(le)
+            ab = np.exp(lb) * causal[sel]
+            phq = feature_map(q, self.W)
+            num = ae @ Ve + ab @ Vb + phq @ self.H
+            den = ae.sum(axis=1) + ab.sum(axis=1) + phq @ self.s
+            y[h, sel] = num / den[:, None]
+        return y
+
+    # -- one update interval (notes §2.4 and §2.6) -------------------------
+    def step(self, Q, K, V, rows=None, choose=None) -> np.ndarray:
+        """Process one block of new tokens: read, advance window, score, keep, fold.
+
+        Q [Gq, n, d], K/V [n, d].  `rows` (bool [Gq, n]) limits which outputs
+        are computed (others are NaN).  `choose(record)` may return another
+        retained set; it is adopted only if `valid_alternative` accepts it
+        under this oracle's own scores (tie handling, R5).
+        """
+        Q = np.asarray(Q, np.float64)
+        if Q.ndim == 2:
+            Q = Q[:, None, :]
+        P = self._append(K, V)
+        y = self._read(Q, P, rows)
+        # advance the window: the block enters, the oldest pairs beyond eta leave (R2)
+        self.window.extend(P)
+        n_leave = max(0, len(self.window) - self.eta)
+        L, self.window = self.window[:n_leave], self.window[n_leave:]
+        E = self.cache + L                          # candidate set E
+        rec = dict(t0=P[0], n=len(P), E=E, L=L, sre=None, keep=None, fold=[], adopted=False,
+                   cache_before=list(self.cache), window_after=list(self.window),
+                   folded_before=len(self.folded))
+        if len(E) <= self.lam:                      # R6
+            self.cache = sorted(E)
+        else:
+            sre = self_recall_error(self.phiK[E], self.V[E], self.H, self.s)   # pre-fold state
+            keep = top_lambda(E, sre, self.lam)
+            rec.update(sre=sre, keep=keep)
+            if choose is not None:
+                alt = choose(rec)
+                if alt is not None and sorted(alt) != keep:
+                    if not valid_alternative(E, sre, self.lam, list(alt)):
+                        raise ValueError("rejected retained set: not a top-lambda set up to ties")
+                    keep = sorted(alt)
+                    rec.update(keep=keep, adopted=True)
+            ks = set(keep)
+            S = [e for e in E if e not in ks]
+            self._fold(S)
+            self.cache = keep
+            rec["fold"] = S
+        self.log.append(rec)
+        return y
+
+    def _fold(self, S: list[int]) -> None:
+        """Eqs. 12-13: H += sum phi(k) v^T, s += sum phi(k) over the pairs S leaving E."""
+        self.H = self.H + self.phiK[S].T @ self.V[S]
+        self.s = self.s + self.phiK[S].sum(axis=0)
+        self.folded.extend(S)
+
+    def prefill(self, Q, K, V, chunk: int, rows=None, choose=None) -> np.ndarray:
+        """Chunkwise prefill (Eq. 15): blocks of `chunk` tokens, in order."""
+        Q = np.asarray(Q)
+        n = K.shape[0]
+        assert n % chunk == 0
+        out = []
+        for c0 in range(0, n, chunk):
+            r = None if rows is None else rows[:, c0:c0 + chunk]
+            out.append(self.step(Q[:, c0:c0 + chunk], K[c0:c0 + chunk], V[c0:c0 + chunk], r, choose))
+        return np.concatenate(out, axis=1)
+
+    def decode(self, q, k, v, choose=None) -> np.ndarray:
+        """Per-token decode step: one block of a single token (R3)."""
+        return self.step(np.asarray(q).reshape(-1, 1, self.d), k, v, None, choose)[:, 0]

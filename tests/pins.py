@@ -1,0 +1,222 @@
+"""Independent checks that pin the CPU oracle to what the LoLA pages fix.
+
+Each check recomputes its expectation from a closed form, a textbook routine
+or brute force; none reuses the oracle's loop.  They are plain functions so
+that tests/test_oracle_pins.py can run them on the oracle as written and on
+deliberately broken copies of it (planted mistakes must be caught).
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import synth
+
+
+def small(T=48, d=8, Dh=4, eta=8, lam=6, C=4, Gq=2, **kw):
+    """A tiny workload (fp32 values) built from the shared seeded generator."""
+    base = dict(B=1, Hq=Gq, Hkv=1, T=T, d=d, Dh=Dh, eta=eta, lam=lam, chunk=C, dtype="f32",
+                cluster_frac=0.5, n_clusters=3, cluster_std=0.05, n_needles=0,
+                needle_place="none", decode_steps=0, wid=101)
+    base.update(kw)
+    w = synth.Workload("pin-small", **base)
+    a = synth.stream_arrays(w, 0, 0)
+    W = synth.weights(w)[0]
+    return w, a, W
+
+
+def softmax_fm(x, W):
+    """phi via torch.softmax (a library routine), fp64."""
+    z = torch.from_numpy(np.asarray(x, np.float64) @ np.asarray(W, np.float64))
+    return torch.cat([torch.softmax(z, -1), torch.softmax(-z, -1)], -1).numpy()
+
+
+def run(Stream, w, a, W, C=None):
+    st = Stream(W, w.eta, w.lam)
+    y = st.prefill(a["q"], a["k"], a["v"], C or w.chunk)
+    return st, y
+
+
+# (b) eta + lambda >= T: nothing is ever folded and y is causal softmax attention
+def check_full_softmax(Stream, seed_kw=None) -> float:
+    w, a, W = small(T=40, eta=16, lam=24, C=8, **(seed_kw or {}))
+    st, y = run(Stream, w, a, W)
+    q, k, v = (np.asarray(a[x], np.float64) for x in "qkv")
+    ref = np.zeros_like(y)
+    for h in range(q.shape[0]):           # textbook loop
+        for t in range(w.T):
+            l = k[:t + 1] @ q[h, t] / np.sqrt(w.d)
+            p = np.exp(l - l.max())
+            ref[h, t] = (p / p.sum()) @ v[:t + 1]
+    sd = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k)[None].expand(q.shape[0], -1, -1),
+        torch.from_numpy(v)[None].expand(q.shape[0], -1, -1), is_causal=True).numpy()
+    assert np.abs(ref - sd).max() < 1e-12
+    assert len(st.folded) == 0
+    return float(np.abs(y - ref).max())
+
+
+# (a) lambda = 0: the sliding-window + linear-attention hybrid (LoLCATs) in kernel form
+def check_lambda0(Stream) -> float:
+    w, a, W = small(T=48, eta=8, lam=0, C=4)
+    st, y = run(Stream, w, a, W)
+    q, k, v = (np.asarray(a[x], np.float64) for x in "qkv")
+    pk = softmax_fm(k, W)
+    err = 0.0
+    for h in range(q.shape[0]):
+        pq = softmax_fm(q[h], W)
+        for t in range(w.T):
+            t0 = (t // w.chunk) * w.chunk
+            lo = max(0, t0 - w.eta)
+            e = np.exp(k[lo:t + 1] @ q[h, t] / np.sqrt(w.d))
+            kern = pk[:lo] @ pq[t]                    # phi(q)^T phi(k_i), i < t0 - eta
+            num = e @ v[lo:t + 1] + kern @ v[:lo]
+            den = e.sum() + kern.sum()
+            err = max(err, float(np.abs(y[h, t] - num / den).max()))
+    return err
+
+
+# (c) brute-force state and its closed-form sums
+def check_state(Stream) -> float:
+    w, a, W = small()
+    st, _ = run(Stream, w, a, W)
+    k, v = np.asarray(a["k"], np.float64), np.asarray(a["v"], np.float64)
+    F = st.folded
+    assert len(set(F)) == len(F)
+    H = np.zeros((2 * w.Dh, w.d))
+    s = np.zeros(2 * w.Dh)
+    for f in F:
+        p = softmax_fm(k[f:f + 1], W)[0]
+        H += np.outer(p, v[f])
+        s += p
+    e1 = np.abs(H - st.H).max()
+    e2 = abs(st.s.sum() - 2 * len(F))                       # each half of phi sums to 1
+    e3 = np.abs(st.H.sum(axis=0) - 2 * v[F].sum(axis=0)).max() if F else np.abs(st.H).max()
+    return float(max(e1, np.abs(s - st.s).max(), e2, e3))
+
+
+# (d) every retained set is the exhaustive top-lambda of E by an independently computed SRE
+def check_selection(Stream) -> int:
+    w, a, W = small(T=64, eta=8, lam=5, C=4)
+    st, _ = run(Stream, w, a, W)
+    k, v = np.asarray(a["k"], np.float64), np.asarray(a["v"], np.float64)
+    bad = 0
+    for rec in st.log:
+        if rec["sre"] is None:
+            continue
+        F = st.folded[:rec["folded_before"]]
+        D = 2 * w.Dh
+        H = np.zeros((D, w.d))
+        s = np.zeros(D)
+        for f in F:
+            p = softmax_fm(k[f:f + 1], W)[0]
+            H += np.outer(p, v[f])
+            s += p
+        sre = {}
+        for e in rec["E"]:
+            p = softmax_fm(k[e:e + 1], W)[0]
+            den = p @ s
+            pred = (p @ H) / den if den > 0 else np.zeros(w.d)
+            sre[e] = float(((pred - v[e]) ** 2).sum())
+        keep = set(rec["keep"])
+        drop = [e for e in rec["E"] if e not in keep]
+        if len(keep) != w.lam:
+            bad += 1
+        for i in keep:                       # pairwise: each kept beats each dropped
+            for j in drop:
+                if not (sre[i] > sre[j] or (sre[i] == sre[j] and i < j)):
+                    bad += 1
+        if sorted(drop) != sorted(rec["fold"]):
+            bad += 1
+    return bad
+
+
+# (e) identical keys: phi is the same for all, so pred is the mean of the folded values
+def check_identical_keys(Stream) -> float:
+    w, a, W = small(T=40, eta=4, lam=3, C=4)
+    k0 = a["k"][0].copy()
+    a = dict(a, k=np.tile(k0, (w.T, 1)))
+    st, y = run(Stream, w, a, W)
+    v = np.asarray(a["v"], np.float64)
+    q = np.asarray(a["q"], np.float64)
+    err = 0.0
+    for rec in st.log:
+        if rec["sre"] is None:
+            continue
+        F = st.folded[:rec["folded_before"]]
+        vbar = v[F].mean(axis=0) if F else np.zeros(w.d)
+        for i, e in enumerate(rec["E"]):
+            err = max(err, abs(rec["sre"][i] - ((vbar - v[e]) ** 2).sum()))
+    # output closed form: one logit per query, one kernel value per query
+    pk = softmax_fm(k0[None], W)[0]
+    for rec in st.log:
+        t0 = rec["t0"]
+        exact = rec["cache_before"] + [p for p in range(max(0, t0 - w.eta), t0)]
+        F = st.folded[:rec["folded_before"]]
+        for h in range(q.shape[0]):
+            for t in range(t0, t0 + rec["n"]):
+                ex = exact + list(range(t0, t + 1))
+                ea = np.exp(q[h, t] @ k0 / np.sqrt(w.d))
+                c = softmax_fm(q[h, t][None], W)[0] @ pk
+                ref = (ea * v[ex].sum(0) + c * v[F].sum(0)) / (ea * len(ex) + c * len(F))
+                err = max(err, float(np.abs(ref - y[h, t]).max()))
+    return err
+
+
+# (f) partition: every past position lives in exactly one of G, W, F
+def check_partition(Stream) -> int:
+    w, a, W = small(T=64, eta=8, lam=5, C=4)
+    st = Stream(W, w.eta, w.lam)
+    bad = 0
+    for c0 in range(0, w.T, w.chunk):
+        sl = slice(c0, c0 + w.chunk)
+        st.step(a["q"][:, sl], a["k"][sl], a["v"][sl])
+        t = c0 + w.chunk
+        G, Wn, F = st.cache, st.window, st.folded
+        allp = sorted(G + Wn + F)
+        if allp != list(range(t)):
+            bad += 1
+        if Wn != list(range(max(0, t - w.eta), t)):
+            bad += 1
+        if len(G) != min(w.lam, max(0, t - w.eta)):
+            bad += 1
+    return bad
+
+
+# (g) API identities: split calls == one call; decode == blocks of one token
+def check_identities(Stream) -> float:
+    w, a, W = small(T=48, eta=8, lam=5, C=4)
+    st1, y1 = run(Stream, w, a, W)
+    st2 = Stream(W, w.eta, w.lam)
+    y2a = st2.prefill(a["q"][:, :20], a["k"][:20], a["v"][:20], 4)
+    y2b = st2.prefill(a["q"][:, 20:], a["k"][20:], a["v"][20:], 4)
+    e = np.abs(np.concatenate([y2a, y2b], 1) - y1).max()
+    e = max(e, np.abs(st1.H - st2.H).max())
+    st3, y3 = run(Stream, w, a, W, C=1)
+    st4 = Stream(W, w.eta, w.lam)
+    y4 = np.stack([st4.decode(a["q"][:, t], a["k"][t], a["v"][t]) for t in range(w.T)], 1)
+    e = max(e, np.abs(y3 - y4).max(), np.abs(st3.H - st4.H).max())
+    if st3.cache != st4.cache or st1.cache != st2.cache:
+        e = np.inf
+    return float(e)
+
+
+# SRE closed forms: empty state recalls zero; one folded pair recalls its own value
+def check_sre_closed_form(sre_fn) -> float:
+    rng = np.random.default_rng(7)
+    D, d = 6, 5
+    phi = rng.random((4, D)) + 0.1
+    v = rng.standard_normal((4, d))
+    e = np.abs(sre_fn(phi, v, np.zeros((D, d)), np.zeros(D)) - (v * v).sum(1)).max()
+    pf, vf = rng.random(D) + 0.1, rng.standard_normal(d)
+    got = sre_fn(phi, v, np.outer(pf, vf), pf)
+    return float(max(e, np.abs(got - ((v - vf) ** 2).sum(1)).max()))
+
+
+# R5 tie order on exact ties: the older position is kept, the cap is exact
+def check_tie_order(top_fn) -> int:
+    cases = [([7, 3, 5], [2.0, 2.0, 2.0], 1, [3]),
+             ([7, 3, 5], [2.0, 2.0, 2.0], 2, [3, 5]),
+             ([1, 2, 3, 4], [1.0, 3.0, 3.0, 0.0], 1, [2]),
+             ([9, 4, 6, 2], [5.0, 1.0, 5.0, 1.0], 3, [2, 6, 9])]
+    return sum(sorted(top_fn(E, np.array(s), lam)) != want for E, s, lam, want in cases)
