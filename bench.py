@@ -1,0 +1,499 @@
+#!/usr/bin/env python
+"""Throughput of the LoLA chunkwise hybrid-attention layer on B200: one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lola|reference]
+                    [--workload 2] [--no-decode]
+
+A step is one pass of the whole layer over one batch of synthetic input:
+reset the memories, then chunkwise prefill of B x T tokens (window advance,
+SRE scoring, top-lambda retention, fold and the hybrid output of every
+chunk).  The default workload is the Llama-3.1-8B-shaped 4K prefill (32 q /
+8 kv heads, d = 128, phi dim 128, eta = lambda = 256, chunk 64, bf16 inputs).
+The line also carries the per-token decode throughput of the 8B-shaped decode
+workload (B = 64 after a 4096-token prefill) under "decode".
+
+Multi-GPU: one process per GPU; every rank runs its own copy of the workload
+(the path shards into independent (sequence, kv head) streams and needs no
+collective), timing is the max over ranks, value = all ranks' tokens / time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "prefill tokens/s and decode tokens/s at 1 B200; % of roofline; oracle match"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work (counts only what the method must compute or move)
+# ---------------------------------------------------------------------------
+def prefill_work(w: synth.Workload) -> dict:
+    """FLOPs and bytes per prefill launch of each kernel class."""
+    B, T, Hq, Hkv, d, Dh, D, C = w.B, w.T, w.Hq, w.Hkv, w.d, w.Dh, w.D, w.chunk
+    e = 2 if w.dtype == "bf16" else 4
+    att = lin = 0
+    scan_fl = 0
+    n_fold = 0
+    for c in range(T // C):
+        t0 = c * C
+        n_g = min(w.lam, max(0, t0 - w.eta))
+        n_w = min(w.eta, t0)
+        # causal chunk: query i sees i + 1 block keys
+        keys = C * (n_g + n_w) + C * (C + 1) // 2
+        att += 4 * d * keys
+        lin += C * (2 * D * d + 2 * D + 2 * d * Dh)
+        n_l = max(0, t0 + C - w.eta) - max(0, t0 - w.eta)
+        if n_l and n_g + n_l > w.lam:
+            n = n_g + n_l
+            f = n - w.lam
+            scan_fl += 2 * n * D * d + 2 * n * D + 3 * n * d + 2 * f * D * d + f * D
+            n_fold += f
+    out_fl = B * Hq * (att + lin)
+    return {
+        "phi": dict(flops=2 * B * T * Hkv * d * Dh,
+                    bytes=B * T * Hkv * d * e + Hkv * d * Dh * e + B * T * Hkv * D * 4),
+        "scan": dict(flops=B * Hkv * scan_fl, bytes=B * Hkv * 2 * D * d * 4),
+        "output": dict(flops=out_fl, bytes=B * T * Hq * d * (e + 4) + 2 * B * T * Hkv * d * e),
+        "total_flops": B * Hkv * scan_fl + out_fl + 2 * B * T * Hkv * d * Dh,
+    }
+
+
+def decode_step_bytes(w: synth.Workload) -> int:
+    """HBM bytes one decode step must move (all streams, steady state)."""
+    e = 2 if w.dtype == "bf16" else 4
+    d, D = w.d, w.D
+    rd = D * d * 4 + D * 4 + w.lam * 2 * d * e + w.eta * 2 * d * e + (w.Gq + 2) * d * e
+    wr = D * d * 4 + D * 4 + w.Gq * d * 4 + 2 * 2 * d * e + 2 * 4
+    return w.B * w.Hkv * (rd + wr)
+
+
+def decode_step_flops(w: synth.Workload) -> int:
+    d, D, n = w.d, w.D, w.lam + 1
+    keys = w.lam + w.eta + 1
+    per = (w.Gq * (4 * d * keys + 2 * D * d + 2 * d * w.Dh) + 2 * n * D * d + 2 * D * d + 2 * d * w.Dh)
+    return w.B * w.Hkv * per
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "sparse_kv_caching_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernels."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        ent = t.get(f"{kernel}@{workload}")
+        if ent and ent.get("source_hash") == kernel_source_hash():
+            return ent["dram_bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.gpu_id:
+                cmd += ["-i", self.gpu_id]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict | None:
+        if not self.proc:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(w: synth.Workload, streams, budget_s: float, gpu=None):
+    """Run the CPU oracle over whole streams until `budget_s` is spent.
+
+    Returns (tokens_equivalent, seconds, streams_done, match) where a stream of
+    T tokens counts as T / Hkv layer tokens (a token spans Hkv streams).  With
+    `gpu` = (y [B,T,Hq,d] tensor, trace [S, chunks+1, lambda]) the oracle follows
+    the library's retained sets up to ties and reports the match.
+    """
+    from oracle import LolaStream, valid_alternative
+    done = 0
+    secs = 0.0
+    match = dict(streams=0, hard_mismatch=0, tie_swaps=0, max_rel_err_y=0.0, rows_checked=0)
+    for (b, g) in streams:
+        a = synth.stream_arrays(w, b, g)
+        Wg = synth.weights(w)[g]
+        t0 = time.perf_counter()
+        st = LolaStream(Wg, w.eta, w.lam)
+        exp = {}
+        stats = dict(hard=0, ties=0)
+
+        def choose(rec):
+            gset = exp.get(rec["t0"])
+            if gset is None or gset == rec["keep"]:
+                return None
+            if valid_alternative(rec["E"], rec["sre"], w.lam, gset):
+                stats["ties"] += 1
+                return gset
+            stats["hard"] += 1
+            return None
+
+        if gpu is not None and w.lam > 0:
+            tr = gpu[1][b * w.Hkv + g]
+            for ci in range(w.T // w.chunk):
+                exp[ci * w.chunk] = sorted(int(p) for p in tr[ci + 1] if p >= 0)
+        y = st.prefill(a["q"][:, :w.T], a["k"][:w.T], a["v"][:w.T], w.chunk,
+                       choose=choose if gpu is not None else None)
+        secs += time.perf_counter() - t0
+        done += 1
+        if gpu is not None:
+            yg = gpu[0][b, :, g * w.Gq:(g + 1) * w.Gq, :].permute(1, 0, 2).double().cpu().numpy()
+            err = float(np.abs(yg - y).max() / np.abs(y).max())
+            match["streams"] += 1
+            match["hard_mismatch"] += stats["hard"]
+            match["tie_swaps"] += stats["ties"]
+            match["max_rel_err_y"] = max(match["max_rel_err_y"], err)
+            match["rows_checked"] += y.shape[0] * y.shape[1]
+        if secs >= budget_s:
+            break
+    return done * w.T / w.Hkv, secs, done, match
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+def run_reference(args, w, rank):
+    if rank != 0:
+        return 0
+    streams = [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    times = []
+    toks = []
+    for i in range(args.warmup + args.steps):
+        s = [streams[i % len(streams)]]
+        n, secs, _, _ = oracle_sample(w, s, budget_s=0.0)
+        if i >= args.warmup:
+            times.append(secs)
+            toks.append(n)
+    value = sum(toks) / sum(times)
+    cores = blas_threads()
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                       "phi_dim": w.D, "eta": w.eta, "lambda": w.lam, "chunk": w.chunk},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"one (sequence, kv head) stream of {w.T} tokens per step "
+                                       f"(= {w.T / w.Hkv:.0f} layer tokens)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="lola", choices=["lola", "reference"])
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work (cpu_baseline)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = synth.workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w, rank)
+
+    import torch
+    import torch.distributed as dist
+    import sparse_kv_caching_b200 as lola
+    from datetime import timedelta
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+
+    def to_dev(x):
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(x).to(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks, peaks_kind = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    gpu_uuid = None
+    try:
+        gpu_uuid = "GPU-" + str(props.uuid)
+    except Exception:
+        pass
+
+    # ---- prefill workload -------------------------------------------------
+    full = synth.full_arrays(w)
+    q, k, v, W = (to_dev(full[x]) for x in ("q", "k", "v", "W"))
+    cfg = lola.make_config(w.B, w.Hq, w.Hkv, w.d, w.Dh, w.eta, w.lam, w.chunk, w.dtype, w.T)
+    layer = lola.LolaLayer(cfg, W, device=dev)
+    y = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)   # > L2 (126 MB)
+
+    def step():
+        layer.reset()
+        layer.prefill(q, k, v, y)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    clocks = ClockSampler(gpu_uuid)
+    clocks.start()
+    layer.profile(True)
+    launches0 = lola.launch_count()
+    total_ms = 0.0
+    stream = torch.cuda.current_stream()
+    for _ in range(args.steps):
+        flush.zero_()
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        step()
+        ev1.record(stream)
+        ev1.synchronize()
+        total_ms += ev0.elapsed_time(ev1)
+    barrier()
+    launches = lola.launch_count() - launches0
+    prof = layer.profile_read()
+    layer.profile(False)
+    clk = clocks.stop()
+    ms_step = max_over_ranks(total_ms / args.steps)
+    tokens = w.B * w.T * world
+    value = tokens / (ms_step / 1e3)
+
+    work = prefill_work(w)
+    # dominant kernel by measured time
+    dom = max(("phi", "scan", "output"), key=lambda kk: prof[kk][0])
+    dom_ms = prof[dom][0] / max(1, prof[dom][1])
+    fl = work[dom]["flops"]
+    achieved = fl / (dom_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"]
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
+                "traffic": traffic_for(dom, w.name),
+                "flops_per_launch": fl, "ms_per_launch": dom_ms}
+    shares = {kk: round(prof[kk][0] / max(1e-9, sum(p[0] for p in prof.values())), 4) for kk in prof}
+    layer_roof_ms = max(work["total_flops"] / (peak * 1e12), 0.0) * 1e3
+    # ---- e2e through the host-buffer entry point ------------------------------
+    hq, hk, hv = (torch.from_numpy(full[x].view(np.int16) if full[x].dtype == np.uint16 else full[x])
+                  .pin_memory() for x in ("q", "k", "v"))
+    if w.dtype == "bf16":
+        hq, hk, hv = (x.view(torch.bfloat16) for x in (hq, hk, hv))
+    hy = torch.empty((w.B, w.T, w.Hq, w.d), dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 5))
+    for _ in range(2):
+        layer.reset()
+        layer.prefill_host(hq, hk, hv, hy)
+    barrier()
+    e2e_ms = 0.0
+    for _ in range(e2e_steps):
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        layer.reset()
+        layer.prefill_host(hq, hk, hv, hy)
+        ev1.record(stream)
+        ev1.synchronize()
+        e2e_ms += ev0.elapsed_time(ev1)
+    e2e_ms = max_over_ranks(e2e_ms / e2e_steps)
+    h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
+    d2h = hy.numel() * 4
+    # y and trace of the last device-path step, for the oracle match
+    layer.reset()
+    layer.prefill(q, k, v, y)
+    torch.cuda.synchronize()
+    ex = layer.export()
+    trace = ex["trace_pos"].cpu().numpy() if w.lam > 0 else None
+    y_host = y.cpu()
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d,
+                       "phi_dim": w.D, "eta": w.eta, "lambda": w.lam, "chunk": w.chunk,
+                       "input_dtype": w.dtype, "l2": "flushed between timed steps (256 MB write)",
+                       "parallelism": f"replicas x{world} (independent streams)"},
+            "roofline": roofline,
+            "layer_roofline": {"flops": work["total_flops"], "ms_at_peak": layer_roof_ms,
+                               "frac": layer_roof_ms / ms_step},
+            "kernel_time_share": shares,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            }
+    del layer, full, q, k, v, y, hq, hk, hv, hy
+    torch.cuda.empty_cache()
+
+    # ---- decode workload ----------------------------------------------------
+    if not args.no_decode:
+        wd = synth.workload(4)
+        fd = synth.full_arrays(wd)
+        qd, kd, vd, Wd = (to_dev(fd[x]) for x in ("q", "k", "v", "W"))
+        del fd
+        cfgd = lola.make_config(wd.B, wd.Hq, wd.Hkv, wd.d, wd.Dh, wd.eta, wd.lam, wd.chunk, wd.dtype, wd.T)
+        ld = lola.LolaLayer(cfgd, Wd, device=dev)
+        ld.prefill(qd[:, :wd.T].contiguous(), kd[:, :wd.T].contiguous(), vd[:, :wd.T].contiguous())
+        steps_d = min(200, wd.decode_steps - args.warmup)
+        qs = [qd[:, t].contiguous() for t in range(wd.T, wd.T + args.warmup + steps_d)]
+        ks = [kd[:, t].contiguous() for t in range(wd.T, wd.T + args.warmup + steps_d)]
+        vs = [vd[:, t].contiguous() for t in range(wd.T, wd.T + args.warmup + steps_d)]
+        yd = torch.empty((wd.B, wd.Hq, wd.d), dtype=torch.float32, device=dev)
+        for i in range(args.warmup):
+            ld.decode(qs[i], ks[i], vs[i], yd)
+        barrier()
+        ld.profile(True)
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for i in range(args.warmup, args.warmup + steps_d):
+            ld.decode(qs[i], ks[i], vs[i], yd)
+        ev1.record(stream)
+        ev1.synchronize()
+        dms = max_over_ranks(ev0.elapsed_time(ev1) / steps_d)
+        pd = ld.profile_read()
+        kms = pd["decode"][0] / max(1, pd["decode"][1])
+        by = decode_step_bytes(wd)
+        line["decode"] = {
+            "workload": wd.name, "value": wd.B * world / (dms / 1e3), "unit": "tokens/s", "ms_per_step": dms,
+            "steps": steps_d, "B": wd.B, "context": f"{wd.T} prefilled + up to {steps_d} decoded",
+            "roofline": {"bound": "hbm", "kernel": "decode", "achieved": by / (kms / 1e3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": by / (kms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                         "bytes_per_launch": by, "ms_per_launch": kms,
+                         "peak_kind": f"{peaks_kind} HBM copy", "traffic": traffic_for("decode", wd.name)},
+            "flops_per_step": decode_step_flops(wd)}
+        del ld, qd, kd, vd, qs, ks, vs
+        torch.cuda.empty_cache()
+
+    # ---- cpu_baseline: the oracle on a bounded sample, plus the oracle match ----
+    if rank == 0:
+        streams = [(0, 0), (w.B - 1, w.Hkv - 1)] + [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+        seen = []
+        for s in streams:
+            if s not in seen:
+                seen.append(s)
+        n, secs, done, match = oracle_sample(w, seen, args.cpu_budget, gpu=(y_host, trace))
+        line["cpu_baseline"] = {"value": n / secs, "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{done} whole (sequence, kv head) streams of {w.T} tokens "
+                                          f"(= {n:.0f} layer tokens), {secs:.1f} s",
+                                "oracle_match": match}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

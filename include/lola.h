@@ -1,0 +1,168 @@
+/*
+ * lola.h - C ABI of the B200 (sm_100a) LoLA hybrid-attention layer.
+ *
+ * The layer is the inference step of "LoLA: Low-Rank Linear Attention With
+ * Sparse Caching" (arXiv 2505.23666v3) as its close-reading notes describe
+ * it: every query reads a sliding window W of the eta most recent KV pairs,
+ * a sparse global cache G of at most lambda raw KV pairs and a linear state
+ * (H, s), under one shared softmax normaliser (notes §2.5, Eq. 14).  After
+ * each block of tokens the pairs leaving the window and the cache members
+ * are scored by Self-Recall Error against the state (notes §2.3, Eq. 10), the
+ * lambda highest are kept in G and the rest are folded into (H, s)
+ * (notes §2.4, Eqs. 11-13).  Prefill runs this chunk by chunk (notes §2.6,
+ * Eq. 15, Fig. 2); decode runs it one token at a time (notes §2.4, Fig. 1).
+ *
+ * Conventions (all entry points):
+ *   - Every pointer named "device" is CUDA device memory on the current
+ *     device; "host" pointers are page-locked (pinned) host memory.
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  All work is enqueued asynchronously on it, in stream order.
+ *   - The caller owns every buffer.  The library allocates no device memory:
+ *     persistent state and per-call scratch live in the caller's `dev_buf`,
+ *     sized by lola_state_bytes().  The library owns only the small host
+ *     handle returned by lola_state_init().
+ *   - Return value 0 = LOLA_OK; a negative value is one of the LOLA_ERR_*
+ *     codes below and lola_last_error_string() describes it (thread-local).
+ *     No entry point aborts the process or traps on the device.
+ *   - Feature map phi(x) = [softmax(x W_g), softmax(-x W_g)] (Hedgehog form,
+ *     fixed by this library; the pages leave phi as "learned"), D = 2 Dh.
+ *   - Sequences of a batch advance in lock step: every call processes the
+ *     same number of tokens for all B sequences.
+ *
+ * Layouts (row-major, contiguous):
+ *   q  [B][T][Hq][d], k and v [B][T][Hkv][d]   in `dtype`
+ *   y  [B][T][Hq][d]                            float32
+ *   W  [Hkv][d][Dh]                             in `dtype`
+ *   Query head h reads kv head h / (Hq / Hkv) (grouped-query attention).
+ */
+#ifndef LOLA_H
+#define LOLA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LOLA_OK                 0
+#define LOLA_ERR_INVALID_ARG   (-1)  /* null pointer, bad size, T % chunk != 0, ...    */
+#define LOLA_ERR_BUF_TOO_SMALL (-2)  /* dev_buf smaller than lola_state_bytes()         */
+#define LOLA_ERR_CUDA          (-3)  /* a CUDA call or kernel launch failed             */
+#define LOLA_ERR_TIMEOUT       (-4)  /* a bounded device-side wait gave up              */
+#define LOLA_ERR_UNSUPPORTED   (-5)  /* shape outside the compiled kernel variants      */
+
+#define LOLA_DTYPE_F32  0
+#define LOLA_DTYPE_BF16 1
+
+/* Shape and budget of one layer.  Supported: d in {64, 128}, Dh in {32, 64},
+ * 1 <= Hq / Hkv <= 8 and Hq % Hkv == 0, eta >= 1, 0 <= lambda <= 2048,
+ * 1 <= chunk <= 256, max_tokens % chunk == 0. */
+typedef struct lola_config {
+    int B;           /* sequences in the batch                                   */
+    int Hq;          /* query heads                                              */
+    int Hkv;         /* key/value heads                                          */
+    int d;           /* head dimension (d_k = d_v)                               */
+    int Dh;          /* feature-map half width; D = 2 Dh                         */
+    int eta;         /* sliding-window size: exact pairs preceding a block       */
+    int lambda;      /* sparse-cache capacity                                    */
+    int chunk;       /* prefill block length C                                   */
+    int dtype;       /* LOLA_DTYPE_F32 or LOLA_DTYPE_BF16 (q, k, v, W)           */
+    int max_tokens;  /* largest T of one lola_prefill_chunked call (sizes scratch) */
+} lola_config;
+
+typedef struct lola_state lola_state;   /* opaque host handle */
+
+/* Device views of the state (for checks and checkpoints).  Slot layouts:
+ *   H [B*Hkv][D][d] f32, s [B*Hkv][D] f32,
+ *   cache_k / cache_v [B*Hkv][lambda][d] dtype, cache_phik [B*Hkv][lambda][D] f32,
+ *   cache_pos [B*Hkv][lambda] int32 (-1 = empty slot),
+ *   win_k / win_v [B*Hkv][eta][d] dtype, win_phik [B*Hkv][eta][D] f32; the pair at
+ *   position p sits in window slot p % eta.
+ *   trace_pos: for stream i, trace_pos + i*trace_stride holds [trace_len][lambda]
+ *   int32: the cache positions (by slot) entering each chunk of the last
+ *   lola_prefill_chunked call, then the final set (trace_len = chunks + 1);
+ *   trace_t0 is the first position of that call. */
+typedef struct lola_state_view {
+    long long t;            /* tokens processed per sequence                  */
+    int n_cache;            /* occupied cache slots (slots 0 .. n_cache-1)   */
+    float* H;
+    float* s;
+    void* cache_k;
+    void* cache_v;
+    float* cache_phik;
+    int* cache_pos;
+    void* win_k;
+    void* win_v;
+    float* win_phik;
+    int* trace_pos;
+    int trace_len;          /* chunks of the last prefill call + 1 (0 if none)    */
+    int trace_stride;       /* ints between the traces of consecutive streams     */
+    long long trace_t0;
+} lola_state_view;
+
+/* Bytes of device memory one layer state needs (persistent state, prefill
+ * scratch and host-I/O staging).  Returns LOLA_ERR_INVALID_ARG or
+ * LOLA_ERR_UNSUPPORTED for a configuration outside the limits above. */
+int lola_state_bytes(const lola_config* cfg, size_t* bytes);
+
+/* Bind a state to `dev_buf` (device, >= lola_state_bytes bytes, 256-byte
+ * aligned), copy W (device, [Hkv][d][Dh] in dtype) into it and clear the
+ * memories (t = 0, empty window and cache, H = 0, s = 0).  Enqueued on
+ * `stream`; *out receives a new host handle.  Memories: notes §2.4, Fig. 1. */
+int lola_state_init(const lola_config* cfg, const void* W, void* dev_buf, size_t bytes,
+                    void* stream, lola_state** out);
+
+/* Clear the memories again (t = 0) without touching W.  Enqueued on stream. */
+int lola_state_reset(lola_state* st, void* stream);
+
+/* Release the host handle.  The caller still owns (and frees) dev_buf. */
+int lola_state_free(lola_state* st);
+
+/* Chunkwise prefill (notes §2.6, Eq. 15): process T new tokens of every
+ * sequence in blocks of `chunk`.  For each block, every query reads the
+ * state entering the block (Eq. 14); then the window advances, the leaving
+ * pairs and the cache are scored by SRE (Eq. 10), the top lambda stay
+ * cached (older position wins exact ties) and the rest are folded (Eqs.
+ * 12-13).  q, k, v: device, layouts above; y: device float32 [B][T][Hq][d].
+ * T must be a positive multiple of chunk and <= max_tokens.  Calls may split
+ * a sequence at any chunk-aligned point; the result equals one call. */
+int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const void* v,
+                         int T, float* y, void* stream);
+
+/* One decode step (notes §2.4, Fig. 1; a block of one token): q [B][Hq][d],
+ * k and v [B][Hkv][d] (device, dtype); y [B][Hq][d] float32 (device). */
+int lola_decode_step(lola_state* st, const void* q, const void* k, const void* v,
+                     float* y, void* stream);
+
+/* Same as lola_prefill_chunked / lola_decode_step, with pinned HOST buffers:
+ * the inputs are copied into device staging inside dev_buf, the layer runs,
+ * and y is copied back, all enqueued on `stream` (synchronise before reading y). */
+int lola_prefill_chunked_host(lola_state* st, const void* q, const void* k, const void* v,
+                              int T, float* y, void* stream);
+int lola_decode_step_host(lola_state* st, const void* q, const void* k, const void* v,
+                          float* y, void* stream);
+
+/* Fill *out with device views of the state (no copy, no synchronisation). */
+int lola_state_export(const lola_state* st, lola_state_view* out);
+
+/* Tracing aid.  Kernel classes, in this order: 0 feature map, 1 scan (memory
+ * update chain), 2 output, 3 finalize, 4 decode.  While enabled, every kernel
+ * launch of `st` is bracketed by CUDA events recorded on its stream.
+ * lola_profile_read waits for those events, adds their elapsed times (ms) and
+ * launch counts into ms[0..4] and launches[0..4] (n >= 5 entries each) and
+ * forgets them.  Enabling does not change what the kernels compute. */
+#define LOLA_KERNEL_CLASSES 5
+int lola_profile_enable(lola_state* st, int on);
+int lola_profile_read(lola_state* st, float* ms, long long* launches, int n);
+
+/* Number of kernels this library has launched in this process. */
+long long lola_launch_count(void);
+
+/* Text of the last error raised on this host thread ("" if none). */
+const char* lola_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOLA_H */

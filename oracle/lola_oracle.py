@@ -135,9 +135,9 @@ class LolaStream:
         self.d, self.Dh = self.W.shape
         self.D = 2 * self.Dh
         self.eta, self.lam = int(eta), int(lam)
-        self.K = np.zeros((0, self.d))
-        self.V = np.zeros((0, self.d))
-        self.phiK = np.zeros((0, self.D))
+        self._K = np.zeros((0, self.d))
+        self._V = np.zeros((0, self.d))
+        self._phiK = np.zeros((0, self.D))
         self.t = 0
         self.window: list[int] = []     # W: positions, oldest first
         self.cache: list[int] = []      # G: positions (sorted)
@@ -146,15 +146,34 @@ class LolaStream:
         self.s = np.zeros(self.D)
         self.log: list[dict] = []
 
-    # -- history ----------------------------------------------------------
+    # -- history (positions 0 .. t-1; storage grows geometrically) -------
+    @property
+    def K(self) -> np.ndarray:
+        return self._K[:self.t]
+
+    @property
+    def V(self) -> np.ndarray:
+        return self._V[:self.t]
+
+    @property
+    def phiK(self) -> np.ndarray:
+        return self._phiK[:self.t]
+
     def _append(self, k: np.ndarray, v: np.ndarray) -> list[int]:
         k = np.asarray(k, np.float64).reshape(-1, self.d)
         v = np.asarray(v, np.float64).reshape(-1, self.d)
-        self.K = np.concatenate([self.K, k])
-        self.V = np.concatenate([self.V, v])
-        self.phiK = np.concatenate([self.phiK, feature_map(k, self.W)])
-        P = list(range(self.t, self.t + len(k)))
-        self.t += len(k)
+        n = len(k)
+        if self.t + n > len(self._K):
+            cap = max(self.t + n, 2 * len(self._K), 64)
+            for name, width in (("_K", self.d), ("_V", self.d), ("_phiK", self.D)):
+                grown = np.zeros((cap, width))
+                grown[:self.t] = getattr(self, name)[:self.t]
+                setattr(self, name, grown)
+        self._K[self.t:self.t + n] = k
+        self._V[self.t:self.t + n] = v
+        self._phiK[self.t:self.t + n] = feature_map(k, self.W)
+        P = list(range(self.t, self.t + n))
+        self.t += n
         return P
 
     # -- read (Eq. 14 with the state entering the block; R3, R8) ----------

@@ -1,0 +1,365 @@
+// C ABI of the LoLA layer (declared in include/lola.h): argument checks,
+// the layout of the caller's device buffer, and the kernel sequence of each
+// call.  No device allocation happens here; every byte lives in dev_buf.
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <atomic>
+#include <string>
+#include <vector>
+
+#include "lola.h"
+#include "lola_internal.h"
+
+namespace lola {
+size_t decode_smem_bytes(const Dims& dm);
+}
+
+struct lola_prof_mark {
+    int cls;
+    cudaEvent_t a, b;
+};
+
+struct lola_state {
+    lola_config cfg;
+    lola::Dims dm;
+    lola::Layout L;
+    char* base;
+    size_t bytes;
+    long long t;
+    int last_nc;
+    long long last_t0;
+    bool prof = false;
+    std::vector<lola_prof_mark> marks;
+    std::vector<cudaEvent_t> pool;
+};
+
+namespace {
+
+thread_local std::string g_err;
+std::atomic<long long> g_launches{0};
+
+cudaEvent_t take_event(lola_state* st) {
+    if (!st->pool.empty()) { cudaEvent_t e = st->pool.back(); st->pool.pop_back(); return e; }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+// Run one launcher; count its kernels and, when profiling, bracket it with events.
+template <typename F>
+cudaError_t traced(lola_state* st, int cls, int kernels, cudaStream_t s, F&& launch) {
+    cudaEvent_t a = nullptr, b = nullptr;
+    if (st->prof) { a = take_event(st); b = take_event(st); if (a) cudaEventRecord(a, s); }
+    cudaError_t e = launch();
+    if (e == cudaSuccess) g_launches += kernels;
+    if (st->prof && a && b) {
+        cudaEventRecord(b, s);
+        st->marks.push_back({cls, a, b});
+    }
+    return e;
+}
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_err = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    return fail(LOLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxSmem = 227 * 1024;
+
+int make_dims(const lola_config* c, lola::Dims* dm) {
+    if (!c) return fail(LOLA_ERR_INVALID_ARG, "null config");
+    if (c->B < 1 || c->Hq < 1 || c->Hkv < 1 || c->Hq % c->Hkv)
+        return fail(LOLA_ERR_INVALID_ARG, "bad heads/batch: B=%d Hq=%d Hkv=%d", c->B, c->Hq, c->Hkv);
+    if (c->Hq / c->Hkv > 8) return fail(LOLA_ERR_UNSUPPORTED, "Hq/Hkv=%d > 8", c->Hq / c->Hkv);
+    if (c->d != 64 && c->d != 128) return fail(LOLA_ERR_UNSUPPORTED, "d=%d (64 or 128)", c->d);
+    if (c->Dh != 32 && c->Dh != 64) return fail(LOLA_ERR_UNSUPPORTED, "Dh=%d (32 or 64)", c->Dh);
+    if (c->eta < 1) return fail(LOLA_ERR_INVALID_ARG, "eta=%d < 1", c->eta);
+    if (c->lambda < 0 || c->lambda > 2048) return fail(LOLA_ERR_UNSUPPORTED, "lambda=%d (0..2048)", c->lambda);
+    if (c->chunk < 1 || c->chunk > 256) return fail(LOLA_ERR_UNSUPPORTED, "chunk=%d (1..256)", c->chunk);
+    if (c->max_tokens < c->chunk || c->max_tokens % c->chunk)
+        return fail(LOLA_ERR_INVALID_ARG, "max_tokens=%d must be a positive multiple of chunk=%d",
+                    c->max_tokens, c->chunk);
+    if (c->dtype != LOLA_DTYPE_F32 && c->dtype != LOLA_DTYPE_BF16)
+        return fail(LOLA_ERR_INVALID_ARG, "dtype=%d", c->dtype);
+    dm->B = c->B; dm->Hq = c->Hq; dm->Hkv = c->Hkv; dm->Gq = c->Hq / c->Hkv;
+    dm->d = c->d; dm->Dh = c->Dh; dm->D = 2 * c->Dh;
+    dm->eta = c->eta; dm->lam = c->lambda; dm->C = c->chunk; dm->dtype = c->dtype;
+    dm->S = c->B * c->Hkv; dm->max_tokens = c->max_tokens; dm->nc_max = c->max_tokens / c->chunk;
+    dm->esize = c->dtype == LOLA_DTYPE_BF16 ? 2 : 4;
+    if (lola::scan_smem_bytes(*dm) > (size_t)kMaxSmem)
+        return fail(LOLA_ERR_UNSUPPORTED, "lambda + chunk too large for the scan kernel's shared memory");
+    if (lola::decode_smem_bytes(*dm) > (size_t)kMaxSmem)
+        return fail(LOLA_ERR_UNSUPPORTED, "lambda + eta too large for the decode kernel's shared memory");
+    return LOLA_OK;
+}
+
+lola::Layout make_layout(const lola::Dims& dm) {
+    lola::Layout L{};
+    size_t off = 0;
+    auto take = [&](size_t n) { size_t r = off; off = (off + n + 255) & ~(size_t)255; return r; };
+    const size_t S = dm.S, e = dm.esize, snaps = (size_t)dm.nc_max + 1, T = dm.max_tokens;
+    L.W = take((size_t)dm.Hkv * dm.d * dm.Dh * e);
+    L.H = take(S * dm.D * dm.d * 4);
+    L.s = take(S * dm.D * 4);
+    L.cache_k = take(S * dm.lam * dm.d * e);
+    L.cache_v = take(S * dm.lam * dm.d * e);
+    L.cache_phik = take(S * dm.lam * dm.D * 4);
+    L.cache_pos = take(S * dm.lam * 4);
+    L.win_k = take(S * dm.eta * dm.d * e);
+    L.win_v = take(S * dm.eta * dm.d * e);
+    L.win_phik = take(S * dm.eta * dm.D * 4);
+    L.phik_new = take(S * T * dm.D * 4);
+    L.snap_pos = take(S * snaps * dm.lam * 4);
+    L.snap_H = take(S * snaps * dm.D * dm.d * 4);
+    L.snap_s = take(S * snaps * dm.D * 4);
+    L.io_q = take((size_t)dm.B * T * dm.Hq * dm.d * e);
+    L.io_k = take((size_t)dm.B * T * dm.Hkv * dm.d * e);
+    L.io_v = take((size_t)dm.B * T * dm.Hkv * dm.d * e);
+    L.io_y = take((size_t)dm.B * T * dm.Hq * dm.d * 4);
+    L.err = take(256);
+    L.total = off;
+    return L;
+}
+
+lola::StatePtrs state_ptrs(const lola_state* st) {
+    lola::StatePtrs p;
+    char* b = st->base;
+    p.W = b + st->L.W;
+    p.H = (float*)(b + st->L.H);
+    p.s = (float*)(b + st->L.s);
+    p.cache_k = b + st->L.cache_k;
+    p.cache_v = b + st->L.cache_v;
+    p.cache_phik = (float*)(b + st->L.cache_phik);
+    p.cache_pos = (int*)(b + st->L.cache_pos);
+    p.win_k = b + st->L.win_k;
+    p.win_v = b + st->L.win_v;
+    p.win_phik = (float*)(b + st->L.win_phik);
+    return p;
+}
+
+int clear_state(lola_state* st, cudaStream_t s) {
+    const lola::Dims& dm = st->dm;
+    const lola::Layout& L = st->L;
+    // everything from H up to (not including) the prefill scratch
+    cudaError_t e = cudaMemsetAsync(st->base + L.H, 0, L.phik_new - L.H, s);
+    if (e == cudaSuccess && dm.lam > 0)
+        e = cudaMemsetAsync(st->base + L.cache_pos, 0xFF, (size_t)dm.S * dm.lam * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the state");
+    st->t = 0;
+    st->last_nc = -1;
+    st->last_t0 = 0;
+    return LOLA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lola_last_error_string(void) { return g_err.c_str(); }
+
+int lola_state_bytes(const lola_config* cfg, size_t* bytes) {
+    lola::Dims dm;
+    int rc = make_dims(cfg, &dm);
+    if (rc) return rc;
+    if (!bytes) return fail(LOLA_ERR_INVALID_ARG, "null bytes pointer");
+    *bytes = make_layout(dm).total;
+    return LOLA_OK;
+}
+
+int lola_state_init(const lola_config* cfg, const void* W, void* dev_buf, size_t bytes,
+                    void* stream, lola_state** out) {
+    lola::Dims dm;
+    int rc = make_dims(cfg, &dm);
+    if (rc) return rc;
+    if (!W || !dev_buf || !out) return fail(LOLA_ERR_INVALID_ARG, "null W, dev_buf or out");
+    if ((uintptr_t)dev_buf & 255) return fail(LOLA_ERR_INVALID_ARG, "dev_buf is not 256-byte aligned");
+    const lola::Layout L = make_layout(dm);
+    if (bytes < L.total)
+        return fail(LOLA_ERR_BUF_TOO_SMALL, "dev_buf has %zu bytes, needs %zu", bytes, L.total);
+    lola_state* st = new lola_state();
+    st->cfg = *cfg;
+    st->dm = dm;
+    st->L = L;
+    st->base = (char*)dev_buf;
+    st->bytes = bytes;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(st->base + L.W, W, (size_t)dm.Hkv * dm.d * dm.Dh * dm.esize,
+                                    cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) { delete st; return cuda_fail(e, "copying W"); }
+    rc = clear_state(st, s);
+    if (rc) { delete st; return rc; }
+    *out = st;
+    return LOLA_OK;
+}
+
+int lola_state_reset(lola_state* st, void* stream) {
+    if (!st) return fail(LOLA_ERR_INVALID_ARG, "null state");
+    return clear_state(st, (cudaStream_t)stream);
+}
+
+int lola_state_free(lola_state* st) {
+    if (st) {
+        for (auto& m : st->marks) { cudaEventDestroy(m.a); cudaEventDestroy(m.b); }
+        for (auto e : st->pool) cudaEventDestroy(e);
+    }
+    delete st;
+    return LOLA_OK;
+}
+
+int lola_profile_enable(lola_state* st, int on) {
+    if (!st) return fail(LOLA_ERR_INVALID_ARG, "null state");
+    st->prof = on != 0;
+    return LOLA_OK;
+}
+
+int lola_profile_read(lola_state* st, float* ms, long long* launches, int n) {
+    if (!st || !ms || !launches || n < LOLA_KERNEL_CLASSES)
+        return fail(LOLA_ERR_INVALID_ARG, "null argument or n < %d", LOLA_KERNEL_CLASSES);
+    for (int i = 0; i < LOLA_KERNEL_CLASSES; ++i) { ms[i] = 0.f; launches[i] = 0; }
+    int rc = LOLA_OK;
+    for (auto& m : st->marks) {
+        float t = 0.f;
+        cudaError_t e = cudaEventSynchronize(m.b);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&t, m.a, m.b);
+        if (e != cudaSuccess && rc == LOLA_OK) rc = cuda_fail(e, "reading profile events");
+        ms[m.cls] += t;
+        launches[m.cls] += 1;
+        st->pool.push_back(m.a);
+        st->pool.push_back(m.b);
+    }
+    st->marks.clear();
+    return rc;
+}
+
+long long lola_launch_count(void) { return g_launches.load(); }
+
+int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const void* v, int T,
+                         float* y, void* stream) {
+    if (!st || !q || !k || !v || !y) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    const lola::Dims& dm = st->dm;
+    if (T < 1 || T % dm.C || T > dm.max_tokens)
+        return fail(LOLA_ERR_INVALID_ARG, "T=%d must be a positive multiple of chunk=%d and <= max_tokens=%d",
+                    T, dm.C, dm.max_tokens);
+    if (st->t + (long long)T >= 0x7fffffffLL) return fail(LOLA_ERR_INVALID_ARG, "position overflow");
+    lola::PrefillArgs a{};
+    a.dm = dm;
+    a.sp = state_ptrs(st);
+    a.q = q; a.k = k; a.v = v; a.y = y;
+    a.T = T;
+    a.t_start = (int)st->t;
+    a.nc = T / dm.C;
+    a.phik_new = (float*)(st->base + st->L.phik_new);
+    a.snap_pos = (int*)(st->base + st->L.snap_pos);
+    a.snap_H = (float*)(st->base + st->L.snap_H);
+    a.snap_s = (float*)(st->base + st->L.snap_s);
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if ((e = traced(st, 0, 1, s, [&] { return lola::launch_phi_keys(a, s); })) != cudaSuccess)
+        return cuda_fail(e, "feature-map kernel");
+    if ((e = traced(st, 1, 1, s, [&] { return lola::launch_scan(a, s); })) != cudaSuccess)
+        return cuda_fail(e, "scan kernel");
+    if ((e = traced(st, 2, 1, s, [&] { return lola::launch_output(a, s); })) != cudaSuccess)
+        return cuda_fail(e, "output kernel");
+    if ((e = traced(st, 3, dm.lam > 0 ? 2 : 1, s, [&] { return lola::launch_finalize(a, s); })) != cudaSuccess)
+        return cuda_fail(e, "finalize kernels");
+    st->last_nc = a.nc;
+    st->last_t0 = st->t;
+    st->t += T;
+    return LOLA_OK;
+}
+
+int lola_decode_step(lola_state* st, const void* q, const void* k, const void* v, float* y,
+                     void* stream) {
+    if (!st || !q || !k || !v || !y) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    if (st->t + 1 >= 0x7fffffffLL) return fail(LOLA_ERR_INVALID_ARG, "position overflow");
+    lola::DecodeArgs a{};
+    a.dm = st->dm;
+    a.sp = state_ptrs(st);
+    a.q = q; a.k = k; a.v = v; a.y = y;
+    a.t = (int)st->t;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = traced(st, 4, 1, s, [&] { return lola::launch_decode(a, s); });
+    if (e != cudaSuccess) return cuda_fail(e, "decode kernel");
+    st->t += 1;
+    return LOLA_OK;
+}
+
+int lola_prefill_chunked_host(lola_state* st, const void* q, const void* k, const void* v, int T,
+                              float* y, void* stream) {
+    if (!st || !q || !k || !v || !y) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    const lola::Dims& dm = st->dm;
+    if (T < 1 || T % dm.C || T > dm.max_tokens)
+        return fail(LOLA_ERR_INVALID_ARG, "T=%d must be a positive multiple of chunk and <= max_tokens", T);
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t nq = (size_t)dm.B * T * dm.Hq * dm.d, nk = (size_t)dm.B * T * dm.Hkv * dm.d;
+    char* b = st->base;
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(b + st->L.io_q, q, nq * dm.esize, cudaMemcpyHostToDevice, s)) ||
+        (e = cudaMemcpyAsync(b + st->L.io_k, k, nk * dm.esize, cudaMemcpyHostToDevice, s)) ||
+        (e = cudaMemcpyAsync(b + st->L.io_v, v, nk * dm.esize, cudaMemcpyHostToDevice, s)))
+        return cuda_fail(e, "host-to-device copy");
+    int rc = lola_prefill_chunked(st, b + st->L.io_q, b + st->L.io_k, b + st->L.io_v, T,
+                                  (float*)(b + st->L.io_y), stream);
+    if (rc) return rc;
+    if ((e = cudaMemcpyAsync(y, b + st->L.io_y, nq * 4, cudaMemcpyDeviceToHost, s)))
+        return cuda_fail(e, "device-to-host copy");
+    return LOLA_OK;
+}
+
+int lola_decode_step_host(lola_state* st, const void* q, const void* k, const void* v, float* y,
+                          void* stream) {
+    if (!st || !q || !k || !v || !y) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    const lola::Dims& dm = st->dm;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t nq = (size_t)dm.B * dm.Hq * dm.d, nk = (size_t)dm.B * dm.Hkv * dm.d;
+    char* b = st->base;
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(b + st->L.io_q, q, nq * dm.esize, cudaMemcpyHostToDevice, s)) ||
+        (e = cudaMemcpyAsync(b + st->L.io_k, k, nk * dm.esize, cudaMemcpyHostToDevice, s)) ||
+        (e = cudaMemcpyAsync(b + st->L.io_v, v, nk * dm.esize, cudaMemcpyHostToDevice, s)))
+        return cuda_fail(e, "host-to-device copy");
+    int rc = lola_decode_step(st, b + st->L.io_q, b + st->L.io_k, b + st->L.io_v,
+                              (float*)(b + st->L.io_y), stream);
+    if (rc) return rc;
+    if ((e = cudaMemcpyAsync(y, b + st->L.io_y, nq * 4, cudaMemcpyDeviceToHost, s)))
+        return cuda_fail(e, "device-to-host copy");
+    return LOLA_OK;
+}
+
+int lola_state_export(const lola_state* st, lola_state_view* out) {
+    if (!st || !out) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    const lola::StatePtrs p = state_ptrs(st);
+    const lola::Dims& dm = st->dm;
+    std::memset(out, 0, sizeof *out);
+    out->t = st->t;
+    const long long left = st->t - dm.eta;
+    out->n_cache = (int)(left <= 0 ? 0 : (left < dm.lam ? left : dm.lam));
+    out->H = p.H;
+    out->s = p.s;
+    out->cache_k = p.cache_k;
+    out->cache_v = p.cache_v;
+    out->cache_phik = p.cache_phik;
+    out->cache_pos = p.cache_pos;
+    out->win_k = p.win_k;
+    out->win_v = p.win_v;
+    out->win_phik = p.win_phik;
+    out->trace_pos = (int*)(st->base + st->L.snap_pos);
+    out->trace_len = st->last_nc < 0 ? 0 : st->last_nc + 1;
+    out->trace_stride = (dm.nc_max + 1) * dm.lam;
+    out->trace_t0 = st->last_t0;
+    return LOLA_OK;
+}
+
+}  // extern "C"

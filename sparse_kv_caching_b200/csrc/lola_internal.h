@@ -1,0 +1,89 @@
+// Internal declarations shared by the LoLA kernels and the C ABI layer.
+//
+// Memory model of one stream (one sequence b and kv head g, st = b*Hkv + g),
+// all inside the caller's device buffer:
+//   H [D][d] f32, s [D] f32                        linear state (notes §2.2, Eqs. 3-5)
+//   cache slots: k, v [lambda][d] (dtype), phik [lambda][D] f32, pos [lambda] i32
+//                                                  sparse global cache G (notes §2.4)
+//   window ring: k, v [eta][d] (dtype), phik [eta][D] f32; position p in slot p % eta
+//                                                  sliding window W (notes §2.4)
+// The window always holds positions [max(0, t - eta), t) and the cache
+// occupies slots [0, min(lambda, max(0, t - eta))) at a block boundary t, so
+// both are functions of t alone; only the slot contents need storage.
+//
+// Where a pair of the current prefill call lives (t_start = first position
+// of the call): p >= t_start -> the call's input arrays; t_start - eta <= p
+// < t_start -> the window ring; p < t_start - eta -> a cache slot that held
+// it when the call began (such a member never changes slot while cached).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace lola {
+
+constexpr int kThreads = 512;
+
+struct Layout {            // byte offsets inside dev_buf (all 256-aligned)
+    size_t W, H, s, cache_k, cache_v, cache_phik, cache_pos, win_k, win_v, win_phik;
+    size_t phik_new, snap_pos, snap_H, snap_s, io_q, io_k, io_v, io_y, err;
+    size_t total;
+};
+
+struct Dims {
+    int B, Hq, Hkv, Gq, d, Dh, D, eta, lam, C, dtype, S, max_tokens, nc_max;
+    int esize;             // bytes per input element
+};
+
+// Pointers to the persistent state of all streams.
+struct StatePtrs {
+    const void* W;
+    float* H;
+    float* s;
+    void* cache_k;
+    void* cache_v;
+    float* cache_phik;
+    int* cache_pos;
+    void* win_k;
+    void* win_v;
+    float* win_phik;
+};
+
+struct PrefillArgs {
+    Dims dm;
+    StatePtrs sp;
+    const void* q;         // [B][T][Hq][d]
+    const void* k;         // [B][T][Hkv][d]
+    const void* v;
+    float* y;              // [B][T][Hq][d]
+    int T;                 // tokens in this call
+    int t_start;           // position of the first token of the call
+    int nc;                // chunks in this call
+    float* phik_new;       // [S][max_tokens][D]
+    int* snap_pos;         // [S][nc_max+1][lambda]
+    float* snap_H;         // [S][nc_max+1][D][d]
+    float* snap_s;         // [S][nc_max+1][D]
+};
+
+struct DecodeArgs {
+    Dims dm;
+    StatePtrs sp;
+    const void* q;         // [B][Hq][d]
+    const void* k;         // [B][Hkv][d]
+    const void* v;
+    float* y;              // [B][Hq][d]
+    int t;                 // position of the new token
+};
+
+// Launchers (each returns cudaGetLastError() of its launch).
+cudaError_t launch_phi_keys(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_scan(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_output(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_finalize(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_clear(const Dims& dm, const StatePtrs& sp, cudaStream_t s);
+
+// Shared-memory bytes a scan CTA needs (0 if the shape is unsupported).
+size_t scan_smem_bytes(const Dims& dm);
+
+}  // namespace lola
