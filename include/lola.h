@@ -158,6 +158,27 @@ int lola_profile_read(lola_state* st, float* ms, long long* launches, int n);
 /* Number of kernels this library has launched in this process. */
 long long lola_launch_count(void);
 
+/* One-shot prefill that allocates nothing (this entry point has no
+ * counterpart in the paper; it serves callers that cannot call cudaMalloc,
+ * such as a plugin that only receives input and output pointers from its
+ * host application, or code running where another component owns every
+ * device allocation).  It runs lola_prefill_chunked on a fresh state (t = 0)
+ * for T tokens of q, k, v and writes y (all device, layouts above; W device
+ * [Hkv][d][Dh]).  The state and all scratch live in one array built into the
+ * library, LOLA_NOALLOC_SCRATCH_BYTES (64 MiB) of device memory that every
+ * GPU which loads the library holds until the process exits.  Configurations
+ * whose state and scratch exceed it are rejected with LOLA_ERR_BUF_TOO_SMALL
+ * (the need grows with B * Hkv and max_tokens; the 8B-shaped 4K prefill with
+ * B = 1 fits).  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  Every call reuses the same array and clears the
+ * memories first, so calls whose GPU work overlaps (different streams, or
+ * several host threads) race and corrupt each other: serialise them, e.g. on
+ * one stream.  The state is not kept after the call. */
+#define LOLA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int lola_prefill_once_noalloc(const lola_config* cfg, const void* W, const void* q, const void* k,
+                              const void* v, int T, float* y, void* stream);
+
 /* Text of the last error raised on this host thread ("" if none). */
 const char* lola_last_error_string(void);
 

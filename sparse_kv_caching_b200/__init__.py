@@ -25,7 +25,8 @@ ERRORS = {0: "OK", -1: "INVALID_ARG", -2: "BUF_TOO_SMALL", -3: "CUDA", -4: "TIME
 EXPORTS = ("lola_state_bytes", "lola_state_init", "lola_state_reset", "lola_state_free",
            "lola_prefill_chunked", "lola_decode_step", "lola_prefill_chunked_host",
            "lola_decode_step_host", "lola_state_export", "lola_profile_enable",
-           "lola_profile_read", "lola_launch_count", "lola_last_error_string")
+           "lola_profile_read", "lola_launch_count", "lola_prefill_once_noalloc",
+           "lola_last_error_string")
 KERNEL_CLASSES = ("phi", "scan", "output", "finalize", "decode")
 
 
@@ -70,6 +71,7 @@ def lib() -> ctypes.CDLL:
     L.lola_state_export.argtypes = [vp, POINTER(LolaStateView)]
     L.lola_profile_enable.argtypes = [vp, c_int]
     L.lola_profile_read.argtypes = [vp, POINTER(ctypes.c_float), POINTER(c_longlong), c_int]
+    L.lola_prefill_once_noalloc.argtypes = [POINTER(LolaConfig), vp, vp, vp, vp, c_int, vp, vp]
     L.lola_launch_count.argtypes = []
     L.lola_launch_count.restype = c_longlong
     L.lola_last_error_string.argtypes = []
@@ -101,6 +103,24 @@ def state_bytes(cfg: LolaConfig) -> int:
 def launch_count() -> int:
     """Kernels launched by liblola.so in this process."""
     return int(lib().lola_launch_count())
+
+
+def prefill_once_noalloc(cfg: LolaConfig, W, q, k, v, y, stream=None):
+    """One-shot prefill from an empty state using the library's built-in scratch array.
+
+    For callers that cannot allocate device memory: nothing is allocated here
+    or in the library; q, k, v, W and y are the caller's device tensors.
+    Calls share the built-in array, so overlapping calls race.
+    """
+    for x in (W, q, k, v, y):
+        if not (isinstance(x, torch.Tensor) and x.is_cuda and x.is_contiguous()):
+            raise ValueError("W, q, k, v, y must be contiguous CUDA tensors")
+    if y.dtype != torch.float32:
+        raise ValueError("y must be float32")
+    _check(lib().lola_prefill_once_noalloc(byref(cfg), c_void_p(W.data_ptr()), c_void_p(q.data_ptr()),
+                                           c_void_p(k.data_ptr()), c_void_p(v.data_ptr()), q.shape[1],
+                                           c_void_p(y.data_ptr()), _stream(stream)))
+    return y
 
 
 def _stream(stream=None) -> c_void_p:

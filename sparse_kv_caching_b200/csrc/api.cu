@@ -363,3 +363,76 @@ int lola_state_export(const lola_state* st, lola_state_view* out) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// One-shot prefill for callers that cannot allocate device memory.
+//
+// Its persistent state and scratch live in a file-scope device array of
+// LOLA_NOALLOC_SCRATCH_BYTES, created when the library's module is loaded on a
+// device and held by that device until the process exits.  Host code only
+// ever sees the array's host-side stand-in symbol; the device address comes
+// from cudaGetSymbolAddress, fetched once per device (with that device
+// current) on the first call there and cached.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[LOLA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(LOLA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the built-in scratch array");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LOLA_OK;
+}
+
+}  // namespace
+
+extern "C" int lola_prefill_once_noalloc(const lola_config* cfg, const void* W, const void* q,
+                                         const void* k, const void* v, int T, float* y,
+                                         void* stream) {
+    lola::Dims dm;
+    int rc = make_dims(cfg, &dm);
+    if (rc) return rc;
+    if (!W || !q || !k || !v || !y) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    if (T < 1 || T % dm.C || T > dm.max_tokens)
+        return fail(LOLA_ERR_INVALID_ARG, "T=%d must be a positive multiple of chunk=%d and <= max_tokens=%d",
+                    T, dm.C, dm.max_tokens);
+    const lola::Layout L = make_layout(dm);
+    const size_t need = L.io_q;          // state + prefill scratch; no host-I/O staging here
+    if (need > (size_t)LOLA_NOALLOC_SCRATCH_BYTES)
+        return fail(LOLA_ERR_BUF_TOO_SMALL,
+                    "this configuration needs %zu bytes of state and scratch; the built-in array holds %zu "
+                    "(lower max_tokens, or use lola_state_init with a caller buffer)",
+                    need, (size_t)LOLA_NOALLOC_SCRATCH_BYTES);
+    void* base = nullptr;
+    rc = noalloc_scratch(&base);
+    if (rc) return rc;
+    lola_state st;
+    st.cfg = *cfg;
+    st.dm = dm;
+    st.L = L;
+    st.base = (char*)base;
+    st.bytes = need;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(st.base + L.W, W, (size_t)dm.Hkv * dm.d * dm.Dh * dm.esize,
+                                    cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copying W");
+    rc = clear_state(&st, s);           // the array keeps the previous call's contents
+    if (rc) return rc;
+    return lola_prefill_chunked(&st, q, k, v, T, y, stream);
+}
