@@ -14,7 +14,8 @@
  *
  * Conventions (all entry points):
  *   - Every pointer named "device" is CUDA device memory on the current
- *     device; "host" pointers are page-locked (pinned) host memory.
+ *     device; "host" pointers are page-locked (pinned) host memory.  q, k, v
+ *     and y must be 16-byte aligned (LOLA_ERR_INVALID_ARG otherwise).
  *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *     stream.  All work is enqueued asynchronously on it, in stream order.
  *   - The caller owns every buffer.  The library allocates no device memory:
@@ -28,6 +29,10 @@
  *     fixed by this library; the pages leave phi as "learned"), D = 2 Dh.
  *   - Sequences of a batch advance in lock step: every call processes the
  *     same number of tokens for all B sequences.
+ *   - Precision: SRE, selection, fold and the state are f32.  With bf16
+ *     inputs the prefill output runs Q K^T in bf16 and P V in f16 on the
+ *     tensor cores (f32 accumulation), so values v must satisfy |v| < 65504;
+ *     the linear branch phi(q)^T H runs in tf32.  f32 inputs run in f32.
  *
  * Layouts (row-major, contiguous):
  *   q  [B][T][Hq][d], k and v [B][T][Hkv][d]   in `dtype`
@@ -98,6 +103,8 @@ typedef struct lola_state_view {
     int trace_len;          /* chunks of the last prefill call + 1 (0 if none)    */
     int trace_stride;       /* ints between the traces of consecutive streams     */
     long long trace_t0;
+    int* err_word;          /* device int, nonzero once a bounded device wait gave
+                               up (LOLA_ERR_TIMEOUT condition); cleared by reset */
 } lola_state_view;
 
 /* Bytes of device memory one layer state needs (persistent state, prefill
@@ -157,6 +164,18 @@ int lola_profile_read(lola_state* st, float* ms, long long* launches, int n);
 
 /* Number of kernels this library has launched in this process. */
 long long lola_launch_count(void);
+
+/* Diagnostic self-test of the tensor-core building blocks (no counterpart in
+ * the paper): one CTA computes C[128][N] = A[128][K] * B with tcgen05.mma from
+ * the shared-memory operand layouts the kernels use, accumulating in tensor
+ * memory.  mode bit 0: B given MN-major as [K][N] (else K-major as [N][K]);
+ * bit 1: f32 inputs computed as tf32 (else bf16 inputs); bit 2 (with bit 1):
+ * 3xTF32 split products.  A, B, C, err are device pointers (C f32 row-major,
+ * *err set to 1 if the MMA completion wait gave up).  Requires M = 128,
+ * 16 <= N <= 256 with N % 16 == 0, K a multiple of 16 (bf16) or 8 (tf32), and
+ * operands that fit in shared memory. */
+int lola_selftest_umma(int mode, const void* A, const void* B, float* C, int M, int N, int K,
+                       int* err, void* stream);
 
 /* One-shot prefill that allocates nothing (this entry point has no
  * counterpart in the paper; it serves callers that cannot call cudaMalloc,

@@ -25,7 +25,7 @@ ERRORS = {0: "OK", -1: "INVALID_ARG", -2: "BUF_TOO_SMALL", -3: "CUDA", -4: "TIME
 EXPORTS = ("lola_state_bytes", "lola_state_init", "lola_state_reset", "lola_state_free",
            "lola_prefill_chunked", "lola_decode_step", "lola_prefill_chunked_host",
            "lola_decode_step_host", "lola_state_export", "lola_profile_enable",
-           "lola_profile_read", "lola_launch_count", "lola_prefill_once_noalloc",
+           "lola_profile_read", "lola_launch_count", "lola_prefill_once_noalloc", "lola_selftest_umma",
            "lola_last_error_string")
 KERNEL_CLASSES = ("phi", "scan", "output", "finalize", "decode")
 
@@ -41,7 +41,7 @@ class LolaStateView(ctypes.Structure):
                 ("cache_k", c_void_p), ("cache_v", c_void_p), ("cache_phik", c_void_p),
                 ("cache_pos", c_void_p), ("win_k", c_void_p), ("win_v", c_void_p),
                 ("win_phik", c_void_p), ("trace_pos", c_void_p), ("trace_len", c_int),
-                ("trace_stride", c_int), ("trace_t0", c_longlong)]
+                ("trace_stride", c_int), ("trace_t0", c_longlong), ("err_word", c_void_p)]
 
 
 class LolaError(RuntimeError):
@@ -72,6 +72,7 @@ def lib() -> ctypes.CDLL:
     L.lola_profile_enable.argtypes = [vp, c_int]
     L.lola_profile_read.argtypes = [vp, POINTER(ctypes.c_float), POINTER(c_longlong), c_int]
     L.lola_prefill_once_noalloc.argtypes = [POINTER(LolaConfig), vp, vp, vp, vp, c_int, vp, vp]
+    L.lola_selftest_umma.argtypes = [c_int, vp, vp, vp, c_int, c_int, c_int, vp, vp]
     L.lola_launch_count.argtypes = []
     L.lola_launch_count.restype = c_longlong
     L.lola_last_error_string.argtypes = []
@@ -265,7 +266,8 @@ class LolaLayer:
                    cache_pos=self._view(v.cache_pos, (S, c.lambda_), torch.int32),
                    win_k=self._view(v.win_k, (S, c.eta, c.d), self.dtype),
                    win_v=self._view(v.win_v, (S, c.eta, c.d), self.dtype),
-                   win_phik=self._view(v.win_phik, (S, c.eta, D), torch.float32))
+                   win_phik=self._view(v.win_phik, (S, c.eta, D), torch.float32),
+                   err_word=self._view(v.err_word, (1,), torch.int32))
         if v.trace_len > 0 and c.lambda_ > 0:
             stride = v.trace_stride
             full = self._view(v.trace_pos, (S, stride), torch.int32)

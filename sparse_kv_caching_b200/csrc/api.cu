@@ -14,6 +14,9 @@
 
 namespace lola {
 size_t decode_smem_bytes(const Dims& dm);
+size_t selftest_smem(int mode, int M, int N, int K);
+cudaError_t launch_selftest(int mode, const void* A, const void* B, float* C, int M, int N, int K, int* err,
+                            cudaStream_t s);
 }
 
 struct lola_prof_mark {
@@ -154,6 +157,7 @@ int clear_state(lola_state* st, cudaStream_t s) {
     const lola::Layout& L = st->L;
     // everything from H up to (not including) the prefill scratch
     cudaError_t e = cudaMemsetAsync(st->base + L.H, 0, L.phik_new - L.H, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(st->base + L.err, 0, 256, s);
     if (e == cudaSuccess && dm.lam > 0)
         e = cudaMemsetAsync(st->base + L.cache_pos, 0xFF, (size_t)dm.S * dm.lam * 4, s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the state");
@@ -162,6 +166,8 @@ int clear_state(lola_state* st, cudaStream_t s) {
     st->last_t0 = 0;
     return LOLA_OK;
 }
+
+bool misaligned(const void* p) { return ((uintptr_t)p & 15u) != 0; }
 
 }  // namespace
 
@@ -245,9 +251,26 @@ int lola_profile_read(lola_state* st, float* ms, long long* launches, int n) {
 
 long long lola_launch_count(void) { return g_launches.load(); }
 
+int lola_selftest_umma(int mode, const void* A, const void* B, float* C, int M, int N, int K, int* err,
+                       void* stream) {
+    if (!A || !B || !C || !err) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    const bool tf32 = mode & 2;
+    if (mode < 0 || mode > 7 || ((mode & 4) && !tf32)) return fail(LOLA_ERR_INVALID_ARG, "mode=%d", mode);
+    if (M != 128 || N < 16 || N > 256 || N % 16 || K < (tf32 ? 8 : 16) || K % (tf32 ? 8 : 16))
+        return fail(LOLA_ERR_INVALID_ARG, "unsupported shape M=%d N=%d K=%d", M, N, K);
+    if (lola::selftest_smem(mode, M, N, K) > (size_t)kMaxSmem)
+        return fail(LOLA_ERR_UNSUPPORTED, "operands do not fit in shared memory");
+    cudaError_t e = lola::launch_selftest(mode, A, B, C, M, N, K, err, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "self-test kernel");
+    g_launches += 1;
+    return LOLA_OK;
+}
+
 int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const void* v, int T,
                          float* y, void* stream) {
     if (!st || !q || !k || !v || !y) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(y))
+        return fail(LOLA_ERR_INVALID_ARG, "q, k, v and y must be 16-byte aligned");
     const lola::Dims& dm = st->dm;
     if (T < 1 || T % dm.C || T > dm.max_tokens)
         return fail(LOLA_ERR_INVALID_ARG, "T=%d must be a positive multiple of chunk=%d and <= max_tokens=%d",
@@ -264,13 +287,16 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
     a.snap_pos = (int*)(st->base + st->L.snap_pos);
     a.snap_H = (float*)(st->base + st->L.snap_H);
     a.snap_s = (float*)(st->base + st->L.snap_s);
+    a.err = (int*)(st->base + st->L.err);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
     if ((e = traced(st, 0, 1, s, [&] { return lola::launch_phi_keys(a, s); })) != cudaSuccess)
         return cuda_fail(e, "feature-map kernel");
     if ((e = traced(st, 1, 1, s, [&] { return lola::launch_scan(a, s); })) != cudaSuccess)
         return cuda_fail(e, "scan kernel");
-    if ((e = traced(st, 2, 1, s, [&] { return lola::launch_output(a, s); })) != cudaSuccess)
+    if ((e = traced(st, 2, 1, s, [&] {
+             return dm.dtype == LOLA_DTYPE_BF16 ? lola::launch_output_tc(a, s) : lola::launch_output(a, s);
+         })) != cudaSuccess)
         return cuda_fail(e, "output kernel");
     if ((e = traced(st, 3, dm.lam > 0 ? 2 : 1, s, [&] { return lola::launch_finalize(a, s); })) != cudaSuccess)
         return cuda_fail(e, "finalize kernels");
@@ -283,12 +309,15 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
 int lola_decode_step(lola_state* st, const void* q, const void* k, const void* v, float* y,
                      void* stream) {
     if (!st || !q || !k || !v || !y) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    if (misaligned(q) || misaligned(k) || misaligned(v) || misaligned(y))
+        return fail(LOLA_ERR_INVALID_ARG, "q, k, v and y must be 16-byte aligned");
     if (st->t + 1 >= 0x7fffffffLL) return fail(LOLA_ERR_INVALID_ARG, "position overflow");
     lola::DecodeArgs a{};
     a.dm = st->dm;
     a.sp = state_ptrs(st);
     a.q = q; a.k = k; a.v = v; a.y = y;
     a.t = (int)st->t;
+    a.err = (int*)(st->base + st->L.err);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = traced(st, 4, 1, s, [&] { return lola::launch_decode(a, s); });
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel");
@@ -359,6 +388,7 @@ int lola_state_export(const lola_state* st, lola_state_view* out) {
     out->trace_len = st->last_nc < 0 ? 0 : st->last_nc + 1;
     out->trace_stride = (dm.nc_max + 1) * dm.lam;
     out->trace_t0 = st->last_t0;
+    out->err_word = (int*)(st->base + st->L.err);
     return LOLA_OK;
 }
 

@@ -61,8 +61,9 @@ struct PrefillArgs {
     int nc;                // chunks in this call
     float* phik_new;       // [S][max_tokens][D]
     int* snap_pos;         // [S][nc_max+1][lambda]
-    float* snap_H;         // [S][nc_max+1][D][d]
+    float* snap_H;         // [S][nc_max+1][d][D] (H_c transposed)
     float* snap_s;         // [S][nc_max+1][D]
+    int* err;              // device error word (bit 0: a bounded wait gave up)
 };
 
 struct DecodeArgs {
@@ -73,12 +74,14 @@ struct DecodeArgs {
     const void* v;
     float* y;              // [B][Hq][d]
     int t;                 // position of the new token
+    int* err;              // device error word
 };
 
 // Launchers (each returns cudaGetLastError() of its launch).
 cudaError_t launch_phi_keys(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_scan(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_output(const PrefillArgs& a, cudaStream_t s);
+cudaError_t launch_output_tc(const PrefillArgs& a, cudaStream_t s);   // bf16 on tcgen05
 cudaError_t launch_finalize(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_clear(const Dims& dm, const StatePtrs& sp, cudaStream_t s);

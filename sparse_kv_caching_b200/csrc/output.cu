@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(256) output_kernel(const __grid_constant__ Pre
     }
     __syncthreads();
 
-    // linear branch: acc = H_c^T phi(q), l = phi(q)^T s_c
+    // linear branch: acc = H_c^T phi(q), l = phi(q)^T s_c (H_c published as [d][D])
     const size_t snaps = (size_t)dm.nc_max + 1;
     const float* Hc = a.snap_H + ((size_t)st * snaps + c) * D * DIM;
     const float* sc = a.snap_s + ((size_t)st * snaps + c) * D;
@@ -105,8 +105,10 @@ __global__ void __launch_bounds__(256) output_kernel(const __grid_constant__ Pre
     for (int j0 = 0; j0 < D; j0 += HT) {
         const int nj = min(HT, D - j0);
         __syncthreads();
-        for (int idx = tid; idx < nj * DIM / 4; idx += 256)
-            reinterpret_cast<float4*>(Vs)[idx] = reinterpret_cast<const float4*>(Hc + (size_t)j0 * DIM)[idx];
+        for (int idx = tid; idx < nj * DIM; idx += 256) {     // snapshot is H^T [d][D]
+            const int jj = idx / DIM, cc = idx % DIM;
+            Vs[jj * DIM + cc] = Hc[(size_t)cc * D + j0 + jj];
+        }
         __syncthreads();
         for (int j = 0; j < nj; ++j) {
             float hv[CPL];

@@ -155,8 +155,13 @@ __global__ void __launch_bounds__(kThreads, 1) scan_kernel(PrefillArgs a) {
         float* sH = a.snap_H + ((size_t)st * snaps + c) * D * DV;
         float* sS = a.snap_s + ((size_t)st * snaps + c) * D;
         for (int j = tid; j < lam; j += kThreads) sp_[j] = slot_pos[j];
-        for (int i = tid; i < D * DV / 4; i += kThreads)
-            reinterpret_cast<float4*>(sH)[i] = reinterpret_cast<const float4*>(Hs)[i];
+        // H_c is published transposed, [d][D], so that a row c holds H[.][c]
+        for (int i = tid; i < DV * (D / 4); i += kThreads) {
+            const int cc = i % DV, j4 = (i / DV) * 4;
+            reinterpret_cast<float4*>(sH + (size_t)cc * D)[j4 / 4] =
+                make_float4(Hs[(j4 + 0) * DV + cc], Hs[(j4 + 1) * DV + cc], Hs[(j4 + 2) * DV + cc],
+                            Hs[(j4 + 3) * DV + cc]);
+        }
         for (int i = tid; i < D; i += kThreads) sS[i] = ss[i];
     };
     publish(0);

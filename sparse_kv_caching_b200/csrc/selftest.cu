@@ -1,0 +1,137 @@
+// Self-test of the tensor-core building blocks (umma.cuh): one CTA computes
+// C[M x N] = A[M x K] * B with tcgen05.mma from the chunk-major shared-memory
+// layouts the kernels use, the accumulator in TMEM, read back by tcgen05.ld.
+// Modes: bit 0 = B is MN-major ([K][N] in global) rather than K-major
+// ([N][K]); bit 1 = tf32 operands (f32 in global) rather than bf16; bit 2 =
+// 3xTF32 (hi*hi + hi*lo + lo*hi, f32-accurate products).
+#include "device_common.cuh"
+#include "umma.cuh"
+
+namespace lola {
+
+struct SelftestArgs {
+    int mode, M, N, K;
+    const void* A;
+    const void* B;
+    float* C;
+    int* err;
+};
+
+// Copy a row-major [R][Kc] global matrix into the chunk-major tile (rows R).
+template <typename T>
+__device__ void fill_chunk_major(uint8_t* dst, const T* src, int R, int Kc, bool split_lo, bool split_hi) {
+    constexpr int TPC = 16 / sizeof(T);           // elements per 16-byte chunk
+    const int nchunks = R * (Kc / TPC);
+    for (int idx = threadIdx.x; idx < nchunks; idx += blockDim.x) {
+        const int r = idx % R, kc = idx / R;
+        const T* s = src + (size_t)r * Kc + kc * TPC;
+        T* d = reinterpret_cast<T*>(dst + (size_t)kc * R * 16 + (size_t)r * 16);
+#pragma unroll
+        for (int i = 0; i < TPC; ++i) {
+            T x = s[i];
+            if constexpr (sizeof(T) == 4) {
+                if (split_hi) x = umma::tf32_hi(x);
+                else if (split_lo) x = x - umma::tf32_hi(x);
+            }
+            d[i] = x;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tbase;
+    const bool bmn = a.mode & 1, tf32 = a.mode & 2, x3 = (a.mode & 4) && tf32;
+    const int M = a.M, N = a.N, K = a.K;
+    const int es = tf32 ? 4 : 2;
+    const size_t szA = (size_t)M * K * es, szB = (size_t)N * K * es;
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + szA;
+    uint8_t* sA2 = sB + szB;                       // lo parts (3xTF32)
+    uint8_t* sB2 = sA2 + szA;
+    const int warp = threadIdx.x >> 5;
+    if (tf32) {
+        const float* A = (const float*)a.A;
+        const float* B = (const float*)a.B;
+        fill_chunk_major<float>(sA, A, M, K, false, x3);
+        if (x3) fill_chunk_major<float>(sA2, A, M, K, true, false);
+        if (bmn) {   // rows = K, chunks along N
+            fill_chunk_major<float>(sB, B, K, N, false, x3);
+            if (x3) fill_chunk_major<float>(sB2, B, K, N, true, false);
+        } else {
+            fill_chunk_major<float>(sB, B, N, K, false, x3);
+            if (x3) fill_chunk_major<float>(sB2, B, N, K, true, false);
+        }
+    } else {
+        fill_chunk_major<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, M, K, false, false);
+        if (bmn) fill_chunk_major<__nv_bfloat16>(sB, (const __nv_bfloat16*)a.B, K, N, false, false);
+        else fill_chunk_major<__nv_bfloat16>(sB, (const __nv_bfloat16*)a.B, N, K, false, false);
+    }
+    umma::fence_async_smem();
+    const uint32_t ncols = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+    if (warp == 0) umma::tmem_alloc(&tbase, ncols);
+    if (threadIdx.x == 0) { umma::mbar_init(&mbar, 1); umma::fence_mbar_init(); }
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tmem = tbase;
+    if (threadIdx.x == 0) {
+        const uint32_t id = umma::idesc(tf32 ? umma::kTF32 : umma::kBF16, M, N, false, bmn);
+        const int kstep = tf32 ? 8 : 16;
+        const uint32_t a0 = umma::smem_addr(sA), b0 = umma::smem_addr(sB);
+        const uint32_t a1 = umma::smem_addr(sA2), b1 = umma::smem_addr(sB2);
+        const uint32_t lboA = M * 16, sboA = 128;
+        const uint32_t lboB = bmn ? 128 : N * 16, sboB = bmn ? K * 16 : 128;
+        const int passes = x3 ? 3 : 1;
+        uint32_t acc = 0;
+        for (int p = 0; p < passes; ++p) {
+            const uint32_t abase = (p == 2) ? a1 : a0;   // pass 0: hi*hi, 1: hi*lo, 2: lo*hi
+            const uint32_t bbase = (p == 1) ? b1 : b0;
+            for (int ks = 0; ks < K / kstep; ++ks) {
+                const uint32_t aoff = ks * 2 * M * 16;
+                const uint32_t boff = bmn ? ks * kstep * 16 : ks * 2 * N * 16;
+                const uint64_t da = umma::sdesc(abase + aoff, lboA, sboA);
+                const uint64_t db = umma::sdesc(bbase + boff, lboB, sboB);
+                if (tf32) umma::mma_tf32(tmem, da, db, id, acc);
+                else umma::mma_bf16(tmem, da, db, id, acc);
+                acc = 1;
+            }
+        }
+        umma::commit(&mbar);
+    }
+    const bool ok = umma::mbar_wait(&mbar, 0);
+    if (!ok && threadIdx.x == 0) atomicExch(a.err, 1);
+    umma::fence_after_sync();
+    const int row = 32 * (warp & 3) + (threadIdx.x & 31);
+    for (int c0 = 0; c0 < N; c0 += 16) {
+        float r[16];
+        umma::tmem_ld16(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + c0, r);
+        umma::tmem_wait_ld();
+        if (row < M)
+            for (int i = 0; i < 16; ++i) a.C[(size_t)row * N + c0 + i] = ok ? r[i] : __int_as_float(0x7fc00000);
+    }
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(tmem, ncols);
+}
+
+size_t selftest_smem(int mode, int M, int N, int K) {
+    const bool tf32 = mode & 2, x3 = (mode & 4) && tf32;
+    const size_t es = tf32 ? 4 : 2;
+    size_t b = (size_t)M * K * es + (size_t)N * K * es;
+    return x3 ? 2 * b : b;
+}
+
+cudaError_t launch_selftest(int mode, const void* A, const void* B, float* C, int M, int N, int K, int* err,
+                            cudaStream_t s) {
+    const size_t bytes = selftest_smem(mode, M, N, K);
+    cudaError_t e = cudaFuncSetAttribute(umma_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)bytes);
+    if (e != cudaSuccess) return e;
+    SelftestArgs a{mode, M, N, K, A, B, C, err};
+    umma_selftest_kernel<<<1, 128, bytes, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace lola

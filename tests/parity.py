@@ -96,6 +96,8 @@ def check_prefill_stream(w, st: LolaStream, a: dict, t_lo: int, t_hi: int, trace
     mask = ~np.isnan(y)
     err = max_rel(y_gpu[mask], y[mask]) if mask.any() else 0.0
     chain.set_mismatch = set_mismatch
+    chain.abs_err = float(np.abs(y_gpu[mask] - y[mask]).max()) if mask.any() else 0.0
+    chain.y_max = float(np.abs(y[mask]).max()) if mask.any() else 0.0
     return err, chain
 
 

@@ -46,28 +46,29 @@ def _check_small(w, splits=None, rows_all=True):
     tol = P.TOL[w.dtype]
     worst = dict(y=0.0, H=0.0, s=0.0)
     ties = hard = setmis = 0
+    abs_err, y_max = 0.0, 0.0              # max |x - r| / max |r| over the whole y tensor
     for b in range(w.B):
         for g in range(w.Hkv):
             st = P.oracle_stream(w, g)
             a = synth.stream_arrays(w, b, g)
             yg = P.gpu_stream_y(y, w, b, g)
-            errs = []
             for ci, (t_lo, t_hi) in enumerate(zip(cuts[:-1], cuts[1:])):
                 nchunks = (t_hi - t_lo) // w.chunk
                 tr = (traces[ci][b * w.Hkv + g] if w.lam > 0
                       else np.full((nchunks + 1, 0), -1))
                 e, chain = P.check_prefill_stream(w, st, a, t_lo, t_hi, tr, yg[:, t_lo:t_hi])
-                errs.append(e)
+                abs_err = max(abs_err, chain.abs_err)
+                y_max = max(y_max, chain.y_max)
                 ties += chain.ties
                 hard += chain.hard
                 setmis += chain.set_mismatch
-            worst["y"] = max(worst["y"], max(errs))
             S = b * w.Hkv + g
             worst["H"] = max(worst["H"], P.max_rel(ex["H"][S].double().cpu().numpy(), st.H) if st.folded else 0.0)
             worst["s"] = max(worst["s"], P.max_rel(ex["s"][S].double().cpu().numpy(), st.s) if st.folded else 0.0)
             if w.lam > 0:
                 got = sorted(int(p) for p in ex["cache_pos"][S].cpu().numpy() if p >= 0)
                 assert got == sorted(st.cache)
+    worst["y"] = abs_err / y_max
     assert hard == 0 and setmis == 0, (hard, setmis, ties)
     assert worst["y"] <= tol and worst["H"] <= tol and worst["s"] <= tol, worst
     return worst, ties
