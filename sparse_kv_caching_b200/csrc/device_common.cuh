@@ -38,10 +38,12 @@ __device__ __forceinline__ float warp_max(float x) {
 }
 
 // Exclusive prefix sum of in[0, n) into out[0, n) by the whole block
-// (blockDim.x == kThreads); returns the total.  `tmp` holds >= 32 ints.
+// (blockDim.x a multiple of 32, at most 1024); returns the total.  `tmp`
+// holds >= 32 ints.
 __device__ inline int block_exscan(const int* in, int* out, int n, int* tmp) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int per = (n + kThreads - 1) / kThreads;
+    const int NT = blockDim.x;
+    const int per = (n + NT - 1) / NT;
     const int lo = min(n, tid * per), hi = min(n, lo + per);
     int sum = 0;
     for (int i = lo; i < hi; ++i) sum += in[i];
@@ -53,8 +55,8 @@ __device__ inline int block_exscan(const int* in, int* out, int n, int* tmp) {
     }
     if (lane == 31) tmp[warp] = x;
     __syncthreads();
+    const int NW = NT / 32;
     if (warp == 0) {
-        constexpr int NW = kThreads / 32;
         int w = lane < NW ? tmp[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -66,7 +68,7 @@ __device__ inline int block_exscan(const int* in, int* out, int n, int* tmp) {
     __syncthreads();
     int base = (warp ? tmp[warp - 1] : 0) + x - sum;
     for (int i = lo; i < hi; ++i) { out[i] = base; base += in[i]; }
-    const int total = tmp[kThreads / 32 - 1];
+    const int total = tmp[NW - 1];
     __syncthreads();
     return total;
 }
