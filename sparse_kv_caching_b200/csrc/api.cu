@@ -34,6 +34,7 @@ struct lola_state {
     int last_nc;
     long long last_t0;
     bool prof = false;
+    bool resid_ok = true;     // per-slot decode residuals match (H, s)
     std::vector<lola_prof_mark> marks;
     std::vector<cudaEvent_t> pool;
 };
@@ -123,6 +124,8 @@ lola::Layout make_layout(const lola::Dims& dm) {
     L.win_k = take(S * dm.eta * dm.d * e);
     L.win_v = take(S * dm.eta * dm.d * e);
     L.win_phik = take(S * dm.eta * dm.D * 4);
+    L.cache_R = take(S * dm.lam * dm.d * 4);
+    L.cache_den = take(S * dm.lam * 4);
     L.phik_new = take(S * T * dm.D * 4);
     L.snap_pos = take(S * snaps * dm.lam * 4);
     L.snap_H = take(S * snaps * dm.D * dm.d * 4);
@@ -149,6 +152,8 @@ lola::StatePtrs state_ptrs(const lola_state* st) {
     p.win_k = b + st->L.win_k;
     p.win_v = b + st->L.win_v;
     p.win_phik = (float*)(b + st->L.win_phik);
+    p.cache_R = (float*)(b + st->L.cache_R);
+    p.cache_den = (float*)(b + st->L.cache_den);
     return p;
 }
 
@@ -164,6 +169,7 @@ int clear_state(lola_state* st, cudaStream_t s) {
     st->t = 0;
     st->last_nc = -1;
     st->last_t0 = 0;
+    st->resid_ok = true;
     return LOLA_OK;
 }
 
@@ -303,6 +309,7 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
     st->last_nc = a.nc;
     st->last_t0 = st->t;
     st->t += T;
+    st->resid_ok = false;     // recomputed before the next decode step
     return LOLA_OK;
 }
 
@@ -319,7 +326,13 @@ int lola_decode_step(lola_state* st, const void* q, const void* k, const void* v
     a.t = (int)st->t;
     a.err = (int*)(st->base + st->L.err);
     cudaStream_t s = (cudaStream_t)stream;
-    cudaError_t e = traced(st, 4, 1, s, [&] { return lola::launch_decode(a, s); });
+    cudaError_t e;
+    if (!st->resid_ok) {
+        if ((e = traced(st, 4, st->dm.lam > 0 ? 1 : 0, s, [&] { return lola::launch_residual_init(a, s); })) != cudaSuccess)
+            return cuda_fail(e, "decode residual init kernel");
+        st->resid_ok = true;
+    }
+    e = traced(st, 4, 1, s, [&] { return lola::launch_decode(a, s); });
     if (e != cudaSuccess) return cuda_fail(e, "decode kernel");
     st->t += 1;
     return LOLA_OK;

@@ -1,4 +1,4 @@
-// Per-token LoLA decode step (notes §2.4, Fig. 1; one-token block of §2.6).
+// Per-token LoLA decode step (notes §2.4, Fig. 1; the one-token block of §2.6).
 //
 // For the new token at position t of every stream (sequence b, kv head g):
 //   1. read (Eq. 14) with the memories entering the step: the cache G, the
@@ -9,93 +9,173 @@
 //      fold the single lowest one (ties: the newer position goes; Eqs. 11-13)
 //      and, if that was not l, l takes its slot;
 //   4. the new token enters the window ring at slot t % eta.
-// One CTA per stream; H (D x d fp32) is staged in shared memory for the
-// linear read, the SRE scoring and the rank-1 fold, then written back.
+//
+// SRE without recomputing H^T phi for every candidate: each cache slot keeps
+// its residual R_e = H^T phi_e - den_e v_e and den_e = phi_e . s, so that
+// SRE_e = ||R_e||^2 / den_e^2 (and ||v_e||^2 while den_e = 0, the empty
+// memory recalling zero).  A decode step folds exactly one pair f, a rank-1
+// change of (H, s), after which R_e += k_e (v_f - v_e), den_e += k_e with
+// k_e = phi_e . phi_f: O(lambda (D + d)) work per step instead of
+// O(lambda D d), and no cancellation (the residual itself is stored).
+// residual_init_kernel computes them exactly from (H, s) after a prefill.
 #include "device_common.cuh"
+#include "umma.cuh"
 
 namespace lola {
 
-template <int DIM, int DH>
-struct DecShape {
-    static constexpr int D = 2 * DH;
-    using Sh = SreShape<D, DIM, float>;
-};
+constexpr int kDecThreads = 256;
+constexpr int kDecBatch = 4;      // keys / residual rows a warp loads before consuming them
+constexpr int kDecSlotBatch = 8;  // slot rows per warp in flight while scoring
 
 struct DecOffsets {
-    int Hs, ss, tile, den, qs, phq, kn, vn, phk, red, sc, sre, total;
+    int Hs, ss, Ws, qs, phq, kn, vn, phk, phl, Pl, vf, phf, red, kp, sc, wm, R, part, total;
 };
 
-__host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int lam, int eta) {
-    const int D = 2 * DH, TE = (kThreads / (DIM / 4)) * 8, LD = D + 4;
-    const int NK = lam + eta + 1;
+__host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int lam, int eta, bool r_smem,
+                                                  int esize) {
+    const int D = 2 * DH, NK = lam + eta + 1, NW = kDecThreads / 32;
     DecOffsets o;
     int p = 0;
     auto take = [&](int n) { int r = p; p += (n + 3) & ~3; return r; };
     o.Hs = take(D * DIM);
     o.ss = take(D);
-    o.tile = take(max(TE * LD, max(DIM * DH, 2 * (kThreads / DIM) * Gq * DIM)));
-    o.den = take(TE);
+    o.Ws = 0;                             // set below: W (raw, <= 4 B per element) aliases R/part
     o.qs = take(Gq * DIM);
     o.phq = take(Gq * D);
     o.kn = take(DIM);
     o.vn = take(DIM);
     o.phk = take(D);
-    o.red = take(64);
-    o.sc = take(Gq * NK);
-    o.sre = take(2 * (lam + 1));
+    o.phl = take(D);
+    o.Pl = take(DIM);
+    o.vf = take(DIM);
+    o.phf = take(D);
+    o.red = take(128);
+    o.kp = take(4 * NK);                   // key and value row pointers (64-bit each)
+    o.sc = take(max(Gq * NK, lam + 1));    // slot scores (update phase)
+    o.wm = take(NW * 8 * 2);               // per-warp softmax max and sum per head
+    // R [lam][DIM] (update phase) aliases the read-phase partial sums [NW][Gq][DIM]
+    o.R = take(max(max(r_smem ? lam * DIM : 0, NW * Gq * DIM), (DIM * DH * esize + 3) / 4 + (Gq + 1) * DH));
+    o.part = o.R;
+    o.Ws = o.R + (Gq + 1) * DH;           // after the z scratch rows
     o.total = p;
     return o;
 }
 
+// A quad of 4 lanes handles one row.  The row is cut into 4-element chunks and
+// lane q of the quad takes chunks q, q + 4, q + 8, ...: element u of lane q is
+// row[qidx(q, u)].  Lanes of a quad then read shared-memory operands in
+// different banks, and each chunk is one 16-byte (f32) or 8-byte (bf16) load.
+__device__ __forceinline__ int qidx(int q, int u) { return ((u >> 2) * 4 + q) * 4 + (u & 3); }
+__device__ __forceinline__ float quad_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    return x;
+}
+template <int N>
+__device__ __forceinline__ void load_quarter(const float* row, int q, float (&out)[N / 4]) {
+#pragma unroll
+    for (int i = 0; i < N / 16; ++i) {
+        const float4 f = *reinterpret_cast<const float4*>(row + (4 * i + q) * 4);
+        out[4 * i] = f.x; out[4 * i + 1] = f.y; out[4 * i + 2] = f.z; out[4 * i + 3] = f.w;
+    }
+}
+template <int N>
+__device__ __forceinline__ void load_quarter(const __nv_bfloat16* row, int q, float (&out)[N / 4]) {
+#pragma unroll
+    for (int i = 0; i < N / 16; ++i) {
+        const float4 f = load4(row + (4 * i + q) * 4);
+        out[4 * i] = f.x; out[4 * i + 1] = f.y; out[4 * i + 2] = f.z; out[4 * i + 3] = f.w;
+    }
+}
+
 template <int DIM, int DH, typename TIn>
-__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeArgs a) {
-    constexpr int D = 2 * DH;
-    using Sh = SreShape<D, DIM, TIn>;
+__global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int D = 2 * DH, NT = kDecThreads, NW = NT / 32, CPL = DIM / 32;
     extern __shared__ __align__(16) float smem[];
     const Dims& dm = a.dm;
     const int Gq = dm.Gq, lam = dm.lam, eta = dm.eta, t = a.t;
     const int st = blockIdx.x, b = st / dm.Hkv, g = st % dm.Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const DecOffsets o = dec_offsets(DIM, DH, Gq, lam, eta);
+    const bool rsm = a.r_smem != 0;                 // residual rows staged in shared memory
+    const DecOffsets o = dec_offsets(DIM, DH, Gq, lam, eta, rsm, (int)sizeof(TIn));
     float* Hs = smem + o.Hs;
     float* ss = smem + o.ss;
-    float* tile = smem + o.tile;
-    float* den = smem + o.den;
     float* qs = smem + o.qs;
     float* phq = smem + o.phq;
     float* kn = smem + o.kn;
     float* vn = smem + o.vn;
     float* phk = smem + o.phk;
+    float* phl = smem + o.phl;
+    float* Pl = smem + o.Pl;
+    float* vf = smem + o.vf;
+    float* phf = smem + o.phf;
     float* red = smem + o.red;
+    const TIn** kp = reinterpret_cast<const TIn**>(smem + o.kp);
     float* sc = smem + o.sc;
-    float* sre = smem + o.sre;
-    unsigned long long* keys = reinterpret_cast<unsigned long long*>(red);   // reuses red[0..)
-    float* Ws = tile;
+    float* wm = smem + o.wm;
+    float* Ws = smem + o.Ws;
+    float* Rs = smem + o.R;
+    float* part = smem + o.part;
 
     float* Hg = a.sp.H + (size_t)st * D * DIM;
     float* sg = a.sp.s + (size_t)st * D;
     const TIn* Wg = (const TIn*)a.sp.W + (size_t)g * DIM * DH;
-    for (int i = tid; i < DIM * DH; i += kThreads) Ws[i] = to_f32(Wg[i]);
-    for (int i = tid; i < D * DIM / 4; i += kThreads)
-        reinterpret_cast<float4*>(Hs)[i] = reinterpret_cast<const float4*>(Hg)[i];
-    for (int i = tid; i < D; i += kThreads) ss[i] = sg[i];
+    // H, s and W with asynchronous copies: every chunk in flight at once
+    TIn* Wsm = reinterpret_cast<TIn*>(Ws);
+    for (int i = tid; i < D * DIM / 4; i += NT) umma::cp_async16(Hs + 4 * i, Hg + 4 * i);
+    for (int i = tid; i < D / 4; i += NT) umma::cp_async16(ss + 4 * i, sg + 4 * i);
+    constexpr int WCH = DIM * DH * (int)sizeof(TIn) / 16;
+    for (int i = tid; i < WCH; i += NT)
+        umma::cp_async16(reinterpret_cast<char*>(Wsm) + 16 * i, reinterpret_cast<const char*>(Wg) + 16 * i);
+    umma::cp_async_commit();
     const TIn* qg = (const TIn*)a.q + ((size_t)b * dm.Hq + (size_t)g * Gq) * DIM;
-    for (int i = tid; i < Gq * DIM; i += kThreads) qs[i] = to_f32(qg[i]);
+    for (int i = tid; i < Gq * DIM; i += NT) qs[i] = to_f32(qg[i]);
     const TIn* kg = (const TIn*)a.k + ((size_t)b * dm.Hkv + g) * DIM;
     const TIn* vg = (const TIn*)a.v + ((size_t)b * dm.Hkv + g) * DIM;
-    for (int i = tid; i < DIM; i += kThreads) { kn[i] = to_f32(kg[i]); vn[i] = to_f32(vg[i]); }
+    for (int i = tid; i < DIM; i += NT) { kn[i] = to_f32(kg[i]); vn[i] = to_f32(vg[i]); }
+    const int n_g = min(lam, max(0, t - eta));
+    const int w_lo = max(0, t - eta);
+    const int n_w = t - w_lo;
+    const int NK = n_g + n_w + 1;
+    const size_t cbase = (size_t)st * lam, wbase = (size_t)st * eta;
+    // key row pointers: cache slots, window (ring slot p % eta), then the token itself
+    for (int i = tid; i < NK; i += NT) {
+        const TIn* p;
+        if (i < n_g) p = (const TIn*)a.sp.cache_k + (cbase + i) * DIM;
+        else if (i < n_g + n_w) p = (const TIn*)a.sp.win_k + (wbase + (size_t)((w_lo + i - n_g) % eta)) * DIM;
+        else p = kg;
+        kp[2 * i] = p;
+        // the value row sits at the same offset of the matching value array
+        const TIn* pv;
+        if (i < n_g) pv = (const TIn*)a.sp.cache_v + (cbase + i) * DIM;
+        else if (i < n_g + n_w) pv = (const TIn*)a.sp.win_v + (wbase + (size_t)((w_lo + i - n_g) % eta)) * DIM;
+        else pv = vg;
+        kp[2 * i + 1] = pv;
+    }
+    umma::cp_async_wait<0>();
     __syncthreads();
 
-    // feature map of the queries and of the new key (one warp per row)
-    for (int r = warp; r <= Gq; r += kThreads / 32) {
+    // feature map of the queries and the new key: z = x W (thread per (row, column)), then
+    // softmax(z) and softmax(-z) per row (one warp per row)
+    const int lpos = t - eta, rs = lpos >= 0 ? lpos % eta : 0;
+    const bool leaving = t >= eta;
+    if (leaving)
+        for (int i = tid; i < D; i += NT) phl[i] = a.sp.win_phik[(wbase + rs) * D + i];
+    __syncthreads();
+    float* zs = Rs;                                                   // scratch [Gq + 1][DH]
+    for (int idx = tid; idx < (Gq + 1) * DH; idx += NT) {
+        const int r = idx / DH, col = idx % DH;
         const float* x = r < Gq ? qs + r * DIM : kn;
+        float z = 0.f;
+#pragma unroll 8
+        for (int j = 0; j < DIM; ++j) z = fmaf(x[j], to_f32(Wsm[j * DH + col]), z);
+        zs[idx] = z;
+    }
+    __syncthreads();
+    for (int r = warp; r <= Gq; r += NW) {
         float z[DH / 32];
 #pragma unroll
-        for (int u = 0; u < DH / 32; ++u) z[u] = 0.f;
-        for (int j = 0; j < DIM; ++j) {
-#pragma unroll
-            for (int u = 0; u < DH / 32; ++u) z[u] = fmaf(x[j], Ws[j * DH + lane + 32 * u], z[u]);
-        }
+        for (int u = 0; u < DH / 32; ++u) z[u] = zs[r * DH + lane + 32 * u];
         float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
         for (int u = 0; u < DH / 32; ++u) { mx = fmaxf(mx, z[u]); mn = fminf(mn, z[u]); }
@@ -112,199 +192,359 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
     __syncthreads();
 
-    // ---- read: exact keys (cache, window, self) ----
-    const int n_g = min(lam, max(0, t - eta));
-    const int w_lo = max(0, t - eta);
-    const int n_w = t - w_lo;
-    const int NK = n_g + n_w + 1;
-    const size_t cbase = (size_t)st * lam, wbase = (size_t)st * eta;
-    auto key_row = [&](int i, const TIn*& kp, const TIn*& vp) {
-        if (i < n_g) { kp = (const TIn*)a.sp.cache_k + (cbase + i) * DIM; vp = (const TIn*)a.sp.cache_v + (cbase + i) * DIM; }
-        else if (i < n_g + n_w) {
-            const size_t w = wbase + (size_t)((w_lo + i - n_g) % eta);
-            kp = (const TIn*)a.sp.win_k + w * DIM; vp = (const TIn*)a.sp.win_v + w * DIM;
-        } else { kp = kg; vp = vg; }
-    };
-    const float scale = 1.0f / sqrtf((float)DIM);
-    for (int i = tid; i < NK; i += kThreads) {
-        const TIn *kp, *vp;
-        key_row(i, kp, vp);
-        float accs[8];
-#pragma unroll
-        for (int hh = 0; hh < 8; ++hh) accs[hh] = 0.f;
-        for (int j = 0; j < DIM; j += 4) {
-            const float4 k4 = load4(kp + j);
+    // ---- read: scores (a quad per key), softmax per head, P V (lane owns columns) ----
+    {
+        constexpr int KQ = DIM / 4;                                  // key elements per quad lane
+        const int q4 = lane & 3, rq = lane >> 2;                     // lane in quad, quad in warp
+        const float scale = 1.0f / sqrtf((float)DIM);
+        for (int i0 = warp * 8; i0 < NK; i0 += NW * 8) {
+            const int i = i0 + rq;
+            float kk[KQ];
+            if (i < NK) load_quarter<DIM>(kp[2 * i], q4, kk);
 #pragma unroll
             for (int hh = 0; hh < 8; ++hh) {
                 if (hh < Gq) {
-                    const float* qh = qs + hh * DIM + j;
-                    accs[hh] = fmaf(qh[0], k4.x, fmaf(qh[1], k4.y, fmaf(qh[2], k4.z, fmaf(qh[3], k4.w, accs[hh]))));
+                    float sdot = 0.f;
+                    if (i < NK) {
+#pragma unroll
+                        for (int u = 0; u < KQ; ++u) sdot = fmaf(qs[hh * DIM + qidx(q4, u)], kk[u], sdot);
+                    }
+                    sdot = quad_sum(sdot);
+                    if (i < NK && q4 == 0) sc[hh * NK + i] = sdot * scale;
                 }
             }
         }
-        for (int hh = 0; hh < Gq; ++hh) sc[hh * NK + i] = accs[hh] * scale;
-    }
-    __syncthreads();
-    // per head: max, exponentials, sum; linear denominator
-    for (int hh = warp; hh < Gq; hh += kThreads / 32) {
-        float mx = -INFINITY;
-        for (int i = lane; i < NK; i += 32) mx = fmaxf(mx, sc[hh * NK + i]);
-        mx = warp_max(mx);
-        float sum = 0.f;
-        for (int i = lane; i < NK; i += 32) { const float e = expf(sc[hh * NK + i] - mx); sc[hh * NK + i] = e; sum += e; }
-        sum = warp_sum(sum);
-        float dl = 0.f;
-        for (int j = lane; j < D; j += 32) dl = fmaf(phq[hh * D + j], ss[j], dl);
-        dl = warp_sum(dl);
-        if (lane == 0) { red[hh] = mx; red[8 + hh] = sum; red[16 + hh] = dl; }
-    }
-    __syncthreads();
-    {
-        constexpr int GR = kThreads / DIM;           // key groups
-        const int cidx = tid % DIM, grp = tid / DIM;
-        float aacc[8], lacc[8];
-#pragma unroll
-        for (int hh = 0; hh < 8; ++hh) aacc[hh] = lacc[hh] = 0.f;
-        for (int i = grp; i < NK; i += GR) {
-            const TIn *kp, *vp;
-            key_row(i, kp, vp);
-            const float vv = to_f32(vp[cidx]);
-#pragma unroll
-            for (int hh = 0; hh < 8; ++hh) if (hh < Gq) aacc[hh] = fmaf(sc[hh * NK + i], vv, aacc[hh]);
-        }
-        for (int j = grp; j < D; j += GR) {
-            const float hv = Hs[j * DIM + cidx];
-#pragma unroll
-            for (int hh = 0; hh < 8; ++hh) if (hh < Gq) lacc[hh] = fmaf(phq[hh * D + j], hv, lacc[hh]);
-        }
-        float* ra = tile;                            // [GR][Gq][DIM]
-        float* rl = tile + GR * Gq * DIM;
-        for (int hh = 0; hh < Gq; ++hh) {
-            ra[(grp * Gq + hh) * DIM + cidx] = aacc[hh];
-            rl[(grp * Gq + hh) * DIM + cidx] = lacc[hh];
+        __syncthreads();
+        for (int hh = warp; hh < Gq; hh += NW) {
+            float mx = -INFINITY;
+            for (int i = lane; i < NK; i += 32) mx = fmaxf(mx, sc[hh * NK + i]);
+            mx = warp_max(mx);
+            float sum = 0.f;
+            for (int i = lane; i < NK; i += 32) { const float e = expf(sc[hh * NK + i] - mx); sc[hh * NK + i] = e; sum += e; }
+            sum = warp_sum(sum);
+            float dl = 0.f;
+            for (int j = lane; j < D; j += 32) dl = fmaf(phq[hh * D + j], ss[j], dl);
+            dl = warp_sum(dl);
+            if (lane == 0) { red[hh] = mx; red[8 + hh] = sum; red[16 + hh] = dl; }
         }
         __syncthreads();
-        for (int idx = tid; idx < Gq * DIM; idx += kThreads) {
+        float accp[8][CPL];
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh)
+#pragma unroll
+            for (int u = 0; u < CPL; ++u) accp[hh][u] = 0.f;
+        for (int i0 = warp; i0 < NK; i0 += NW * kDecSlotBatch) {
+            float vv[kDecSlotBatch][CPL];
+#pragma unroll
+            for (int bb = 0; bb < kDecSlotBatch; ++bb) {             // issue the batch's loads first
+                const int i = i0 + bb * NW;
+                if (i < NK) {
+                    const TIn* vr = kp[2 * i + 1] + lane * CPL;
+                    if constexpr (CPL == 4) { const float4 v4 = load4(vr); vv[bb][0] = v4.x; vv[bb][1] = v4.y; vv[bb][2] = v4.z; vv[bb][3] = v4.w; }
+                    else { const float2 v2 = load2(vr); vv[bb][0] = v2.x; vv[bb][1] = v2.y; }
+                }
+            }
+#pragma unroll
+            for (int bb = 0; bb < kDecSlotBatch; ++bb) {
+                const int i = i0 + bb * NW;
+                if (i >= NK) break;
+#pragma unroll
+                for (int hh = 0; hh < 8; ++hh) {
+                    if (hh < Gq) {
+                        const float p = sc[hh * NK + i];
+#pragma unroll
+                        for (int u = 0; u < CPL; ++u) accp[hh][u] = fmaf(p, vv[bb][u], accp[hh][u]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh)
+            if (hh < Gq)
+#pragma unroll
+                for (int u = 0; u < CPL; ++u) part[(warp * Gq + hh) * DIM + lane * CPL + u] = accp[hh][u];
+        __syncthreads();
+        for (int idx = tid; idx < Gq * DIM; idx += NT) {
             const int hh = idx / DIM, cc = idx % DIM;
-            float A = 0.f, L = 0.f;
-            for (int r = 0; r < GR; ++r) { A += ra[(r * Gq + hh) * DIM + cc]; L += rl[(r * Gq + hh) * DIM + cc]; }
+            float A = 0.f;
+            for (int w = 0; w < NW; ++w) A += part[(w * Gq + hh) * DIM + cc];
+            float L = 0.f;
+            for (int j = 0; j < D; ++j) L = fmaf(phq[hh * D + j], Hs[j * DIM + cc], L);
             const float em = expf(-red[hh]);
-            const float yv = (A + em * L) / (red[8 + hh] + em * red[16 + hh]);
-            a.y[((size_t)b * dm.Hq + (size_t)g * Gq + hh) * DIM + cc] = yv;
+            a.y[((size_t)b * dm.Hq + (size_t)g * Gq + hh) * DIM + cc] = (A + em * L) / (red[8 + hh] + em * red[16 + hh]);
         }
         __syncthreads();
     }
 
     // ---- update ----
-    if (t >= eta) {
-        const int lpos = t - eta, rs = lpos % eta;
+    if (leaving) {
         const size_t wsl = wbase + rs;
+        const TIn* vl = (const TIn*)a.sp.win_v + wsl * DIM;
+        // P_l = H^T phi_l, den_l = phi_l . s, R_l = P_l - den_l v_l (pre-fold state)
+        for (int cc = tid; cc < DIM; cc += NT) {
+            float x = 0.f;
+            for (int j = 0; j < D; ++j) x = fmaf(phl[j], Hs[j * DIM + cc], x);
+            Pl[cc] = x;
+        }
+        if (warp == 0) {
+            float x = 0.f;
+            for (int j = lane; j < D; j += 32) x = fmaf(phl[j], ss[j], x);
+            x = warp_sum(x);
+            if (lane == 0) red[32] = x;
+        }
+        __syncthreads();
+        const float den_l = red[32];
+        float* Rg = a.sp.cache_R + cbase * DIM;
+        float* deng = a.sp.cache_den + cbase;
         if (n_g < lam) {
+            // l joins the next free slot (fewer than lambda candidates: keep all)
             const size_t cs = cbase + n_g;
-            for (int i = tid; i < DIM; i += kThreads) {
+            for (int i = tid; i < DIM; i += NT) {
                 ((TIn*)a.sp.cache_k)[cs * DIM + i] = ((const TIn*)a.sp.win_k)[wsl * DIM + i];
-                ((TIn*)a.sp.cache_v)[cs * DIM + i] = ((const TIn*)a.sp.win_v)[wsl * DIM + i];
+                ((TIn*)a.sp.cache_v)[cs * DIM + i] = vl[i];
+                Rg[(size_t)n_g * DIM + i] = Pl[i] - den_l * to_f32(vl[i]);
             }
-            for (int i = tid; i < D; i += kThreads) a.sp.cache_phik[cs * D + i] = a.sp.win_phik[wsl * D + i];
-            if (tid == 0) a.sp.cache_pos[cs] = lpos;
+            for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
+            if (tid == 0) { a.sp.cache_pos[cs] = lpos; deng[n_g] = den_l; }
         } else {
-            const int n = lam + 1;
-            auto phirow = [&](int e) -> const float* {
-                return e < lam ? a.sp.cache_phik + (cbase + e) * D : a.sp.win_phik + wsl * D;
-            };
-            auto vrow = [&](int e) -> const TIn* {
-                return e < lam ? (const TIn*)a.sp.cache_v + (cbase + e) * DIM : (const TIn*)a.sp.win_v + wsl * DIM;
-            };
-            for (int e0 = 0; e0 < n; e0 += Sh::TE) {
-                const int ne = min(Sh::TE, n - e0);
-                load_phi_tile<D>(tile, ne, [&](int e) { return phirow(e0 + e); });
-                __syncthreads();
-                sre_tile<D, DIM, TIn>(Hs, ss, tile, den, ne, [&](int e) { return vrow(e0 + e); }, sre + e0);
+            // scores: slots from their residuals (one warp per slot), l from R_l
+            float* scs = red + 64;                                    // reuse as scratch for the argmin
+            {
+                constexpr int RQ = DIM / 4;
+                const int q4 = lane & 3, rq = lane >> 2;
+                for (int e0 = warp * 8; e0 < lam; e0 += NW * 8) {
+                    const int e = e0 + rq;
+                    float rv[RQ];
+                    float dn = 0.f;
+                    if (e < lam) { load_quarter<DIM>(Rg + (size_t)e * DIM, q4, rv); dn = deng[e]; }
+                    float q = 0.f;
+                    if (e < lam) {
+#pragma unroll
+                        for (int u = 0; u < RQ; ++u) q = fmaf(rv[u], rv[u], q);
+                        if (rsm)
+#pragma unroll
+                            for (int u = 0; u < RQ; ++u) Rs[e * DIM + qidx(q4, u)] = rv[u];
+                    }
+                    q = quad_sum(q);
+                    float vq = 0.f;
+                    if (e < lam && !(dn > 0.f)) {                     // empty memory: SRE = ||v||^2
+                        float vv[RQ];
+                        load_quarter<DIM>((const TIn*)a.sp.cache_v + (cbase + e) * DIM, q4, vv);
+#pragma unroll
+                        for (int u = 0; u < RQ; ++u) vq = fmaf(vv[u], vv[u], vq);
+                    }
+                    vq += __shfl_xor_sync(0xffffffffu, vq, 1);
+                    vq += __shfl_xor_sync(0xffffffffu, vq, 2);
+                    if (e < lam && q4 == 0) sc[e] = dn > 0.f ? q / (dn * dn) : vq;
+                }
             }
-            // the folded pair: lowest SRE, newer position on exact ties (keys are unique)
+            if (warp == 0) {
+                float q = 0.f, vq = 0.f;
+                for (int cc = lane; cc < DIM; cc += 32) {
+                    const float v = to_f32(vl[cc]);
+                    const float r = Pl[cc] - den_l * v;
+                    q = fmaf(r, r, q);
+                    vq = fmaf(v, v, vq);
+                }
+                q = warp_sum(q);
+                vq = warp_sum(vq);
+                if (lane == 0) sc[lam] = den_l > 0.f ? q / (den_l * den_l) : vq;
+            }
+            __syncthreads();
+            // the folded pair: lowest SRE, the newer position on exact ties (keys are unique)
             auto cand_key = [&](int e) -> unsigned long long {
                 const int p = e < lam ? a.sp.cache_pos[cbase + e] : lpos;
-                return ((unsigned long long)__float_as_uint(sre[e]) << 32) | (unsigned long long)(~(unsigned)p);
+                return ((unsigned long long)__float_as_uint(sc[e]) << 32) | (unsigned long long)(~(unsigned)p);
             };
             unsigned long long best = ~0ull;
-            for (int e = tid; e < n; e += kThreads) { const unsigned long long k = cand_key(e); best = k < best ? k : best; }
+            for (int e = tid; e <= lam; e += NT) { const unsigned long long kk = cand_key(e); best = kk < best ? kk : best; }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) {
                 const unsigned long long o2 = __shfl_xor_sync(0xffffffffu, best, off);
                 best = o2 < best ? o2 : best;
             }
+            unsigned long long* keys = reinterpret_cast<unsigned long long*>(scs);
             if (lane == 0) keys[warp] = best;
             __syncthreads();
             unsigned long long bb = keys[0];
-            for (int w = 1; w < kThreads / 32; ++w) bb = keys[w] < bb ? keys[w] : bb;
-            for (int e = tid; e < n; e += kThreads)
-                if (cand_key(e) == bb) reinterpret_cast<int*>(red)[40] = e;
+            for (int w = 1; w < NW; ++w) bb = keys[w] < bb ? keys[w] : bb;
+            int* fsel = reinterpret_cast<int*>(red + 40);
+            for (int e = tid; e <= lam; e += NT)
+                if (cand_key(e) == bb) *fsel = e;
             __syncthreads();
-            const int f = reinterpret_cast<int*>(red)[40];
+            const int f = *fsel;
             // stage the folded pair
-            float* fphi = tile;
-            float* fv = tile + D;
-            for (int i = tid; i < D; i += kThreads) fphi[i] = phirow(f)[i];
-            for (int i = tid; i < DIM; i += kThreads) fv[i] = to_f32(vrow(f)[i]);
+            for (int i = tid; i < D; i += NT) phf[i] = f < lam ? a.sp.cache_phik[(cbase + f) * D + i] : phl[i];
+            for (int i = tid; i < DIM; i += NT) vf[i] = to_f32(f < lam ? ((const TIn*)a.sp.cache_v)[(cbase + f) * DIM + i] : vl[i]);
             __syncthreads();
-            for (int i = tid; i < D * DIM; i += kThreads) {
-                const int j = i / DIM, cc = i % DIM;
-                Hs[i] = fmaf(fphi[j], fv[cc], Hs[i]);
-            }
-            for (int i = tid; i < D; i += kThreads) ss[i] += fphi[i];
-            if (f < lam) {                           // l takes the folded member's slot
-                const size_t cs = cbase + f;
-                for (int i = tid; i < DIM; i += kThreads) {
-                    ((TIn*)a.sp.cache_k)[cs * DIM + i] = ((const TIn*)a.sp.win_k)[wsl * DIM + i];
-                    ((TIn*)a.sp.cache_v)[cs * DIM + i] = ((const TIn*)a.sp.win_v)[wsl * DIM + i];
+            // fold (Eqs. 12-13): H += phi_f v_f^T, s += phi_f
+            for (int i = tid; i < D * DIM; i += NT) Hs[i] = fmaf(phf[i / DIM], vf[i % DIM], Hs[i]);
+            for (int i = tid; i < D; i += NT) ss[i] += phf[i];
+            // residuals of every remaining member follow the rank-1 change
+            // a quad per member: k_e = phi_e . phi_f, R_e += k_e (v_f - v_e), den_e += k_e
+            {
+                constexpr int PQ = D / 4, RQ = DIM / 4;
+                const int q4 = lane & 3, rq = lane >> 2;
+                for (int e0 = warp * 8; e0 <= lam; e0 += NW * 8) {
+                    const int e = e0 + rq;
+                    const bool act = e <= lam && e != f;
+                    float pv[PQ], vv[RQ], r0[RQ];
+                    float d0 = 0.f;
+                    if (act) {
+                        load_quarter<D>(e < lam ? a.sp.cache_phik + (cbase + e) * D : phl, q4, pv);
+                        load_quarter<DIM>(e < lam ? (const TIn*)a.sp.cache_v + (cbase + e) * DIM : vl, q4, vv);
+                        if (e < lam) {
+                            if (rsm) {
+#pragma unroll
+                                for (int u = 0; u < RQ; ++u) r0[u] = Rs[e * DIM + qidx(q4, u)];
+                            } else {
+                                load_quarter<DIM>(Rg + (size_t)e * DIM, q4, r0);
+                            }
+                            d0 = deng[e];
+                        } else {
+#pragma unroll
+                            for (int u = 0; u < RQ; ++u) r0[u] = Pl[qidx(q4, u)] - den_l * vv[u];
+                            d0 = den_l;
+                        }
+                    }
+                    float kap = 0.f;
+                    if (act) {
+#pragma unroll
+                        for (int u = 0; u < PQ; ++u) kap = fmaf(pv[u], phf[qidx(q4, u)], kap);
+                    }
+                    kap = quad_sum(kap);
+                    if (act) {
+                        const int dst = e < lam ? e : f;   // its own slot, or f's slot for the newcomer l
+                        float* rw = Rg + (size_t)dst * DIM;
+#pragma unroll
+                        for (int u = 0; u < RQ; u += 4) {
+                            const int c0 = qidx(q4, u);                       // 4 consecutive columns
+                            *reinterpret_cast<float4*>(rw + c0) = make_float4(
+                                fmaf(kap, vf[c0] - vv[u], r0[u]), fmaf(kap, vf[c0 + 1] - vv[u + 1], r0[u + 1]),
+                                fmaf(kap, vf[c0 + 2] - vv[u + 2], r0[u + 2]), fmaf(kap, vf[c0 + 3] - vv[u + 3], r0[u + 3]));
+                        }
+                        if (q4 == 0) deng[dst] = d0 + kap;
+                    }
                 }
-                for (int i = tid; i < D; i += kThreads) a.sp.cache_phik[cs * D + i] = a.sp.win_phik[wsl * D + i];
+            }
+            if (f < lam) {                                            // l takes the folded member's slot
+                const size_t cs = cbase + f;
+                for (int i = tid; i < DIM; i += NT) {
+                    ((TIn*)a.sp.cache_k)[cs * DIM + i] = ((const TIn*)a.sp.win_k)[wsl * DIM + i];
+                    ((TIn*)a.sp.cache_v)[cs * DIM + i] = vl[i];
+                }
+                for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
                 if (tid == 0) a.sp.cache_pos[cs] = lpos;
             }
             __syncthreads();
-            for (int i = tid; i < D * DIM / 4; i += kThreads)
+            for (int i = tid; i < D * DIM / 4; i += NT)
                 reinterpret_cast<float4*>(Hg)[i] = reinterpret_cast<const float4*>(Hs)[i];
-            for (int i = tid; i < D; i += kThreads) sg[i] = ss[i];
+            for (int i = tid; i < D; i += NT) sg[i] = ss[i];
         }
     }
     __syncthreads();
     // the new token enters the window ring
     {
         const size_t ws = wbase + (size_t)(t % eta);
-        for (int i = tid; i < DIM; i += kThreads) {
+        for (int i = tid; i < DIM; i += NT) {
             ((TIn*)a.sp.win_k)[ws * DIM + i] = kg[i];
             ((TIn*)a.sp.win_v)[ws * DIM + i] = vg[i];
         }
-        for (int i = tid; i < D; i += kThreads) a.sp.win_phik[ws * D + i] = phk[i];
+        for (int i = tid; i < D; i += NT) a.sp.win_phik[ws * D + i] = phk[i];
+    }
+}
+
+// R_e = H^T phi_e - (phi_e . s) v_e and den_e = phi_e . s for every occupied
+// cache slot, from the current state (run before the first decode step that
+// follows a prefill).  Grid (streams, slot blocks of 32); H staged in smem.
+template <int DIM, int DH, typename TIn>
+__global__ void __launch_bounds__(256) residual_init_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int D = 2 * DH, SB = 32;
+    extern __shared__ __align__(16) float smem[];
+    const Dims& dm = a.dm;
+    const int st = blockIdx.x, lam = dm.lam;
+    const int n_g = min(lam, max(0, a.t - dm.eta));
+    const int e0 = blockIdx.y * SB;
+    if (e0 >= n_g) return;
+    const int ne = min(SB, n_g - e0);
+    float* Hs = smem;                  // [D][DIM]
+    float* ph = Hs + D * DIM;          // [SB][D]
+    float* ss = ph + SB * D;           // [D]
+    float* den = ss + D;               // [SB]
+    const size_t cbase = (size_t)st * lam;
+    for (int i = threadIdx.x; i < D * DIM / 4; i += 256)
+        reinterpret_cast<float4*>(Hs)[i] = reinterpret_cast<const float4*>(a.sp.H + (size_t)st * D * DIM)[i];
+    for (int i = threadIdx.x; i < D; i += 256) ss[i] = a.sp.s[(size_t)st * D + i];
+    for (int i = threadIdx.x; i < ne * D; i += 256) ph[i] = a.sp.cache_phik[(cbase + e0) * D + i];
+    __syncthreads();
+    for (int e = threadIdx.x >> 5; e < ne; e += 8) {
+        float x = 0.f;
+        for (int j = threadIdx.x & 31; j < D; j += 32) x = fmaf(ph[e * D + j], ss[j], x);
+        x = warp_sum(x);
+        if ((threadIdx.x & 31) == 0) { den[e] = x; a.sp.cache_den[cbase + e0 + e] = x; }
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < ne * DIM; idx += 256) {
+        const int e = idx / DIM, cc = idx % DIM;
+        float x = 0.f;
+        for (int j = 0; j < D; ++j) x = fmaf(ph[e * D + j], Hs[j * DIM + cc], x);
+        const float v = to_f32(((const TIn*)a.sp.cache_v)[(cbase + e0 + e) * DIM + cc]);
+        a.sp.cache_R[(cbase + e0 + e) * DIM + cc] = x - den[e] * v;
     }
 }
 
 template <int DIM, int DH, typename TIn>
-static cudaError_t launch_dec_t(const DecodeArgs& a, cudaStream_t s) {
-    const size_t bytes = (size_t)dec_offsets(DIM, DH, a.dm.Gq, a.dm.lam, a.dm.eta).total * 4;
+static cudaError_t launch_dec_t(const DecodeArgs& a0, cudaStream_t s) {
+    DecodeArgs a = a0;
+    // two CTAs per SM hide more memory latency than staging the residual rows would save
+    const int es = (int)sizeof(TIn);
+    a.r_smem = dec_offsets(DIM, DH, a.dm.Gq, a.dm.lam, a.dm.eta, true, es).total * 4 <= 100 * 1024 ? 1 : 0;
+    const size_t bytes = (size_t)dec_offsets(DIM, DH, a.dm.Gq, a.dm.lam, a.dm.eta, a.r_smem != 0, es).total * 4;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<DIM, DH, TIn>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
-    decode_kernel<DIM, DH, TIn><<<a.dm.S, kThreads, bytes, s>>>(a);
+    decode_kernel<DIM, DH, TIn><<<a.dm.S, kDecThreads, bytes, s>>>(a);
     return cudaGetLastError();
 }
 
-template <typename TIn>
-static cudaError_t launch_dec_d(const DecodeArgs& a, cudaStream_t s) {
-    const int d = a.dm.d, Dh = a.dm.Dh;
-    if (d == 64 && Dh == 32) return launch_dec_t<64, 32, TIn>(a, s);
-    if (d == 64 && Dh == 64) return launch_dec_t<64, 64, TIn>(a, s);
-    if (d == 128 && Dh == 32) return launch_dec_t<128, 32, TIn>(a, s);
-    if (d == 128 && Dh == 64) return launch_dec_t<128, 64, TIn>(a, s);
-    return cudaErrorInvalidValue;
+template <int DIM, int DH, typename TIn>
+static cudaError_t launch_rinit_t(const DecodeArgs& a, cudaStream_t s) {
+    constexpr int D = 2 * DH;
+    const size_t bytes = (size_t)(D * DIM + 32 * D + D + 32) * 4;
+    cudaError_t e = cudaFuncSetAttribute(residual_init_kernel<DIM, DH, TIn>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.dm.S, (a.dm.lam + 31) / 32);
+    residual_init_kernel<DIM, DH, TIn><<<grid, 256, bytes, s>>>(a);
+    return cudaGetLastError();
 }
+
+#define LOLA_DISPATCH_DIM(FN, a, s)                                              \
+    do {                                                                         \
+        const int d_ = (a).dm.d, Dh_ = (a).dm.Dh;                                \
+        if (d_ == 64 && Dh_ == 32) return FN<64, 32, TIn>(a, s);                \
+        if (d_ == 64 && Dh_ == 64) return FN<64, 64, TIn>(a, s);                \
+        if (d_ == 128 && Dh_ == 32) return FN<128, 32, TIn>(a, s);              \
+        if (d_ == 128 && Dh_ == 64) return FN<128, 64, TIn>(a, s);              \
+        return cudaErrorInvalidValue;                                            \
+    } while (0)
+
+template <typename TIn>
+static cudaError_t launch_dec_d(const DecodeArgs& a, cudaStream_t s) { LOLA_DISPATCH_DIM(launch_dec_t, a, s); }
+template <typename TIn>
+static cudaError_t launch_rinit_d(const DecodeArgs& a, cudaStream_t s) { LOLA_DISPATCH_DIM(launch_rinit_t, a, s); }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s) {
     return a.dm.dtype == 1 ? launch_dec_d<__nv_bfloat16>(a, s) : launch_dec_d<float>(a, s);
 }
 
-size_t decode_smem_bytes(const Dims& dm) {
-    return (size_t)dec_offsets(dm.d, dm.Dh, dm.Gq, dm.lam, dm.eta).total * 4;
+cudaError_t launch_residual_init(const DecodeArgs& a, cudaStream_t s) {
+    if (a.dm.lam == 0) return cudaSuccess;
+    return a.dm.dtype == 1 ? launch_rinit_d<__nv_bfloat16>(a, s) : launch_rinit_d<float>(a, s);
+}
+
+size_t decode_smem_bytes(const Dims& dm) {   // the smaller layout (residuals re-read from global)
+    return (size_t)dec_offsets(dm.d, dm.Dh, dm.Gq, dm.lam, dm.eta, false, dm.esize).total * 4;
 }
 
 }  // namespace lola

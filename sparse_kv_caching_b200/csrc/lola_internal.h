@@ -25,7 +25,7 @@ namespace lola {
 constexpr int kThreads = 512;
 
 struct Layout {            // byte offsets inside dev_buf (all 256-aligned)
-    size_t W, H, s, cache_k, cache_v, cache_phik, cache_pos, win_k, win_v, win_phik;
+    size_t W, H, s, cache_k, cache_v, cache_phik, cache_pos, win_k, win_v, win_phik, cache_R, cache_den;
     size_t phik_new, snap_pos, snap_H, snap_s, io_q, io_k, io_v, io_y, err;
     size_t total;
 };
@@ -47,6 +47,8 @@ struct StatePtrs {
     void* win_k;
     void* win_v;
     float* win_phik;
+    float* cache_R;        // [S][lambda][d]  H^T phi_e - den_e v_e (kept by decode)
+    float* cache_den;      // [S][lambda]     phi_e . s
 };
 
 struct PrefillArgs {
@@ -75,6 +77,7 @@ struct DecodeArgs {
     float* y;              // [B][Hq][d]
     int t;                 // position of the new token
     int* err;              // device error word
+    int r_smem;            // set by the launcher: residual rows fit in shared memory
 };
 
 // Launchers (each returns cudaGetLastError() of its launch).
@@ -84,6 +87,7 @@ cudaError_t launch_output(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_output_tc(const PrefillArgs& a, cudaStream_t s);   // bf16 on tcgen05
 cudaError_t launch_finalize(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_residual_init(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_clear(const Dims& dm, const StatePtrs& sp, cudaStream_t s);
 
 // Shared-memory bytes a scan CTA needs (0 if the shape is unsupported).
