@@ -20,6 +20,7 @@
 #include <cooperative_groups.h>
 
 #include "device_common.cuh"
+#include "umma.cuh"
 
 namespace lola {
 
@@ -275,334 +276,557 @@ __global__ void __launch_bounds__(kThreads, 1) scan_kernel(PrefillArgs a) {
 // ---------------------------------------------------------------------------
 // The same chain split over a thread-block cluster (one cluster per stream).
 //
-// CTA r of the cluster owns columns [r*CW, (r+1)*CW) of H.  Every CTA keeps
-// the phi rows (and its columns of the value rows) of all cache members
-// resident in shared memory, so a block only loads its C newcomers.  Per
-// scored block each CTA computes the partial SRE of every candidate over its
-// own columns; the partials are summed across the cluster through distributed
-// shared memory in a fixed rank order, so every CTA holds bit-identical scores
-// and takes the same (replicated) top-lambda decision; each CTA then folds
-// into its own columns and publishes its rows of H_c^T.
+// CTA r of the cluster owns columns [r*CW, (r+1)*CW) of H.  Every CTA keeps the
+// phi rows, and its slice of the value rows, of the cache members in a pool of
+// lambda + C shared-memory rows: a slot names a pool row, so a newcomer that
+// enters the cache never moves, and the rows of folded pairs go back to a free
+// stack from which the next block's newcomers are fetched with cp.async while
+// the current block finishes.  Per scored block each CTA computes the partial
+// SRE of every candidate over its own columns (cache members first, while the
+// newcomers land); the partials are summed across the cluster through
+// distributed shared memory by a fixed butterfly, so every CTA holds
+// bit-identical scores and takes the same top-lambda decision (one warp selects
+// and does the slot bookkeeping); each CTA then folds into its own columns and
+// publishes its rows of H_c^T straight from registers.
 // ---------------------------------------------------------------------------
 constexpr int kClThreads = 256;
 
 struct ClOffsets {
-    int Hs, ss, phiC, vC, phiL, vL, part, den, score, slot_pos, cand_pos, flags, ranks, keep, free_slots,
-        fold_list, tmp, hist, sbits, eq_list, newslot, sfold, total;
+    int Hs, ss, phi, vv, part, xbuf, score, cand_pos, cand_row, keep, slot_pos, slot_row, new_row, free_rows,
+        fold_row, free_slots, hist, tmp, eq_list, total;
 };
 
 __host__ __device__ inline ClOffsets cl_offsets(int D, int CW, int lam, int C, int esize) {
-    const int NMAX = lam + C, LD = D + 4;
+    const int P = lam + C, LD = D + 4, N4 = (P + 3) & ~3;
     ClOffsets o;
     int p = 0;
     auto take = [&](int n) { int r = p; p += (n + 3) & ~3; return r; };
     o.Hs = take(D * CW);
     o.ss = take(D);
-    o.phiC = take(lam * LD);
-    o.vC = take((lam * CW * esize + 3) / 4);
-    o.phiL = take(C * LD);
-    o.vL = take((C * CW * esize + 3) / 4);
-    o.part = take(2 * NMAX);
-    o.den = take(NMAX);
-    o.score = take(NMAX);
+    o.phi = take(P * LD);
+    o.vv = take((P * CW * esize + 3) / 4);
+    o.part = take(2 * N4);
+    o.xbuf = take(3 * kClThreads);
+    o.score = take(N4);
+    o.cand_pos = take(P);
+    o.cand_row = take(P);
+    o.keep = take(P);
     o.slot_pos = take(lam + 1);
-    o.cand_pos = take(NMAX);
-    o.flags = take(NMAX);
-    o.ranks = take(NMAX);
-    o.keep = take(NMAX);
+    o.slot_row = take(lam + 1);
+    o.new_row = take(C);
+    o.free_rows = take(P);
+    o.fold_row = take(P);
     o.free_slots = take(lam + 1);
-    o.fold_list = take(NMAX);
-    o.tmp = take(64);
     o.hist = take(256);
-    o.sbits = take(NMAX);
-    o.eq_list = take(NMAX);
-    o.newslot = take(C);
-    o.sfold = take(2 * C);
+    o.tmp = take(32);
+    o.eq_list = take(P);
     o.total = p;
     return o;
 }
 
-template <int CW>
-struct ClShape {
-    static constexpr int TX = CW / 4;                          // threads across the CTA's columns
-    static constexpr int TY = kClThreads / TX;
-    static constexpr int EPT = CW >= 64 ? 8 : (CW == 32 ? 8 : (CW == 16 ? 4 : 2));
-    static constexpr int TE = TY * EPT;                        // candidates per pass
+// Selection and slot bookkeeping of one scored block, by one full warp (the same
+// in every CTA of a cluster).  Candidate e (members e < n_g in slot order, then
+// the n_l newcomers in position order) is held by lane e % 32 as bit e / 32 of
+// its registers.  Top-lambda by (score, -position): MSB radix passes of 8 bits
+// over the fp32 score bits (scores are >= 0, so the bit pattern orders like the
+// value) narrow the threshold to a bucket of candidates sharing a bit prefix;
+// once the bucket is small (or the bits are exhausted) its members are ranked
+// exactly by (bits descending, position ascending).  Then: kept newcomers take,
+// in position order, the freed slots (evicted members and never-used slots) in
+// slot order; the folded set is listed by pool row and its rows return to the
+// free stack.  Returns the number of folded pairs.
+template <int KMAX>
+__device__ int select_and_place(const float* score, const int* cand_pos, const int* cand_row, int n, int n_g,
+                                int n_l, int lam, int l_lo, const int* new_row, int* slot_row, int* slot_pos,
+                                int* fold_row, int* free_rows, int nfree, int P, int* free_slots, unsigned* hist,
+                                int* eq_list, int* eq_keep) {
+    const int lane = threadIdx.x & 31;
+    const unsigned lt = (1u << lane) - 1u;
+    unsigned u[KMAX];
+    int crow[KMAX];
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+        const int e = 32 * k + lane;
+        u[k] = e < n ? __float_as_uint(score[e]) : 0u;
+        crow[k] = e < n ? cand_row[e] : 0;
+    }
+    unsigned keepm = 0u;
+    if (lam > 0) {
+        unsigned prefix = 0u, mask = 0u;
+        int kk = lam, cnt = n;             // still to keep from the bucket; bucket size
+        for (int shift = 24; shift >= 0 && cnt > 32 && cnt > kk; shift -= 8) {
+            for (int i = lane; i < 256; i += 32) hist[i] = 0u;
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k)
+                if (32 * k + lane < n && (u[k] & mask) == prefix) atomicAdd(&hist[(u[k] >> shift) & 255u], 1u);
+            __syncwarp();
+            unsigned c[8], lsum = 0u;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) { c[t] = hist[lane * 8 + t]; lsum += c[t]; }
+            unsigned suf = lsum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned y = __shfl_down_sync(0xffffffffu, suf, o);
+                if (lane + o < 32) suf += y;
+            }
+            unsigned above = suf - lsum;   // candidates in higher digits (higher lanes)
+            int hit = -1;
+            unsigned h_above = 0u, h_cnt = 0u;
+#pragma unroll
+            for (int t = 7; t >= 0; --t) {
+                if (above < (unsigned)kk && (unsigned)kk <= above + c[t]) { hit = t; h_above = above; h_cnt = c[t]; }
+                above += c[t];
+            }
+            const int src = __ffs(__ballot_sync(0xffffffffu, hit >= 0)) - 1;
+            const int digit = __shfl_sync(0xffffffffu, lane * 8 + hit, src);
+            kk -= (int)__shfl_sync(0xffffffffu, h_above, src);
+            cnt = (int)__shfl_sync(0xffffffffu, h_cnt, src);
+            prefix |= (unsigned)digit << shift;
+            mask |= 255u << shift;
+            __syncwarp();
+        }
+        // above the bucket: kept; the bucket is listed in candidate order
+        unsigned inbm = 0u;
+        int base = 0;
+#pragma unroll
+        for (int k = 0; k < KMAX; ++k) {
+            const bool valid = 32 * k + lane < n;
+            const unsigned m = u[k] & mask;
+            if (valid && m > prefix) keepm |= 1u << k;
+            const bool inb = valid && m == prefix;
+            if (inb) inbm |= 1u << k;
+            const unsigned b = __ballot_sync(0xffffffffu, inb);
+            if (inb) eq_list[base + __popc(b & lt)] = 32 * k + lane;
+            base += __popc(b);
+        }
+        if (cnt == kk) {
+            keepm |= inbm;
+        } else {
+            __syncwarp();
+            if (cnt <= 32) {               // one member per lane; compare through shuffles
+                const int i = lane < cnt ? eq_list[lane] : 0;
+                const unsigned ui = __float_as_uint(score[i]);
+                const int pi = cand_pos[i];
+                int r = 0;
+                for (int z = 0; z < cnt; ++z) {
+                    const unsigned w = __shfl_sync(0xffffffffu, ui, z);
+                    const int pz = __shfl_sync(0xffffffffu, pi, z);
+                    r += (w > ui || (w == ui && pz < pi)) ? 1 : 0;
+                }
+                if (lane < cnt) eq_keep[lane] = r < kk ? 1 : 0;
+            } else {                       // exact ties over many candidates
+                for (int q = lane; q < cnt; q += 32) {
+                    const int i = eq_list[q];
+                    const unsigned ui = __float_as_uint(score[i]);
+                    const int pi = cand_pos[i];
+                    int r = 0;
+                    for (int z = 0; z < cnt; ++z) {
+                        const int j = eq_list[z];
+                        const unsigned w = __float_as_uint(score[j]);
+                        r += (w > ui || (w == ui && cand_pos[j] < pi)) ? 1 : 0;
+                    }
+                    eq_keep[q] = r < kk ? 1 : 0;
+                }
+            }
+            __syncwarp();
+            base = 0;                      // each owner collects its bucket members' decisions
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k) {
+                const bool inb = (inbm >> k) & 1u;
+                const unsigned b = __ballot_sync(0xffffffffu, inb);
+                if (inb && eq_keep[base + __popc(b & lt)]) keepm |= 1u << k;
+                base += __popc(b);
+            }
+        }
+    }
+    // freed slots, in slot order (member e sits in slot e)
+    int base = 0;
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+        const int j = 32 * k + lane;
+        const bool f = j < lam && (j >= n_g || ((keepm >> k) & 1u) == 0u);
+        const unsigned b = __ballot_sync(0xffffffffu, f);
+        if (f) free_slots[base + __popc(b & lt)] = j;
+        base += __popc(b);
+    }
+    const int n_free_slots = base;
+    __syncwarp();
+    // kept newcomers, in position order, take them in order
+    base = 0;
+    for (int i0 = 0; i0 < n_l; i0 += 32) {
+        const int i = i0 + lane;
+        const int e = min(n_g + i, n - 1);
+        const unsigned km = __shfl_sync(0xffffffffu, keepm, e & 31);
+        const bool kept = i < n_l && ((km >> (e >> 5)) & 1u);
+        const unsigned b = __ballot_sync(0xffffffffu, kept);
+        const int fs = base + __popc(b & lt);
+        if (kept && fs < n_free_slots) {             // always true when exactly lam are kept
+            const int sl = free_slots[fs];
+            slot_row[sl] = new_row[i];
+            slot_pos[sl] = l_lo + i;
+        }
+        base += __popc(b);
+    }
+    // the folded set S = E \ G_new, by pool row; the rows return to the free stack
+    base = 0;
+#pragma unroll
+    for (int k = 0; k < KMAX; ++k) {
+        const bool f = 32 * k + lane < n && ((keepm >> k) & 1u) == 0u;
+        const unsigned b = __ballot_sync(0xffffffffu, f);
+        const int q = base + __popc(b & lt);
+        if (f && nfree + q < P) {                    // always true when exactly lam are kept
+            fold_row[q] = crow[k];
+            free_rows[nfree + q] = crow[k];
+        }
+        base += __popc(b);
+    }
+    return min(base, P - nfree);
+}
+
+// Largest lambda + C the cluster scan handles (candidates held 32 per register).
+template <int D>
+struct ClMax {
+    static constexpr int KMAX = D == 128 ? 14 : 28;
+    static constexpr int NMAX = 32 * KMAX;
 };
 
-template <int D, int CW, typename TIn>
+template <int D, int DV, int NCL, typename TIn>
 __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_constant__ PrefillArgs a) {
     namespace cg = cooperative_groups;
-    using Sh = ClShape<CW>;
-    constexpr int NT = kClThreads, LD = D + 4;
+    constexpr int CW = DV / NCL, NT = kClThreads, NW = NT / 32, LD = D + 4;
+    constexpr int TX = CW / 4, TY = NT / TX;                  // SRE threads: columns x candidates
+    constexpr int EPT = CW >= 32 ? 8 : (CW == 16 ? 4 : 2);
+    constexpr int TE = TY * EPT;                              // candidates per SRE pass
+    constexpr int VCH = CW * (int)sizeof(TIn) / 16;           // 16-byte pieces of a value slice
+    static_assert(CW >= 8 && CW <= 64 && (CW * sizeof(TIn)) % 16 == 0 && VCH <= 32, "unsupported column split");
+    static_assert(32 % NCL == 0, "butterfly groups must tile a warp");
     cg::cluster_group cluster = cg::this_cluster();
-    const int NCL = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
     extern __shared__ __align__(16) float smem[];
     const Dims& dm = a.dm;
-    const int lam = dm.lam, C = dm.C, eta = dm.eta, DV = dm.d, NMAX = lam + C;
+    const int lam = dm.lam, C = dm.C, eta = dm.eta, P = lam + C, N4 = (P + 3) & ~3;
     const int st = blockIdx.x / NCL, b = st / dm.Hkv, g = st % dm.Hkv;
     const int col0 = rank * CW;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const ClOffsets o = cl_offsets(D, CW, lam, C, (int)sizeof(TIn));
     float* Hs = smem + o.Hs;                                   // [D][CW]
-    float* ss = smem + o.ss;
-    float* phiC = smem + o.phiC;                               // [lam][LD]
-    TIn* vC = reinterpret_cast<TIn*>(smem + o.vC);             // [lam][CW]
-    float* phiL = smem + o.phiL;                               // [C][LD]
-    TIn* vL = reinterpret_cast<TIn*>(smem + o.vL);             // [C][CW]
-    float* part = smem + o.part;                               // [2][NMAX]
-    float* den = smem + o.den;
+    float* ss = smem + o.ss;                                   // [D]
+    float* phi = smem + o.phi;                                 // pool [P][LD]
+    TIn* vv = reinterpret_cast<TIn*>(smem + o.vv);             // pool [P][CW]
+    float* part = smem + o.part;                               // [2][N4] partial SRE
+    float* xbuf = smem + o.xbuf;                               // split-D exchange of the newcomer pass
     float* score = smem + o.score;
-    int* slot_pos = reinterpret_cast<int*>(smem + o.slot_pos);
     int* cand_pos = reinterpret_cast<int*>(smem + o.cand_pos);
-    int* flags = reinterpret_cast<int*>(smem + o.flags);
-    int* ranks = reinterpret_cast<int*>(smem + o.ranks);
+    int* cand_row = reinterpret_cast<int*>(smem + o.cand_row);
     int* keep = reinterpret_cast<int*>(smem + o.keep);
+    int* slot_pos = reinterpret_cast<int*>(smem + o.slot_pos);
+    int* slot_row = reinterpret_cast<int*>(smem + o.slot_row);
+    int* new_row = reinterpret_cast<int*>(smem + o.new_row);
+    int* free_rows = reinterpret_cast<int*>(smem + o.free_rows);
+    int* fold_row = reinterpret_cast<int*>(smem + o.fold_row);
     int* free_slots = reinterpret_cast<int*>(smem + o.free_slots);
-    int* fold_list = reinterpret_cast<int*>(smem + o.fold_list);
-    int* tmp = reinterpret_cast<int*>(smem + o.tmp);
     unsigned* hist = reinterpret_cast<unsigned*>(smem + o.hist);
-    unsigned* sbits = reinterpret_cast<unsigned*>(smem + o.sbits);
+    int* tmp = reinterpret_cast<int*>(smem + o.tmp);
     int* eq_list = reinterpret_cast<int*>(smem + o.eq_list);
-    int* newslot = reinterpret_cast<int*>(smem + o.newslot);
-    float* sfold = smem + o.sfold;                             // fold staging: row offsets, values
 
-    // ---- load the state: own columns of H, s, slot positions, resident rows ----
+    // cp.async the phi rows and this CTA's value slices of n_rows pairs into pool rows
+    auto fetch = [&](int n_rows, auto pos_of, auto slot_of, auto row_of) {
+        for (int i = warp; i < n_rows; i += NW) {                 // a warp per row
+            const PairRef<TIn> r = pair_ref<TIn>(a, st, b, g, pos_of(i), slot_of(i));
+            const int row = row_of(i);
+            for (int q = lane; q < D / 4; q += 32) umma::cp_async16(phi + (size_t)row * LD + 4 * q, r.phik + 4 * q);
+            if (lane < VCH)
+                umma::cp_async16(reinterpret_cast<char*>(vv + (size_t)row * CW) + 16 * lane,
+                                 reinterpret_cast<const char*>(r.v + col0) + 16 * lane);
+        }
+        umma::cp_async_commit();
+    };
+
+    // ---- state: own columns of H, s, slots, resident rows ----
     const float* Hg = a.sp.H + (size_t)st * D * DV;
-    for (int i = tid; i < D * CW; i += NT) Hs[i] = Hg[(size_t)(i / CW) * DV + col0 + i % CW];
-    for (int i = tid; i < D; i += NT) ss[i] = a.sp.s[(size_t)st * D + i];
-    for (int j = tid; j < lam; j += NT) slot_pos[j] = a.sp.cache_pos[(size_t)st * lam + j];
-    __syncthreads();
+    for (int i = tid; i < D * (CW / 4); i += NT) {
+        const int j = i / (CW / 4), u = i % (CW / 4);
+        umma::cp_async16(Hs + j * CW + 4 * u, Hg + (size_t)j * DV + col0 + 4 * u);
+    }
+    for (int i = tid; i < D / 4; i += NT) umma::cp_async16(ss + 4 * i, a.sp.s + (size_t)st * D + 4 * i);
     const int n_g0 = min(lam, max(0, a.t_start - eta));
-    for (int idx = tid; idx < n_g0 * (D / 4); idx += NT) {
-        const int e = idx / (D / 4), j4 = (idx % (D / 4)) * 4;
-        const PairRef<TIn> r = pair_ref<TIn>(a, st, b, g, slot_pos[e], e);
-        *reinterpret_cast<float4*>(phiC + e * LD + j4) = *reinterpret_cast<const float4*>(r.phik + j4);
+    for (int j = tid; j < lam; j += NT) {
+        slot_pos[j] = a.sp.cache_pos[(size_t)st * lam + j];
+        slot_row[j] = j;
     }
-    for (int idx = tid; idx < n_g0 * CW; idx += NT) {
-        const int e = idx / CW, cl = idx % CW;
-        vC[e * CW + cl] = pair_ref<TIn>(a, st, b, g, slot_pos[e], e).v[col0 + cl];
-    }
+    for (int k = tid; k < P - n_g0; k += NT) free_rows[k] = P - 1 - k;      // popped from the top
+    int nfree = P - n_g0;
+    __syncthreads();
+    fetch(n_g0, [&](int i) { return slot_pos[i]; }, [](int i) { return i; }, [](int i) { return i; });
+
+    // the newcomers of block c (the pairs leaving the window) into rows from the free stack;
+    // always commits one cp.async group
+    auto prefetch = [&](int c) {
+        int n_l = 0, l_lo = 0;
+        if (c < a.nc) {
+            const int t0 = a.t_start + c * C;
+            l_lo = max(0, t0 - eta);
+            n_l = max(0, t0 + C - eta) - l_lo;
+        }
+        for (int i = tid; i < n_l; i += NT) new_row[i] = free_rows[nfree - 1 - i];
+        fetch(n_l, [&](int i) { return l_lo + i; }, [](int) { return 0; },
+              [&](int i) { return free_rows[nfree - 1 - i]; });
+        nfree -= n_l;
+    };
+    prefetch(0);
 
     const size_t snaps = (size_t)dm.nc_max + 1;
-    auto publish = [&](int c) {
-        float* sH = a.snap_H + ((size_t)st * snaps + c) * D * DV;          // H_c^T [DV][D]
-        for (int i = tid; i < CW * (D / 4); i += NT) {
-            const int cl = i / (D / 4), j4 = (i % (D / 4)) * 4;
-            reinterpret_cast<float4*>(sH + (size_t)(col0 + cl) * D)[j4 / 4] =
-                make_float4(Hs[(j4 + 0) * CW + cl], Hs[(j4 + 1) * CW + cl], Hs[(j4 + 2) * CW + cl],
-                            Hs[(j4 + 3) * CW + cl]);
-        }
-        if (rank == 0) {
-            int* sp_ = a.snap_pos + ((size_t)st * snaps + c) * lam;
+    auto snapH = [&](int c) { return a.snap_H + ((size_t)st * snaps + c) * D * DV; };   // H_c^T [DV][D]
+    // slot positions by slices across the cluster, s by rank 0
+    auto publish_pos_s = [&](int c, bool with_s) {
+        int* sp_ = a.snap_pos + ((size_t)st * snaps + c) * lam;
+        for (int j = rank * NT + tid; j < lam; j += NCL * NT) sp_[j] = slot_pos[j];
+        if (with_s && rank == 0) {
             float* sS = a.snap_s + ((size_t)st * snaps + c) * D;
-            for (int j = tid; j < lam; j += NT) sp_[j] = slot_pos[j];
             for (int i = tid; i < D; i += NT) sS[i] = ss[i];
         }
     };
+    auto publish_H = [&](int c) {
+        float* sH = snapH(c);
+        for (int i = tid; i < D * (CW / 4); i += NT) {
+            const int j = i % D, u = i / D;
+            const float4 h = *reinterpret_cast<const float4*>(Hs + j * CW + 4 * u);
+            float* dst = sH + (size_t)(col0 + 4 * u) * D + j;
+            dst[0] = h.x; dst[D] = h.y; dst[2 * D] = h.z; dst[3 * D] = h.w;
+        }
+    };
+    umma::cp_async_wait<1>();                                  // state and resident rows landed
     __syncthreads();
-    publish(0);
+    publish_H(0);
+    publish_pos_s(0, true);
+
+    // Partial SRE over this CTA's columns (notes §2.3, Eq. 10): for each candidate,
+    // den_e = phi_e . s and pred = H^T phi_e restricted to the CTA's columns are
+    // accumulated in one pass over phi_e; the partial is || pred / den_e - v_e ||^2
+    // over those columns (the zero prediction when den_e == 0).  Every thread of a
+    // tile works (out-of-range candidates repeat a valid row and are not stored),
+    // so the inner loop has no branches and its loads pipeline.
+    auto finish = [&](int e, bool ok, const float (&acc)[4], float dn, int tx, float* mypart, bool store) {
+        float pt = 0.f;
+        if (ok) {
+            const TIn* vr = vv + (size_t)cand_row[e] * CW + 4 * tx;
+            float pr[4] = {0.f, 0.f, 0.f, 0.f};
+            if (dn > 0.f) {
+                const float rdn = 1.f / dn;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) pr[u] = acc[u] * rdn;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) { const float r = pr[u] - to_f32(vr[u]); pt = fmaf(r, r, pt); }
+        }
+#pragma unroll
+        for (int off = TX / 2; off > 0; off >>= 1) pt += __shfl_xor_sync(0xffffffffu, pt, off);
+        if (store && ok && tx == 0) mypart[e] = pt;
+    };
+    // cache members: thread (tx, ty) takes columns 4tx..4tx+3 of EPT candidates
+    auto sre_members = [&](int e_lo, int e_hi, float* mypart) {
+        const int tx = tid % TX, ty = tid / TX;
+        for (int e0 = e_lo; e0 < e_hi; e0 += TE) {
+            float acc[EPT][4], d0[EPT], d1[EPT];
+            const float* rows[EPT];
+#pragma unroll
+            for (int i = 0; i < EPT; ++i) {
+                acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+                d0[i] = d1[i] = 0.f;
+                rows[i] = phi + (size_t)cand_row[min(e0 + ty + i * TY, e_hi - 1)] * LD;
+            }
+#pragma unroll 2
+            for (int j = 0; j < D; j += 4) {
+                const float4 h0 = *reinterpret_cast<const float4*>(Hs + (j + 0) * CW + 4 * tx);
+                const float4 h1 = *reinterpret_cast<const float4*>(Hs + (j + 1) * CW + 4 * tx);
+                const float4 h2 = *reinterpret_cast<const float4*>(Hs + (j + 2) * CW + 4 * tx);
+                const float4 h3 = *reinterpret_cast<const float4*>(Hs + (j + 3) * CW + 4 * tx);
+                const float4 s4 = *reinterpret_cast<const float4*>(ss + j);
+#pragma unroll
+                for (int i = 0; i < EPT; ++i) {
+                    const float4 f = *reinterpret_cast<const float4*>(rows[i] + j);
+                    acc[i][0] = fmaf(f.x, h0.x, acc[i][0]); acc[i][1] = fmaf(f.x, h0.y, acc[i][1]);
+                    acc[i][2] = fmaf(f.x, h0.z, acc[i][2]); acc[i][3] = fmaf(f.x, h0.w, acc[i][3]);
+                    acc[i][0] = fmaf(f.y, h1.x, acc[i][0]); acc[i][1] = fmaf(f.y, h1.y, acc[i][1]);
+                    acc[i][2] = fmaf(f.y, h1.z, acc[i][2]); acc[i][3] = fmaf(f.y, h1.w, acc[i][3]);
+                    acc[i][0] = fmaf(f.z, h2.x, acc[i][0]); acc[i][1] = fmaf(f.z, h2.y, acc[i][1]);
+                    acc[i][2] = fmaf(f.z, h2.z, acc[i][2]); acc[i][3] = fmaf(f.z, h2.w, acc[i][3]);
+                    acc[i][0] = fmaf(f.w, h3.x, acc[i][0]); acc[i][1] = fmaf(f.w, h3.y, acc[i][1]);
+                    acc[i][2] = fmaf(f.w, h3.z, acc[i][2]); acc[i][3] = fmaf(f.w, h3.w, acc[i][3]);
+                    d0[i] = fmaf(f.x, s4.x, d0[i]); d1[i] = fmaf(f.y, s4.y, d1[i]);
+                    d0[i] = fmaf(f.z, s4.z, d0[i]); d1[i] = fmaf(f.w, s4.w, d1[i]);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < EPT; ++i) {
+                const int e = e0 + ty + i * TY;
+                finish(e, e < e_hi, acc[i], d0[i] + d1[i], tx, mypart, true);
+            }
+        }
+    };
+    // newcomers: the sum over D is split in KS parts so that a block of C candidates
+    // still occupies every thread; the parts meet in shared memory
+    constexpr int KS = (NT / (TX * 64) >= 2) ? 2 : 1;
+    constexpr int TB = NT / (TX * KS), DK = D / KS;
+    auto sre_new = [&](int e_lo, int e_hi, float* mypart) {
+        const int tx = tid % TX, ks = (tid / TX) % KS, tb = tid / (TX * KS);
+        for (int e0 = e_lo; e0 < e_hi; e0 += TB) {
+            const int e = e0 + tb;
+            const float* row = phi + (size_t)cand_row[min(e, e_hi - 1)] * LD + ks * DK;
+            const float* hb = Hs + (size_t)(ks * DK) * CW + 4 * tx;
+            const float* sb = ss + ks * DK;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f}, d0 = 0.f, d1 = 0.f;
+#pragma unroll 4
+            for (int j = 0; j < DK; j += 4) {
+                const float4 f = *reinterpret_cast<const float4*>(row + j);
+                const float4 h0 = *reinterpret_cast<const float4*>(hb + (j + 0) * CW);
+                const float4 h1 = *reinterpret_cast<const float4*>(hb + (j + 1) * CW);
+                const float4 h2 = *reinterpret_cast<const float4*>(hb + (j + 2) * CW);
+                const float4 h3 = *reinterpret_cast<const float4*>(hb + (j + 3) * CW);
+                const float4 s4 = *reinterpret_cast<const float4*>(sb + j);
+                acc[0] = fmaf(f.x, h0.x, acc[0]); acc[1] = fmaf(f.x, h0.y, acc[1]);
+                acc[2] = fmaf(f.x, h0.z, acc[2]); acc[3] = fmaf(f.x, h0.w, acc[3]);
+                acc[0] = fmaf(f.y, h1.x, acc[0]); acc[1] = fmaf(f.y, h1.y, acc[1]);
+                acc[2] = fmaf(f.y, h1.z, acc[2]); acc[3] = fmaf(f.y, h1.w, acc[3]);
+                acc[0] = fmaf(f.z, h2.x, acc[0]); acc[1] = fmaf(f.z, h2.y, acc[1]);
+                acc[2] = fmaf(f.z, h2.z, acc[2]); acc[3] = fmaf(f.z, h2.w, acc[3]);
+                acc[0] = fmaf(f.w, h3.x, acc[0]); acc[1] = fmaf(f.w, h3.y, acc[1]);
+                acc[2] = fmaf(f.w, h3.z, acc[2]); acc[3] = fmaf(f.w, h3.w, acc[3]);
+                d0 = fmaf(f.x, s4.x, d0); d1 = fmaf(f.y, s4.y, d1);
+                d0 = fmaf(f.z, s4.z, d0); d1 = fmaf(f.w, s4.w, d1);
+            }
+            if constexpr (KS == 2) {
+                float* xb = xbuf + (tb * TX + tx) * 6;
+                if (ks == 1) { xb[0] = acc[0]; xb[1] = acc[1]; xb[2] = acc[2]; xb[3] = acc[3]; xb[4] = d0; xb[5] = d1; }
+                __syncthreads();
+                if (ks == 0) {
+                    acc[0] += xb[0]; acc[1] += xb[1]; acc[2] += xb[2]; acc[3] += xb[3]; d0 += xb[4]; d1 += xb[5];
+                }
+            }
+            finish(e, e < e_hi && ks == 0, acc, d0 + d1, tx, mypart, true);
+            if (KS == 2 && e0 + TB < e_hi) __syncthreads();     // the exchange buffer is reused
+        }
+    };
 
     int pb = 0;
-    const int tx = tid % Sh::TX, ty = tid / Sh::TX;
     for (int c = 0; c < a.nc; ++c) {
         const int t0 = a.t_start + c * C;
         const int n_g = min(lam, max(0, t0 - eta));
-        const int l_lo = max(0, t0 - eta), l_hi = max(0, t0 + C - eta);
-        const int n_l = l_hi - l_lo;
-        if (n_l > 0) {
-            // newcomers (the pairs leaving the window): phi rows and own value columns
-            for (int idx = tid; idx < n_l * (D / 4); idx += NT) {
-                const int i = idx / (D / 4), j4 = (idx % (D / 4)) * 4;
-                const PairRef<TIn> r = pair_ref<TIn>(a, st, b, g, l_lo + i, 0);
-                *reinterpret_cast<float4*>(phiL + i * LD + j4) = *reinterpret_cast<const float4*>(r.phik + j4);
+        const int l_lo = max(0, t0 - eta), n_l = max(0, t0 + C - eta) - l_lo;
+        const int n = n_g + n_l;
+        const bool scored = n_l > 0 && n > lam;
+        if (n_l > 0 && !scored) {
+            // every candidate fits: all newcomers join, in their pool rows (notes §2.4)
+            for (int i = tid; i < n_l; i += NT) {
+                slot_row[n_g + i] = new_row[i];
+                slot_pos[n_g + i] = l_lo + i;
             }
-            for (int idx = tid; idx < n_l * CW; idx += NT) {
-                const int i = idx / CW, cl = idx % CW;
-                vL[i * CW + cl] = pair_ref<TIn>(a, st, b, g, l_lo + i, 0).v[col0 + cl];
+        } else if (scored) {
+            for (int e = tid; e < n; e += NT) {
+                cand_pos[e] = e < n_g ? slot_pos[e] : l_lo + (e - n_g);
+                cand_row[e] = e < n_g ? slot_row[e] : new_row[e - n_g];
             }
             __syncthreads();
-            if (n_g + n_l <= lam) {
-                // every candidate fits: all newcomers join (notes §2.4)
-                for (int idx = tid; idx < n_l * (D / 4); idx += NT) {
-                    const int i = idx / (D / 4), j4 = (idx % (D / 4)) * 4;
-                    *reinterpret_cast<float4*>(phiC + (n_g + i) * LD + j4) =
-                        *reinterpret_cast<const float4*>(phiL + i * LD + j4);
-                }
-                for (int idx = tid; idx < n_l * CW; idx += NT) vC[n_g * CW + idx] = vL[idx];
-                for (int i = tid; i < n_l; i += NT) slot_pos[n_g + i] = l_lo + i;
-            } else {
-                const int n = n_g + n_l;
-                for (int i = tid; i < n; i += NT) cand_pos[i] = i < n_g ? slot_pos[i] : l_lo + (i - n_g);
-                auto phirow = [&](int e) -> const float* { return e < n_g ? phiC + e * LD : phiL + (e - n_g) * LD; };
-                auto vrow = [&](int e) -> const TIn* { return e < n_g ? vC + e * CW : vL + (e - n_g) * CW; };
-                // den_e = phi_e . s (replicated in every CTA; one thread per candidate)
-                for (int e = tid; e < n; e += NT) {
-                    const float* pr = phirow(e);
-                    float x = 0.f;
-#pragma unroll 8
-                    for (int j = 0; j < D; j += 4) {
-                        const float4 f = *reinterpret_cast<const float4*>(pr + j);
-                        const float4 t = *reinterpret_cast<const float4*>(ss + j);
-                        x = fmaf(f.x, t.x, x); x = fmaf(f.y, t.y, x); x = fmaf(f.z, t.z, x); x = fmaf(f.w, t.w, x);
-                    }
-                    den[e] = x;
-                }
-                __syncthreads();
-                // partial SRE over the CTA's columns
-                float* mypart = part + pb * NMAX;
-                for (int e0 = 0; e0 < n; e0 += Sh::TE) {
-                    float acc[Sh::EPT][4];
-                    const float* rows[Sh::EPT];
+            float* mypart = part + pb * N4;
+            if (lam > 0) sre_members(0, n_g, mypart);           // members are resident
+            umma::cp_async_wait<0>();                          // the newcomers have landed
+            __syncthreads();
+            if (lam > 0) {
+                sre_new(n_g, n, mypart);
+                cluster.sync();                                // partials visible cluster-wide
+                // score_e = sum of the cluster's partials, by a butterfly over NCL lanes
+                constexpr int GPW = 32 / NCL, KB = 4;
+                const int r = lane % NCL, gs = lane / NCL;
+                const float4* src = reinterpret_cast<const float4*>(cluster.map_shared_rank(mypart, r));
+                const int G4 = (n + 3) / 4;
+                for (int gw = warp * GPW; gw < G4; gw += KB * NW * GPW) {     // warp-uniform trip count
+                    float4 x[KB];
 #pragma unroll
-                    for (int i = 0; i < Sh::EPT; ++i) {
-                        acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-                        const int e = e0 + ty + i * Sh::TY;
-                        rows[i] = phirow(e < n ? e : 0);
+                    for (int k = 0; k < KB; ++k) {
+                        const int gi = gw + k * NW * GPW + gs;
+                        x[k] = gi < G4 ? src[gi] : make_float4(0.f, 0.f, 0.f, 0.f);
                     }
-                    for (int j = 0; j < D; j += 4) {
-                        const float4 h0 = *reinterpret_cast<const float4*>(Hs + (j + 0) * CW + 4 * tx);
-                        const float4 h1 = *reinterpret_cast<const float4*>(Hs + (j + 1) * CW + 4 * tx);
-                        const float4 h2 = *reinterpret_cast<const float4*>(Hs + (j + 2) * CW + 4 * tx);
-                        const float4 h3 = *reinterpret_cast<const float4*>(Hs + (j + 3) * CW + 4 * tx);
 #pragma unroll
-                        for (int i = 0; i < Sh::EPT; ++i) {
-                            if (e0 + i * Sh::TY >= n) break;       // CTA-uniform: no candidate in this slot
-                            const float4 f = *reinterpret_cast<const float4*>(rows[i] + j);
-                            acc[i][0] = fmaf(f.x, h0.x, acc[i][0]); acc[i][1] = fmaf(f.x, h0.y, acc[i][1]);
-                            acc[i][2] = fmaf(f.x, h0.z, acc[i][2]); acc[i][3] = fmaf(f.x, h0.w, acc[i][3]);
-                            acc[i][0] = fmaf(f.y, h1.x, acc[i][0]); acc[i][1] = fmaf(f.y, h1.y, acc[i][1]);
-                            acc[i][2] = fmaf(f.y, h1.z, acc[i][2]); acc[i][3] = fmaf(f.y, h1.w, acc[i][3]);
-                            acc[i][0] = fmaf(f.z, h2.x, acc[i][0]); acc[i][1] = fmaf(f.z, h2.y, acc[i][1]);
-                            acc[i][2] = fmaf(f.z, h2.z, acc[i][2]); acc[i][3] = fmaf(f.z, h2.w, acc[i][3]);
-                            acc[i][0] = fmaf(f.w, h3.x, acc[i][0]); acc[i][1] = fmaf(f.w, h3.y, acc[i][1]);
-                            acc[i][2] = fmaf(f.w, h3.z, acc[i][2]); acc[i][3] = fmaf(f.w, h3.w, acc[i][3]);
+                    for (int k = 0; k < KB; ++k) {
+#pragma unroll
+                        for (int off = NCL / 2; off > 0; off >>= 1) {
+                            x[k].x += __shfl_xor_sync(0xffffffffu, x[k].x, off);
+                            x[k].y += __shfl_xor_sync(0xffffffffu, x[k].y, off);
+                            x[k].z += __shfl_xor_sync(0xffffffffu, x[k].z, off);
+                            x[k].w += __shfl_xor_sync(0xffffffffu, x[k].w, off);
                         }
+                        const int gi = gw + k * NW * GPW + gs;
+                        if (r == 0 && gi < G4) reinterpret_cast<float4*>(score)[gi] = x[k];
                     }
-#pragma unroll
-                    for (int i = 0; i < Sh::EPT; ++i) {
-                        const int e = e0 + ty + i * Sh::TY;
-                        float pt = 0.f;
-                        if (e < n) {
-                            const float dn = den[e];
-                            const TIn* vr = vrow(e) + 4 * tx;
-                            float pr[4] = {0.f, 0.f, 0.f, 0.f};
-                            if (dn > 0.f) {
-                                const float rdn = 1.f / dn;
-#pragma unroll
-                                for (int u = 0; u < 4; ++u) pr[u] = acc[i][u] * rdn;
-                            }
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) { const float r = pr[u] - to_f32(vr[u]); pt = fmaf(r, r, pt); }
-                        }
-#pragma unroll
-                        for (int off = Sh::TX / 2; off > 0; off >>= 1) pt += __shfl_xor_sync(0xffffffffu, pt, off);
-                        if (tx == 0 && e < n) mypart[e] = pt;
-                    }
-                }
-                cluster.sync();                                 // partials visible cluster-wide
-                for (int e = tid; e < n; e += NT) {
-                    float sum = 0.f;
-                    for (int r = 0; r < NCL; ++r) sum += cluster.map_shared_rank(mypart, r)[e];
-                    score[e] = sum;
                 }
                 pb ^= 1;
                 __syncthreads();
-                if (lam > 0) {
-                    select_top(score, cand_pos, n, lam, keep, sbits, hist, tmp, eq_list);
-                } else {
-                    for (int i = tid; i < n; i += NT) keep[i] = 0;
-                    __syncthreads();
-                }
-                // slot bookkeeping, identical in every CTA
-                for (int j = tid; j < lam; j += NT) flags[j] = (j >= n_g || keep[j] == 0) ? 1 : 0;
-                __syncthreads();
-                block_exscan(flags, ranks, lam, tmp);
-                for (int j = tid; j < lam; j += NT) if (flags[j]) free_slots[ranks[j]] = j;
-                __syncthreads();
-                for (int i = tid; i < n_l; i += NT) flags[i] = keep[n_g + i];
-                __syncthreads();
-                block_exscan(flags, ranks, n_l, tmp);
-                for (int i = tid; i < n_l; i += NT) newslot[i] = flags[i] ? free_slots[ranks[i]] : -1;
-                __syncthreads();
-                for (int e = tid; e < n; e += NT) flags[e] = keep[e] ? 0 : 1;
-                __syncthreads();
-                const int nf = block_exscan(flags, ranks, n, tmp);
-                for (int e = tid; e < n; e += NT) if (flags[e]) fold_list[ranks[e]] = e;
-                __syncthreads();
-                // fold into the CTA's columns (notes §2.4, Eqs. 12-13): the folded rows are
-                // staged contiguously, then each thread updates a block of H rows x 4
-                // columns with an outer-product loop.
-                int* foff = reinterpret_cast<int*>(sfold);         // [nf] phi-row offsets (floats)
-                int* voff = foff + C;                              // [nf] value-row offsets (elements)
-                for (int q = tid; q < nf; q += NT) {
-                    foff[q] = (int)(phirow(fold_list[q]) - smem);
-                    voff[q] = (int)(vrow(fold_list[q]) - reinterpret_cast<const TIn*>(smem));
-                }
-                __syncthreads();
-                {
-                    constexpr int FX = CW / 4, FY = NT / FX, RPT = (D + FY - 1) / FY;
-                    const int fx = tid % FX, fy = tid / FX;
-                    float hr[RPT][4];
-#pragma unroll
-                    for (int r = 0; r < RPT; ++r) {
-                        const int j = fy + r * FY;
-                        if (j < D) {
-                            const float4 h4 = *reinterpret_cast<const float4*>(Hs + j * CW + 4 * fx);
-                            hr[r][0] = h4.x; hr[r][1] = h4.y; hr[r][2] = h4.z; hr[r][3] = h4.w;
-                        }
-                    }
-                    for (int q = 0; q < nf; ++q) {
-                        const float4 v4 = load4(reinterpret_cast<const TIn*>(smem) + voff[q] + 4 * fx);
-                        const float* fphi = smem + foff[q];
-#pragma unroll
-                        for (int r = 0; r < RPT; ++r) {
-                            const int j = fy + r * FY;
-                            if (j < D) {
-                                const float ph = fphi[j];
-                                hr[r][0] = fmaf(ph, v4.x, hr[r][0]); hr[r][1] = fmaf(ph, v4.y, hr[r][1]);
-                                hr[r][2] = fmaf(ph, v4.z, hr[r][2]); hr[r][3] = fmaf(ph, v4.w, hr[r][3]);
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int r = 0; r < RPT; ++r) {
-                        const int j = fy + r * FY;
-                        if (j < D)
-                            *reinterpret_cast<float4*>(Hs + j * CW + 4 * fx) =
-                                make_float4(hr[r][0], hr[r][1], hr[r][2], hr[r][3]);
-                    }
-                }
-                for (int j = tid; j < D; j += NT) {
-                    float accs = 0.f;
-                    for (int q = 0; q < nf; ++q) accs += smem[foff[q] + j];
-                    ss[j] += accs;
-                }
-                __syncthreads();
-                // retained newcomers move into the freed slots (resident rows follow)
-                for (int idx = tid; idx < n_l * (D / 4); idx += NT) {
-                    const int i = idx / (D / 4), j4 = (idx % (D / 4)) * 4;
-                    if (newslot[i] >= 0)
-                        *reinterpret_cast<float4*>(phiC + newslot[i] * LD + j4) =
-                            *reinterpret_cast<const float4*>(phiL + i * LD + j4);
-                }
-                for (int idx = tid; idx < n_l * CW; idx += NT) {
-                    const int i = idx / CW, cl = idx % CW;
-                    if (newslot[i] >= 0) vC[newslot[i] * CW + cl] = vL[i * CW + cl];
-                }
-                for (int i = tid; i < n_l; i += NT)
-                    if (newslot[i] >= 0) slot_pos[newslot[i]] = l_lo + i;
             }
+            if (warp == 0) {
+                const int nfo = select_and_place<ClMax<D>::KMAX>(
+                    score, cand_pos, cand_row, n, n_g, n_l, lam, l_lo, new_row, slot_row, slot_pos, fold_row,
+                    free_rows, nfree, P, free_slots, hist, eq_list, keep);
+                if (lane == 0) tmp[0] = nfo;
+            }
+            __syncthreads();
+            const int nf = tmp[0];
+            // fold into this CTA's columns (notes §2.4, Eqs. 12-13) and publish H_{c+1}^T
+            // and s_{c+1}: a thread owns H[j][4 columns]; the threads of column group 0
+            // also carry s[j].  Folded rows are taken four at a time.
+            {
+                float* sH = snapH(c + 1);
+                float* sS = a.snap_s + ((size_t)st * snaps + (c + 1)) * D;
+                const int nf4 = nf & ~3;
+                for (int it = tid; it < D * (CW / 4); it += NT) {
+                    const int j = it % D, c4 = (it / D) * 4;
+                    float4 h = *reinterpret_cast<const float4*>(Hs + j * CW + c4);
+                    float sacc = 0.f;
+                    int q = 0;
+                    for (; q < nf4; q += 4) {
+                        const int4 r4 = *reinterpret_cast<const int4*>(fold_row + q);
+                        const float p0 = phi[(size_t)r4.x * LD + j], p1 = phi[(size_t)r4.y * LD + j];
+                        const float p2 = phi[(size_t)r4.z * LD + j], p3 = phi[(size_t)r4.w * LD + j];
+                        const float4 v0 = load4(vv + (size_t)r4.x * CW + c4), v1 = load4(vv + (size_t)r4.y * CW + c4);
+                        const float4 v2 = load4(vv + (size_t)r4.z * CW + c4), v3 = load4(vv + (size_t)r4.w * CW + c4);
+                        h.x = fmaf(p0, v0.x, h.x); h.y = fmaf(p0, v0.y, h.y); h.z = fmaf(p0, v0.z, h.z); h.w = fmaf(p0, v0.w, h.w);
+                        h.x = fmaf(p1, v1.x, h.x); h.y = fmaf(p1, v1.y, h.y); h.z = fmaf(p1, v1.z, h.z); h.w = fmaf(p1, v1.w, h.w);
+                        h.x = fmaf(p2, v2.x, h.x); h.y = fmaf(p2, v2.y, h.y); h.z = fmaf(p2, v2.z, h.z); h.w = fmaf(p2, v2.w, h.w);
+                        h.x = fmaf(p3, v3.x, h.x); h.y = fmaf(p3, v3.y, h.y); h.z = fmaf(p3, v3.z, h.z); h.w = fmaf(p3, v3.w, h.w);
+                        sacc += p0; sacc += p1; sacc += p2; sacc += p3;
+                    }
+                    for (; q < nf; ++q) {
+                        const int r = fold_row[q];
+                        const float p0 = phi[(size_t)r * LD + j];
+                        const float4 v0 = load4(vv + (size_t)r * CW + c4);
+                        h.x = fmaf(p0, v0.x, h.x); h.y = fmaf(p0, v0.y, h.y); h.z = fmaf(p0, v0.z, h.z); h.w = fmaf(p0, v0.w, h.w);
+                        sacc += p0;
+                    }
+                    *reinterpret_cast<float4*>(Hs + j * CW + c4) = h;
+                    float* dst = sH + (size_t)(col0 + c4) * D + j;
+                    dst[0] = h.x; dst[D] = h.y; dst[2 * D] = h.z; dst[3 * D] = h.w;
+                    if (c4 == 0) {
+                        const float sj = ss[j] + sacc;
+                        ss[j] = sj;
+                        if (rank == 0) sS[j] = sj;
+                    }
+                }
+            }
+            nfree += nf;
+            publish_pos_s(c + 1, false);
         }
         __syncthreads();
-        publish(c + 1);
-        __syncthreads();
+        prefetch(c + 1);
+        if (!scored) {
+            publish_H(c + 1);
+            publish_pos_s(c + 1, true);
+        }
     }
     float* Ho = a.sp.H + (size_t)st * D * DV;
     for (int i = tid; i < D * CW; i += NT) Ho[(size_t)(i / CW) * DV + col0 + i % CW] = Hs[i];
     if (rank == 0)
         for (int i = tid; i < D; i += NT) a.sp.s[(size_t)st * D + i] = ss[i];
+    umma::cp_async_wait<0>();
     cluster.sync();                                             // peers may still read our partials
 }
 
@@ -634,21 +858,21 @@ static cudaError_t launch_scan_d(const PrefillArgs& a, cudaStream_t s) {
     return cudaErrorInvalidValue;
 }
 
-template <int D, int CW, typename TIn>
-static cudaError_t launch_scan_cl_t(const PrefillArgs& a, int ncl, cudaStream_t s) {
-    const size_t bytes = scan_cl_smem_bytes(a.dm, CW);
-    auto kern = scan_cl_kernel<D, CW, TIn>;
+template <int D, int DV, int NCL, typename TIn>
+static cudaError_t launch_scan_cl_t(const PrefillArgs& a, cudaStream_t s) {
+    const size_t bytes = scan_cl_smem_bytes(a.dm, DV / NCL);
+    auto kern = scan_cl_kernel<D, DV, NCL, TIn>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess && ncl > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e == cudaSuccess && NCL > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(a.dm.S * ncl);
+    cfg.gridDim = dim3(a.dm.S * NCL);
     cfg.blockDim = dim3(kClThreads);
     cfg.dynamicSmemBytes = bytes;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = ncl;
+    attr[0].val.clusterDim.x = NCL;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
@@ -663,24 +887,33 @@ static cudaError_t launch_scan_cl_t(const PrefillArgs& a, int ncl, cudaStream_t 
 }
 
 template <int D, typename TIn>
-static cudaError_t launch_scan_cl_d(const PrefillArgs& a, int cw, int ncl, cudaStream_t s) {
-    switch (cw) {
-        case 8: return launch_scan_cl_t<D, 8, TIn>(a, ncl, s);
-        case 16: return launch_scan_cl_t<D, 16, TIn>(a, ncl, s);
-        case 32: return launch_scan_cl_t<D, 32, TIn>(a, ncl, s);
-        case 64: return launch_scan_cl_t<D, 64, TIn>(a, ncl, s);
+static cudaError_t launch_scan_cl_d(const PrefillArgs& a, int ncl, cudaStream_t s) {
+    if (a.dm.d == 128) {
+        switch (ncl) {
+            case 2: return launch_scan_cl_t<D, 128, 2, TIn>(a, s);
+            case 4: return launch_scan_cl_t<D, 128, 4, TIn>(a, s);
+            case 8: return launch_scan_cl_t<D, 128, 8, TIn>(a, s);
+            case 16: return launch_scan_cl_t<D, 128, 16, TIn>(a, s);
+        }
+    } else if (a.dm.d == 64) {
+        switch (ncl) {
+            case 2: return launch_scan_cl_t<D, 64, 2, TIn>(a, s);
+            case 4: return launch_scan_cl_t<D, 64, 4, TIn>(a, s);
+            case 8: return launch_scan_cl_t<D, 64, 8, TIn>(a, s);
+        }
     }
     return cudaErrorNotSupported;
 }
 
 // Cluster size for a shape: the largest power of two <= 16 with the whole grid
-// in one wave of SMs and the resident rows within shared memory; 0 = none.
+// in one wave of SMs and the row pool within shared memory; 0 = none.
 static int pick_cluster(const Dims& dm, int num_sms) {
     for (int ncl = 16; ncl >= 2; ncl >>= 1) {
         const int cw = dm.d / ncl;
         if (cw < 8 || cw > 64) continue;
         if (dm.S * ncl > num_sms) continue;
         if (scan_cl_smem_bytes(dm, cw) > 227 * 1024) continue;
+        if (dm.lam + dm.C > (dm.D == 128 ? ClMax<128>::NMAX : ClMax<64>::NMAX)) continue;
         return ncl;
     }
     return 0;
@@ -699,9 +932,9 @@ cudaError_t launch_scan(const PrefillArgs& a, cudaStream_t s) {
         if (cw > 64 || scan_cl_smem_bytes(a.dm, cw) > 227 * 1024) break;
         cudaError_t e;
         if (a.dm.D == 128)
-            e = a.dm.dtype == 1 ? launch_scan_cl_d<128, __nv_bfloat16>(a, cw, ncl, s) : launch_scan_cl_d<128, float>(a, cw, ncl, s);
+            e = a.dm.dtype == 1 ? launch_scan_cl_d<128, __nv_bfloat16>(a, ncl, s) : launch_scan_cl_d<128, float>(a, ncl, s);
         else
-            e = a.dm.dtype == 1 ? launch_scan_cl_d<64, __nv_bfloat16>(a, cw, ncl, s) : launch_scan_cl_d<64, float>(a, cw, ncl, s);
+            e = a.dm.dtype == 1 ? launch_scan_cl_d<64, __nv_bfloat16>(a, ncl, s) : launch_scan_cl_d<64, float>(a, ncl, s);
         if (e != cudaErrorNotSupported) return e;                // launched (or a real error)
     }
     return a.dm.dtype == 1 ? launch_scan_d<__nv_bfloat16>(a, s) : launch_scan_d<float>(a, s);
