@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) scan_kernel(PrefillArgs a) {
 constexpr int kClThreads = 256;
 
 struct ClOffsets {
-    int Hs, ss, phi, vv, part, xbuf, score, cand_pos, cand_row, keep, slot_pos, slot_row, new_row, free_rows,
+    int Hs, ss, phi, vv, part, score, cand_pos, cand_row, keep, slot_pos, slot_row, new_row, free_rows,
         fold_row, free_slots, hist, tmp, eq_list, total;
 };
 
@@ -306,7 +306,6 @@ __host__ __device__ inline ClOffsets cl_offsets(int D, int CW, int lam, int C, i
     o.phi = take(P * LD);
     o.vv = take((P * CW * esize + 3) / 4);
     o.part = take(2 * N4);
-    o.xbuf = take(3 * kClThreads);
     o.score = take(N4);
     o.cand_pos = take(P);
     o.cand_row = take(P);
@@ -495,9 +494,9 @@ template <int D, int DV, int NCL, typename TIn>
 __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_constant__ PrefillArgs a) {
     namespace cg = cooperative_groups;
     constexpr int CW = DV / NCL, NT = kClThreads, NW = NT / 32, LD = D + 4;
-    constexpr int TX = CW / 4, TY = NT / TX;                  // SRE threads: columns x candidates
-    constexpr int EPT = CW >= 32 ? 8 : (CW == 16 ? 4 : 2);
-    constexpr int TE = TY * EPT;                              // candidates per SRE pass
+    constexpr int CPT = 8, TX = CW / CPT, TY = NT / TX;       // SRE threads: 8 columns x EPT candidates
+    constexpr int EPT = CW == 8 ? 2 : (CW == 16 ? 3 : (CW == 32 ? 5 : 8));
+    constexpr int TE = TY * EPT;                              // candidates per SRE tile
     constexpr int VCH = CW * (int)sizeof(TIn) / 16;           // 16-byte pieces of a value slice
     static_assert(CW >= 8 && CW <= 64 && (CW * sizeof(TIn)) % 16 == 0 && VCH <= 32, "unsupported column split");
     static_assert(32 % NCL == 0, "butterfly groups must tile a warp");
@@ -515,7 +514,6 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
     float* phi = smem + o.phi;                                 // pool [P][LD]
     TIn* vv = reinterpret_cast<TIn*>(smem + o.vv);             // pool [P][CW]
     float* part = smem + o.part;                               // [2][N4] partial SRE
-    float* xbuf = smem + o.xbuf;                               // split-D exchange of the newcomer pass
     float* score = smem + o.score;
     int* cand_pos = reinterpret_cast<int*>(smem + o.cand_pos);
     int* cand_row = reinterpret_cast<int*>(smem + o.cand_row);
@@ -601,59 +599,48 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
     publish_H(0);
     publish_pos_s(0, true);
 
-    // Partial SRE over this CTA's columns (notes §2.3, Eq. 10): for each candidate,
-    // den_e = phi_e . s and pred = H^T phi_e restricted to the CTA's columns are
-    // accumulated in one pass over phi_e; the partial is || pred / den_e - v_e ||^2
-    // over those columns (the zero prediction when den_e == 0).  Every thread of a
-    // tile works (out-of-range candidates repeat a valid row and are not stored),
-    // so the inner loop has no branches and its loads pipeline.
-    auto finish = [&](int e, bool ok, const float (&acc)[4], float dn, int tx, float* mypart, bool store) {
-        float pt = 0.f;
-        if (ok) {
-            const TIn* vr = vv + (size_t)cand_row[e] * CW + 4 * tx;
-            float pr[4] = {0.f, 0.f, 0.f, 0.f};
-            if (dn > 0.f) {
-                const float rdn = 1.f / dn;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) pr[u] = acc[u] * rdn;
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) { const float r = pr[u] - to_f32(vr[u]); pt = fmaf(r, r, pt); }
-        }
-#pragma unroll
-        for (int off = TX / 2; off > 0; off >>= 1) pt += __shfl_xor_sync(0xffffffffu, pt, off);
-        if (store && ok && tx == 0) mypart[e] = pt;
-    };
-    // cache members: thread (tx, ty) takes columns 4tx..4tx+3 of EPT candidates
-    auto sre_members = [&](int e_lo, int e_hi, float* mypart) {
+    // Partial SRE over this CTA's columns (notes §2.3, Eq. 10) of candidates [0, n):
+    // for each candidate, den_e = phi_e . s and pred = H^T phi_e restricted to the
+    // CTA's columns are accumulated in one pass over phi_e; the partial is
+    // || pred / den_e - v_e ||^2 over those columns (the zero prediction when
+    // den_e == 0).  Thread (tx, ty) takes 8 columns of EPT candidates with paired
+    // fp32 FMAs; every thread of a tile works (out-of-range candidates repeat a
+    // valid row and are not stored), so the inner loop has no branches.
+    auto sre_all = [&](int n, float* mypart) {
         const int tx = tid % TX, ty = tid / TX;
-        for (int e0 = e_lo; e0 < e_hi; e0 += TE) {
-            float acc[EPT][4], d0[EPT], d1[EPT];
+        const float* hb = Hs + CPT * tx;
+        for (int e0 = 0; e0 < n; e0 += TE) {
+            unsigned long long a2[EPT][CPT / 2];
+            float d0[EPT], d1[EPT];
             const float* rows[EPT];
 #pragma unroll
             for (int i = 0; i < EPT; ++i) {
-                acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+#pragma unroll
+                for (int u = 0; u < CPT / 2; ++u) a2[i][u] = 0ull;
                 d0[i] = d1[i] = 0.f;
-                rows[i] = phi + (size_t)cand_row[min(e0 + ty + i * TY, e_hi - 1)] * LD;
+                rows[i] = phi + (size_t)cand_row[min(e0 + ty + i * TY, n - 1)] * LD;
             }
 #pragma unroll 2
             for (int j = 0; j < D; j += 4) {
-                const float4 h0 = *reinterpret_cast<const float4*>(Hs + (j + 0) * CW + 4 * tx);
-                const float4 h1 = *reinterpret_cast<const float4*>(Hs + (j + 1) * CW + 4 * tx);
-                const float4 h2 = *reinterpret_cast<const float4*>(Hs + (j + 2) * CW + 4 * tx);
-                const float4 h3 = *reinterpret_cast<const float4*>(Hs + (j + 3) * CW + 4 * tx);
+                float4 h[4][2];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    h[r][0] = *reinterpret_cast<const float4*>(hb + (j + r) * CW);
+                    h[r][1] = *reinterpret_cast<const float4*>(hb + (j + r) * CW + 4);
+                }
                 const float4 s4 = *reinterpret_cast<const float4*>(ss + j);
 #pragma unroll
                 for (int i = 0; i < EPT; ++i) {
                     const float4 f = *reinterpret_cast<const float4*>(rows[i] + j);
-                    acc[i][0] = fmaf(f.x, h0.x, acc[i][0]); acc[i][1] = fmaf(f.x, h0.y, acc[i][1]);
-                    acc[i][2] = fmaf(f.x, h0.z, acc[i][2]); acc[i][3] = fmaf(f.x, h0.w, acc[i][3]);
-                    acc[i][0] = fmaf(f.y, h1.x, acc[i][0]); acc[i][1] = fmaf(f.y, h1.y, acc[i][1]);
-                    acc[i][2] = fmaf(f.y, h1.z, acc[i][2]); acc[i][3] = fmaf(f.y, h1.w, acc[i][3]);
-                    acc[i][0] = fmaf(f.z, h2.x, acc[i][0]); acc[i][1] = fmaf(f.z, h2.y, acc[i][1]);
-                    acc[i][2] = fmaf(f.z, h2.z, acc[i][2]); acc[i][3] = fmaf(f.z, h2.w, acc[i][3]);
-                    acc[i][0] = fmaf(f.w, h3.x, acc[i][0]); acc[i][1] = fmaf(f.w, h3.y, acc[i][1]);
-                    acc[i][2] = fmaf(f.w, h3.z, acc[i][2]); acc[i][3] = fmaf(f.w, h3.w, acc[i][3]);
+                    const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const unsigned long long ff = f2pack(fv[r], fv[r]);
+                        a2[i][0] = f2fma(ff, f2pack(h[r][0].x, h[r][0].y), a2[i][0]);
+                        a2[i][1] = f2fma(ff, f2pack(h[r][0].z, h[r][0].w), a2[i][1]);
+                        a2[i][2] = f2fma(ff, f2pack(h[r][1].x, h[r][1].y), a2[i][2]);
+                        a2[i][3] = f2fma(ff, f2pack(h[r][1].z, h[r][1].w), a2[i][3]);
+                    }
                     d0[i] = fmaf(f.x, s4.x, d0[i]); d1[i] = fmaf(f.y, s4.y, d1[i]);
                     d0[i] = fmaf(f.z, s4.z, d0[i]); d1[i] = fmaf(f.w, s4.w, d1[i]);
                 }
@@ -661,51 +648,30 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
 #pragma unroll
             for (int i = 0; i < EPT; ++i) {
                 const int e = e0 + ty + i * TY;
-                finish(e, e < e_hi, acc[i], d0[i] + d1[i], tx, mypart, true);
-            }
-        }
-    };
-    // newcomers: the sum over D is split in KS parts so that a block of C candidates
-    // still occupies every thread; the parts meet in shared memory
-    constexpr int KS = (NT / (TX * 64) >= 2) ? 2 : 1;
-    constexpr int TB = NT / (TX * KS), DK = D / KS;
-    auto sre_new = [&](int e_lo, int e_hi, float* mypart) {
-        const int tx = tid % TX, ks = (tid / TX) % KS, tb = tid / (TX * KS);
-        for (int e0 = e_lo; e0 < e_hi; e0 += TB) {
-            const int e = e0 + tb;
-            const float* row = phi + (size_t)cand_row[min(e, e_hi - 1)] * LD + ks * DK;
-            const float* hb = Hs + (size_t)(ks * DK) * CW + 4 * tx;
-            const float* sb = ss + ks * DK;
-            float acc[4] = {0.f, 0.f, 0.f, 0.f}, d0 = 0.f, d1 = 0.f;
-#pragma unroll 4
-            for (int j = 0; j < DK; j += 4) {
-                const float4 f = *reinterpret_cast<const float4*>(row + j);
-                const float4 h0 = *reinterpret_cast<const float4*>(hb + (j + 0) * CW);
-                const float4 h1 = *reinterpret_cast<const float4*>(hb + (j + 1) * CW);
-                const float4 h2 = *reinterpret_cast<const float4*>(hb + (j + 2) * CW);
-                const float4 h3 = *reinterpret_cast<const float4*>(hb + (j + 3) * CW);
-                const float4 s4 = *reinterpret_cast<const float4*>(sb + j);
-                acc[0] = fmaf(f.x, h0.x, acc[0]); acc[1] = fmaf(f.x, h0.y, acc[1]);
-                acc[2] = fmaf(f.x, h0.z, acc[2]); acc[3] = fmaf(f.x, h0.w, acc[3]);
-                acc[0] = fmaf(f.y, h1.x, acc[0]); acc[1] = fmaf(f.y, h1.y, acc[1]);
-                acc[2] = fmaf(f.y, h1.z, acc[2]); acc[3] = fmaf(f.y, h1.w, acc[3]);
-                acc[0] = fmaf(f.z, h2.x, acc[0]); acc[1] = fmaf(f.z, h2.y, acc[1]);
-                acc[2] = fmaf(f.z, h2.z, acc[2]); acc[3] = fmaf(f.z, h2.w, acc[3]);
-                acc[0] = fmaf(f.w, h3.x, acc[0]); acc[1] = fmaf(f.w, h3.y, acc[1]);
-                acc[2] = fmaf(f.w, h3.z, acc[2]); acc[3] = fmaf(f.w, h3.w, acc[3]);
-                d0 = fmaf(f.x, s4.x, d0); d1 = fmaf(f.y, s4.y, d1);
-                d0 = fmaf(f.z, s4.z, d0); d1 = fmaf(f.w, s4.w, d1);
-            }
-            if constexpr (KS == 2) {
-                float* xb = xbuf + (tb * TX + tx) * 6;
-                if (ks == 1) { xb[0] = acc[0]; xb[1] = acc[1]; xb[2] = acc[2]; xb[3] = acc[3]; xb[4] = d0; xb[5] = d1; }
-                __syncthreads();
-                if (ks == 0) {
-                    acc[0] += xb[0]; acc[1] += xb[1]; acc[2] += xb[2]; acc[3] += xb[3]; d0 += xb[4]; d1 += xb[5];
+                float pt = 0.f;
+                if (e < n) {
+                    float acc[CPT];
+#pragma unroll
+                    for (int u = 0; u < CPT / 2; ++u) f2unpack(a2[i][u], acc[2 * u], acc[2 * u + 1]);
+                    const float dn = d0[i] + d1[i];
+                    const TIn* vr = vv + (size_t)cand_row[e] * CW + CPT * tx;
+                    const float4 va = load4(vr), vb = load4(vr + 4);
+                    const float vf[CPT] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+                    float pr[CPT];
+#pragma unroll
+                    for (int u = 0; u < CPT; ++u) pr[u] = 0.f;
+                    if (dn > 0.f) {
+                        const float rdn = 1.f / dn;
+#pragma unroll
+                        for (int u = 0; u < CPT; ++u) pr[u] = acc[u] * rdn;
+                    }
+#pragma unroll
+                    for (int u = 0; u < CPT; ++u) { const float r = pr[u] - vf[u]; pt = fmaf(r, r, pt); }
                 }
+#pragma unroll
+                for (int off = TX / 2; off > 0; off >>= 1) pt += __shfl_xor_sync(0xffffffffu, pt, off);
+                if (tx == 0 && e < n) mypart[e] = pt;
             }
-            finish(e, e < e_hi && ks == 0, acc, d0 + d1, tx, mypart, true);
-            if (KS == 2 && e0 + TB < e_hi) __syncthreads();     // the exchange buffer is reused
         }
     };
 
@@ -729,11 +695,10 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
             }
             __syncthreads();
             float* mypart = part + pb * N4;
-            if (lam > 0) sre_members(0, n_g, mypart);           // members are resident
             umma::cp_async_wait<0>();                          // the newcomers have landed
             __syncthreads();
             if (lam > 0) {
-                sre_new(n_g, n, mypart);
+                sre_all(n, mypart);
                 cluster.sync();                                // partials visible cluster-wide
                 // score_e = sum of the cluster's partials, by a butterfly over NCL lanes
                 constexpr int GPW = 32 / NCL, KB = 4;
@@ -772,40 +737,60 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
             __syncthreads();
             const int nf = tmp[0];
             // fold into this CTA's columns (notes §2.4, Eqs. 12-13) and publish H_{c+1}^T
-            // and s_{c+1}: a thread owns H[j][4 columns]; the threads of column group 0
-            // also carry s[j].  Folded rows are taken four at a time.
+            // and s_{c+1}: a thread owns H[j][8 columns] (paired FMAs); the threads of
+            // column group 0 also carry s[j].  Folded rows are taken four at a time.
             {
                 float* sH = snapH(c + 1);
                 float* sS = a.snap_s + ((size_t)st * snaps + (c + 1)) * D;
                 const int nf4 = nf & ~3;
-                for (int it = tid; it < D * (CW / 4); it += NT) {
-                    const int j = it % D, c4 = (it / D) * 4;
-                    float4 h = *reinterpret_cast<const float4*>(Hs + j * CW + c4);
+                for (int it = tid; it < D * (CW / 8); it += NT) {
+                    const int j = it % D, c8 = (it / D) * 8;
+                    float* hp = Hs + j * CW + c8;
+                    const float4 h0 = *reinterpret_cast<const float4*>(hp), h1 = *reinterpret_cast<const float4*>(hp + 4);
+                    unsigned long long h2[4] = {f2pack(h0.x, h0.y), f2pack(h0.z, h0.w), f2pack(h1.x, h1.y), f2pack(h1.z, h1.w)};
                     float sacc = 0.f;
                     int q = 0;
                     for (; q < nf4; q += 4) {
                         const int4 r4 = *reinterpret_cast<const int4*>(fold_row + q);
-                        const float p0 = phi[(size_t)r4.x * LD + j], p1 = phi[(size_t)r4.y * LD + j];
-                        const float p2 = phi[(size_t)r4.z * LD + j], p3 = phi[(size_t)r4.w * LD + j];
-                        const float4 v0 = load4(vv + (size_t)r4.x * CW + c4), v1 = load4(vv + (size_t)r4.y * CW + c4);
-                        const float4 v2 = load4(vv + (size_t)r4.z * CW + c4), v3 = load4(vv + (size_t)r4.w * CW + c4);
-                        h.x = fmaf(p0, v0.x, h.x); h.y = fmaf(p0, v0.y, h.y); h.z = fmaf(p0, v0.z, h.z); h.w = fmaf(p0, v0.w, h.w);
-                        h.x = fmaf(p1, v1.x, h.x); h.y = fmaf(p1, v1.y, h.y); h.z = fmaf(p1, v1.z, h.z); h.w = fmaf(p1, v1.w, h.w);
-                        h.x = fmaf(p2, v2.x, h.x); h.y = fmaf(p2, v2.y, h.y); h.z = fmaf(p2, v2.z, h.z); h.w = fmaf(p2, v2.w, h.w);
-                        h.x = fmaf(p3, v3.x, h.x); h.y = fmaf(p3, v3.y, h.y); h.z = fmaf(p3, v3.z, h.z); h.w = fmaf(p3, v3.w, h.w);
-                        sacc += p0; sacc += p1; sacc += p2; sacc += p3;
+                        const int rr[4] = {r4.x, r4.y, r4.z, r4.w};
+                        float p[4];
+                        float4 va[4], vb[4];
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            p[t] = phi[(size_t)rr[t] * LD + j];
+                            va[t] = load4(vv + (size_t)rr[t] * CW + c8);
+                            vb[t] = load4(vv + (size_t)rr[t] * CW + c8 + 4);
+                        }
+#pragma unroll
+                        for (int t = 0; t < 4; ++t) {
+                            const unsigned long long pp = f2pack(p[t], p[t]);
+                            h2[0] = f2fma(pp, f2pack(va[t].x, va[t].y), h2[0]);
+                            h2[1] = f2fma(pp, f2pack(va[t].z, va[t].w), h2[1]);
+                            h2[2] = f2fma(pp, f2pack(vb[t].x, vb[t].y), h2[2]);
+                            h2[3] = f2fma(pp, f2pack(vb[t].z, vb[t].w), h2[3]);
+                            sacc += p[t];
+                        }
                     }
                     for (; q < nf; ++q) {
                         const int r = fold_row[q];
                         const float p0 = phi[(size_t)r * LD + j];
-                        const float4 v0 = load4(vv + (size_t)r * CW + c4);
-                        h.x = fmaf(p0, v0.x, h.x); h.y = fmaf(p0, v0.y, h.y); h.z = fmaf(p0, v0.z, h.z); h.w = fmaf(p0, v0.w, h.w);
+                        const float4 va = load4(vv + (size_t)r * CW + c8), vb = load4(vv + (size_t)r * CW + c8 + 4);
+                        const unsigned long long pp = f2pack(p0, p0);
+                        h2[0] = f2fma(pp, f2pack(va.x, va.y), h2[0]);
+                        h2[1] = f2fma(pp, f2pack(va.z, va.w), h2[1]);
+                        h2[2] = f2fma(pp, f2pack(vb.x, vb.y), h2[2]);
+                        h2[3] = f2fma(pp, f2pack(vb.z, vb.w), h2[3]);
                         sacc += p0;
                     }
-                    *reinterpret_cast<float4*>(Hs + j * CW + c4) = h;
-                    float* dst = sH + (size_t)(col0 + c4) * D + j;
-                    dst[0] = h.x; dst[D] = h.y; dst[2 * D] = h.z; dst[3 * D] = h.w;
-                    if (c4 == 0) {
+                    float hv[8];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) f2unpack(h2[u], hv[2 * u], hv[2 * u + 1]);
+                    *reinterpret_cast<float4*>(hp) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+                    *reinterpret_cast<float4*>(hp + 4) = make_float4(hv[4], hv[5], hv[6], hv[7]);
+                    float* dst = sH + (size_t)(col0 + c8) * D + j;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) dst[(size_t)u * D] = hv[u];
+                    if (c8 == 0) {
                         const float sj = ss[j] + sacc;
                         ss[j] = sj;
                         if (rank == 0) sS[j] = sj;
