@@ -351,14 +351,20 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
     }
     unsigned keepm = 0u;
     if (lam > 0) {
-        unsigned prefix = 0u, mask = 0u;
+        // digits: exponent (bits 30..23), then mantissa bytes; bit 31 is 0 for scores >= 0
+        unsigned prefix = 0u, mask = 0x80000000u;
         int kk = lam, cnt = n;             // still to keep from the bucket; bucket size
-        for (int shift = 24; shift >= 0 && cnt > 32 && cnt > kk; shift -= 8) {
+#pragma unroll 1
+        for (int pass = 0; pass < 4 && cnt > 32 && cnt > kk; ++pass) {
+            const int shift = pass == 3 ? 0 : 23 - 8 * pass;
+            const unsigned dmask = pass == 3 ? 127u : 255u;
             for (int i = lane; i < 256; i += 32) hist[i] = 0u;
             __syncwarp();
 #pragma unroll
-            for (int k = 0; k < KMAX; ++k)
-                if (32 * k + lane < n && (u[k] & mask) == prefix) atomicAdd(&hist[(u[k] >> shift) & 255u], 1u);
+            for (int k = 0; k < KMAX; ++k) {
+                if (32 * k >= n) break;
+                if (32 * k + lane < n && (u[k] & mask) == prefix) atomicAdd(&hist[(u[k] >> shift) & dmask], 1u);
+            }
             __syncwarp();
             unsigned c[8], lsum = 0u;
 #pragma unroll
@@ -382,11 +388,11 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
             kk -= (int)__shfl_sync(0xffffffffu, h_above, src);
             cnt = (int)__shfl_sync(0xffffffffu, h_cnt, src);
             prefix |= (unsigned)digit << shift;
-            mask |= 255u << shift;
+            mask |= dmask << shift;
             __syncwarp();
         }
         // above the bucket: kept; the bucket is listed in candidate order
-        unsigned inbm = 0u;
+        unsigned inbm = 0u, qbase[KMAX];
         int base = 0;
 #pragma unroll
         for (int k = 0; k < KMAX; ++k) {
@@ -396,53 +402,53 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
             const bool inb = valid && m == prefix;
             if (inb) inbm |= 1u << k;
             const unsigned b = __ballot_sync(0xffffffffu, inb);
+            qbase[k] = (unsigned)base + __popc(b & lt);          // bucket index of this lane's member k
             if (inb) eq_list[base + __popc(b & lt)] = 32 * k + lane;
             base += __popc(b);
         }
         if (cnt == kk) {
             keepm |= inbm;
-        } else {
+        } else if (cnt <= 32) {            // one member per lane; rank through shuffles
             __syncwarp();
-            if (cnt <= 32) {               // one member per lane; compare through shuffles
-                const int i = lane < cnt ? eq_list[lane] : 0;
+            const int i = lane < cnt ? eq_list[lane] : 0;
+            const unsigned ui = __float_as_uint(score[i]);
+            const int pi = cand_pos[i];
+            int r = 0;
+#pragma unroll
+            for (int z = 0; z < 32; ++z) {
+                const unsigned w = __shfl_sync(0xffffffffu, ui, z);
+                const int pz = __shfl_sync(0xffffffffu, pi, z);
+                r += (z < cnt && (w > ui || (w == ui && pz < pi))) ? 1 : 0;
+            }
+            const unsigned kb = __ballot_sync(0xffffffffu, lane < cnt && r < kk);   // bit q: member q kept
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k)
+                if (((inbm >> k) & 1u) && ((kb >> qbase[k]) & 1u)) keepm |= 1u << k;
+        } else {                           // exact ties over many candidates
+            __syncwarp();
+            for (int q = lane; q < cnt; q += 32) {
+                const int i = eq_list[q];
                 const unsigned ui = __float_as_uint(score[i]);
                 const int pi = cand_pos[i];
                 int r = 0;
                 for (int z = 0; z < cnt; ++z) {
-                    const unsigned w = __shfl_sync(0xffffffffu, ui, z);
-                    const int pz = __shfl_sync(0xffffffffu, pi, z);
-                    r += (w > ui || (w == ui && pz < pi)) ? 1 : 0;
+                    const int j = eq_list[z];
+                    const unsigned w = __float_as_uint(score[j]);
+                    r += (w > ui || (w == ui && cand_pos[j] < pi)) ? 1 : 0;
                 }
-                if (lane < cnt) eq_keep[lane] = r < kk ? 1 : 0;
-            } else {                       // exact ties over many candidates
-                for (int q = lane; q < cnt; q += 32) {
-                    const int i = eq_list[q];
-                    const unsigned ui = __float_as_uint(score[i]);
-                    const int pi = cand_pos[i];
-                    int r = 0;
-                    for (int z = 0; z < cnt; ++z) {
-                        const int j = eq_list[z];
-                        const unsigned w = __float_as_uint(score[j]);
-                        r += (w > ui || (w == ui && cand_pos[j] < pi)) ? 1 : 0;
-                    }
-                    eq_keep[q] = r < kk ? 1 : 0;
-                }
+                eq_keep[q] = r < kk ? 1 : 0;
             }
             __syncwarp();
-            base = 0;                      // each owner collects its bucket members' decisions
 #pragma unroll
-            for (int k = 0; k < KMAX; ++k) {
-                const bool inb = (inbm >> k) & 1u;
-                const unsigned b = __ballot_sync(0xffffffffu, inb);
-                if (inb && eq_keep[base + __popc(b & lt)]) keepm |= 1u << k;
-                base += __popc(b);
-            }
+            for (int k = 0; k < KMAX; ++k)
+                if (((inbm >> k) & 1u) && eq_keep[qbase[k]]) keepm |= 1u << k;
         }
     }
     // freed slots, in slot order (member e sits in slot e)
     int base = 0;
 #pragma unroll
     for (int k = 0; k < KMAX; ++k) {
+        if (32 * k >= lam) break;
         const int j = 32 * k + lane;
         const bool f = j < lam && (j >= n_g || ((keepm >> k) & 1u) == 0u);
         const unsigned b = __ballot_sync(0xffffffffu, f);
@@ -471,6 +477,7 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
     base = 0;
 #pragma unroll
     for (int k = 0; k < KMAX; ++k) {
+        if (32 * k >= n) break;
         const bool f = 32 * k + lane < n && ((keepm >> k) & 1u) == 0u;
         const unsigned b = __ballot_sync(0xffffffffu, f);
         const int q = base + __popc(b & lt);

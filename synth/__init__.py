@@ -15,6 +15,9 @@ Recipe (per stream = one (sequence b, kv head g)):
     last n_needles query positions of every query head in the group re-query
     them in order (q := k_needle).  Positions are seeded-uniform without
     replacement ("random") or floor((i + 1/2) (T - N) / N) ("uniform").
+  * duplicates (dup_every = m > 0, test workloads only): every position p with
+    p % m == 0 gets an exact copy of the pair (k, v) at position 0, so many
+    candidates carry bit-identical SRE scores (m = 1: all pairs equal).
   * W for kv head g comes from a Generator seeded with (SEED_BASE, workload id,
     W_STREAM, g): W ~ N(0, 1/d), shape [d, Dh].
   * bf16 workloads round q, k, v and W to bf16 (round to nearest even) before
@@ -54,6 +57,7 @@ class Workload:
     needle_place: str = "none"   # "random" | "uniform" | "none"
     decode_steps: int = 0        # tokens appended one by one after prefill
     wid: int = 0                 # seed id
+    dup_every: int = 0           # > 0: pairs at positions p % dup_every == 0 copy pair 0
 
     @property
     def Gq(self) -> int:
@@ -146,6 +150,10 @@ def stream_arrays(w: Workload, b: int, g: int) -> dict:
         k[pos] = kn
         v[pos] = vn
         q[:, w.T - w.n_needles:w.T, :] = kn[None]
+    if w.dup_every > 0:
+        idx = np.arange(0, T, w.dup_every)
+        k[idx] = k[0]
+        v[idx] = v[0]
     return dict(q=_cast(w, q), k=_cast(w, k), v=_cast(w, v))
 
 

@@ -96,6 +96,10 @@ SMALL = {
     "d128-Dh32": dict(base=2, B=1, Hkv=2, Hq=4, T=512, eta=64, lam=64, chunk=64, Dh=32),
     # fp32 inputs at the 8B head shape
     "f32-d128": dict(base=2, B=1, Hkv=2, Hq=4, T=512, eta=64, lam=64, chunk=64, dtype="f32"),
+    # every pair identical: every selection is an exact tie, broken by position
+    "all-equal-pairs": dict(base=2, B=1, Hkv=2, Hq=4, T=512, eta=64, lam=64, chunk=64, dup_every=1),
+    # a third of the pairs identical, among distinct ones
+    "dup-thirds": dict(base=2, B=1, Hkv=2, Hq=4, T=768, eta=64, lam=96, chunk=64, dup_every=3),
 }
 
 
