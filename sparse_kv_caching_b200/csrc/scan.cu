@@ -18,6 +18,7 @@
 // newcomers fill the freed slots in slot order); the fold H += Phi_S^T V_S,
 // s += sum Phi_S with H held in registers.
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "device_common.cuh"
 #include "umma.cuh"
@@ -333,12 +334,15 @@ __host__ __device__ inline ClOffsets cl_offsets(int D, int CW, int lam, int C, i
 // exactly by (bits descending, position ascending).  Then: kept newcomers take,
 // in position order, the freed slots (evicted members and never-used slots) in
 // slot order; the folded set is listed by pool row and its rows return to the
-// free stack.  Returns the number of folded pairs.
-template <int KMAX>
+// free stack (ROWS), or listed by candidate index (no pool).  Returns the number
+// of folded pairs.
+template <int KMAX, bool ROWS>
 __device__ int select_and_place(const float* score, const int* cand_pos, const int* cand_row, int n, int n_g,
                                 int n_l, int lam, int l_lo, const int* new_row, int* slot_row, int* slot_pos,
                                 int* fold_row, int* free_rows, int nfree, int P, int* free_slots, unsigned* hist,
                                 int* eq_list, int* eq_keep) {
+    using Mask = std::conditional_t<(KMAX > 32), unsigned long long, unsigned>;
+    static_assert(KMAX <= 64, "one mask bit per register row");
     const int lane = threadIdx.x & 31;
     const unsigned lt = (1u << lane) - 1u;
     unsigned u[KMAX];
@@ -347,9 +351,9 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
     for (int k = 0; k < KMAX; ++k) {
         const int e = 32 * k + lane;
         u[k] = e < n ? __float_as_uint(score[e]) : 0u;
-        crow[k] = e < n ? cand_row[e] : 0;
+        crow[k] = ROWS ? (e < n ? cand_row[e] : 0) : e;
     }
-    unsigned keepm = 0u;
+    Mask keepm = 0u;
     if (lam > 0) {
         // digits: exponent (bits 30..23), then mantissa bytes; bit 31 is 0 for scores >= 0
         unsigned prefix = 0u, mask = 0x80000000u;
@@ -392,15 +396,16 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
             __syncwarp();
         }
         // above the bucket: kept; the bucket is listed in candidate order
-        unsigned inbm = 0u, qbase[KMAX];
+        Mask inbm = 0u;
+        unsigned qbase[KMAX];
         int base = 0;
 #pragma unroll
         for (int k = 0; k < KMAX; ++k) {
             const bool valid = 32 * k + lane < n;
             const unsigned m = u[k] & mask;
-            if (valid && m > prefix) keepm |= 1u << k;
+            if (valid && m > prefix) keepm |= Mask(1) << k;
             const bool inb = valid && m == prefix;
-            if (inb) inbm |= 1u << k;
+            if (inb) inbm |= Mask(1) << k;
             const unsigned b = __ballot_sync(0xffffffffu, inb);
             qbase[k] = (unsigned)base + __popc(b & lt);          // bucket index of this lane's member k
             if (inb) eq_list[base + __popc(b & lt)] = 32 * k + lane;
@@ -423,7 +428,7 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
             const unsigned kb = __ballot_sync(0xffffffffu, lane < cnt && r < kk);   // bit q: member q kept
 #pragma unroll
             for (int k = 0; k < KMAX; ++k)
-                if (((inbm >> k) & 1u) && ((kb >> qbase[k]) & 1u)) keepm |= 1u << k;
+                if (((inbm >> k) & 1u) && ((kb >> qbase[k]) & 1u)) keepm |= Mask(1) << k;
         } else {                           // exact ties over many candidates
             __syncwarp();
             for (int q = lane; q < cnt; q += 32) {
@@ -441,7 +446,7 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < KMAX; ++k)
-                if (((inbm >> k) & 1u) && eq_keep[qbase[k]]) keepm |= 1u << k;
+                if (((inbm >> k) & 1u) && eq_keep[qbase[k]]) keepm |= Mask(1) << k;
         }
     }
     // freed slots, in slot order (member e sits in slot e)
@@ -462,13 +467,13 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
     for (int i0 = 0; i0 < n_l; i0 += 32) {
         const int i = i0 + lane;
         const int e = min(n_g + i, n - 1);
-        const unsigned km = __shfl_sync(0xffffffffu, keepm, e & 31);
+        const Mask km = __shfl_sync(0xffffffffu, keepm, e & 31);
         const bool kept = i < n_l && ((km >> (e >> 5)) & 1u);
         const unsigned b = __ballot_sync(0xffffffffu, kept);
         const int fs = base + __popc(b & lt);
         if (kept && fs < n_free_slots) {             // always true when exactly lam are kept
             const int sl = free_slots[fs];
-            slot_row[sl] = new_row[i];
+            if (ROWS) slot_row[sl] = new_row[i];
             slot_pos[sl] = l_lo + i;
         }
         base += __popc(b);
@@ -483,7 +488,7 @@ __device__ int select_and_place(const float* score, const int* cand_pos, const i
         const int q = base + __popc(b & lt);
         if (f && nfree + q < P) {                    // always true when exactly lam are kept
             fold_row[q] = crow[k];
-            free_rows[nfree + q] = crow[k];
+            if (ROWS) free_rows[nfree + q] = crow[k];
         }
         base += __popc(b);
     }
@@ -736,7 +741,7 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
                 __syncthreads();
             }
             if (warp == 0) {
-                const int nfo = select_and_place<ClMax<D>::KMAX>(
+                const int nfo = select_and_place<ClMax<D>::KMAX, true>(
                     score, cand_pos, cand_row, n, n_g, n_l, lam, l_lo, new_row, slot_row, slot_pos, fold_row,
                     free_rows, nfree, P, free_slots, hist, eq_list, keep);
                 if (lane == 0) tmp[0] = nfo;
@@ -820,6 +825,348 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
         for (int i = tid; i < D; i += NT) a.sp.s[(size_t)st * D + i] = ss[i];
     umma::cp_async_wait<0>();
     cluster.sync();                                             // peers may still read our partials
+}
+
+// ---------------------------------------------------------------------------
+// The chain over a cluster with the candidate rows left in global memory, for
+// shapes whose lambda + C rows do not fit a shared-memory pool.  Same column
+// split, cluster reduction, selection and fold as scan_cl_kernel; each scored
+// block streams the candidates' phi rows and the CTA's value columns through a
+// double-buffered shared-memory tile with cp.async (a stream's rows stay in L2
+// from block to block), and stages the folded rows the same way.
+// ---------------------------------------------------------------------------
+constexpr int kCgTile = 128;          // candidate rows per tile
+constexpr int kCgKmax = 48;           // lambda + C <= 32 * kCgKmax
+
+struct CgOffsets {
+    int Hs, ss, tphi, tv, part, score, cand_pos, keep, slot_pos, free_slots, fold_e, hist, tmp, eq_list, total;
+};
+
+__host__ __device__ inline CgOffsets cg_offsets(int D, int CW, int lam, int C, int esize) {
+    const int P = lam + C, LD = D + 4, N4 = (P + 3) & ~3;
+    CgOffsets o;
+    int p = 0;
+    auto take = [&](int n) { int r = p; p += (n + 3) & ~3; return r; };
+    o.Hs = take(D * CW);
+    o.ss = take(D);
+    o.tphi = take(2 * kCgTile * LD);
+    o.tv = take((2 * kCgTile * CW * esize + 3) / 4);
+    o.part = take(2 * N4);
+    o.score = take(N4);
+    o.cand_pos = take(P);
+    o.keep = take(P);
+    o.slot_pos = take(lam + 1);
+    o.free_slots = take(lam + 1);
+    o.fold_e = take(P);
+    o.hist = take(256);
+    o.tmp = take(32);
+    o.eq_list = take(P);
+    o.total = p;
+    return o;
+}
+
+template <int D, int DV, int NCL, typename TIn>
+__global__ void __launch_bounds__(kClThreads, 1) scan_cg_kernel(const __grid_constant__ PrefillArgs a) {
+    namespace cg = cooperative_groups;
+    constexpr int CW = DV / NCL, NT = kClThreads, NW = NT / 32, LD = D + 4, TL = kCgTile;
+    constexpr int CPT = 8, TX = CW / CPT, TY = NT / TX, EPT = TL / TY;   // one tile = one SRE pass
+    constexpr int VCH = CW * (int)sizeof(TIn) / 16;                     // 16-byte pieces of a value slice
+    constexpr int HI = D * (CW / 8), ITEMS = (HI + NT - 1) / NT;         // fold items per thread
+    static_assert(CW >= 16 && CW <= 64 && TY * EPT == TL && VCH <= 32, "unsupported column split");
+    static_assert(32 % NCL == 0, "butterfly groups must tile a warp");
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = (int)cluster.block_rank();
+    extern __shared__ __align__(16) float smem[];
+    const Dims& dm = a.dm;
+    const int lam = dm.lam, C = dm.C, eta = dm.eta, P = lam + C, N4 = (P + 3) & ~3;
+    const int st = blockIdx.x / NCL, b = st / dm.Hkv, g = st % dm.Hkv;
+    const int col0 = rank * CW;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const CgOffsets o = cg_offsets(D, CW, lam, C, (int)sizeof(TIn));
+    float* Hs = smem + o.Hs;                                   // [D][CW]
+    float* ss = smem + o.ss;                                   // [D]
+    float* tphi = smem + o.tphi;                               // [2][TL][LD]
+    TIn* tv = reinterpret_cast<TIn*>(smem + o.tv);             // [2][TL][CW]
+    float* part = smem + o.part;                               // [2][N4]
+    float* score = smem + o.score;
+    int* cand_pos = reinterpret_cast<int*>(smem + o.cand_pos);
+    int* keep = reinterpret_cast<int*>(smem + o.keep);
+    int* slot_pos = reinterpret_cast<int*>(smem + o.slot_pos);
+    int* free_slots = reinterpret_cast<int*>(smem + o.free_slots);
+    int* fold_e = reinterpret_cast<int*>(smem + o.fold_e);
+    unsigned* hist = reinterpret_cast<unsigned*>(smem + o.hist);
+    int* tmp = reinterpret_cast<int*>(smem + o.tmp);
+    int* eq_list = reinterpret_cast<int*>(smem + o.eq_list);
+
+    // cp.async the phi rows and this CTA's value slices of nr candidates (list
+    // index i -> candidate cand(i)) into tile buffer bi; always commits a group
+    auto load_tile = [&](int bi, int nr, auto cand) {
+        float* ph = tphi + (size_t)bi * TL * LD;
+        TIn* vb = tv + (size_t)bi * TL * CW;
+        for (int i = warp; i < nr; i += NW) {
+            const int e = cand(i);
+            const PairRef<TIn> r = pair_ref<TIn>(a, st, b, g, cand_pos[e], e);
+            for (int q = lane; q < D / 4; q += 32) umma::cp_async16(ph + (size_t)i * LD + 4 * q, r.phik + 4 * q);
+            if (lane < VCH)
+                umma::cp_async16(reinterpret_cast<char*>(vb + (size_t)i * CW) + 16 * lane,
+                                 reinterpret_cast<const char*>(r.v + col0) + 16 * lane);
+        }
+        umma::cp_async_commit();
+    };
+
+    const float* Hg = a.sp.H + (size_t)st * D * DV;
+    for (int i = tid; i < D * (CW / 4); i += NT) {
+        const int j = i / (CW / 4), u = i % (CW / 4);
+        umma::cp_async16(Hs + j * CW + 4 * u, Hg + (size_t)j * DV + col0 + 4 * u);
+    }
+    for (int i = tid; i < D / 4; i += NT) umma::cp_async16(ss + 4 * i, a.sp.s + (size_t)st * D + 4 * i);
+    umma::cp_async_commit();
+    for (int j = tid; j < lam; j += NT) slot_pos[j] = a.sp.cache_pos[(size_t)st * lam + j];
+    umma::cp_async_wait<0>();
+    __syncthreads();
+
+    const size_t snaps = (size_t)dm.nc_max + 1;
+    auto snapH = [&](int c) { return a.snap_H + ((size_t)st * snaps + c) * D * DV; };
+    auto publish_pos_s = [&](int c, bool with_s) {
+        int* sp_ = a.snap_pos + ((size_t)st * snaps + c) * lam;
+        for (int j = rank * NT + tid; j < lam; j += NCL * NT) sp_[j] = slot_pos[j];
+        if (with_s && rank == 0) {
+            float* sS = a.snap_s + ((size_t)st * snaps + c) * D;
+            for (int i = tid; i < D; i += NT) sS[i] = ss[i];
+        }
+    };
+    auto publish_H = [&](int c) {
+        float* sH = snapH(c);
+        for (int i = tid; i < D * (CW / 4); i += NT) {
+            const int j = i % D, u = i / D;
+            const float4 h = *reinterpret_cast<const float4*>(Hs + j * CW + 4 * u);
+            float* dst = sH + (size_t)(col0 + 4 * u) * D + j;
+            dst[0] = h.x; dst[D] = h.y; dst[2 * D] = h.z; dst[3 * D] = h.w;
+        }
+    };
+    publish_H(0);
+    publish_pos_s(0, true);
+
+    // partial SRE (notes §2.3, Eq. 10) of the cnt candidates e0.. held in tile bi;
+    // thread (tx, ty) takes 8 columns of EPT rows, out-of-range rows repeat a valid one
+    auto sre_tile_cg = [&](int bi, int e0, int cnt, float* mypart) {
+        const float* ph = tphi + (size_t)bi * TL * LD;
+        const TIn* vb = tv + (size_t)bi * TL * CW;
+        const int tx = tid % TX, ty = tid / TX;
+        const float* hb = Hs + CPT * tx;
+        unsigned long long a2[EPT][CPT / 2];
+        float d0[EPT], d1[EPT];
+        const float* rows[EPT];
+#pragma unroll
+        for (int i = 0; i < EPT; ++i) {
+#pragma unroll
+            for (int u = 0; u < CPT / 2; ++u) a2[i][u] = 0ull;
+            d0[i] = d1[i] = 0.f;
+            rows[i] = ph + (size_t)min(ty + i * TY, cnt - 1) * LD;
+        }
+#pragma unroll 2
+        for (int j = 0; j < D; j += 4) {
+            float4 h[4][2];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                h[r][0] = *reinterpret_cast<const float4*>(hb + (j + r) * CW);
+                h[r][1] = *reinterpret_cast<const float4*>(hb + (j + r) * CW + 4);
+            }
+            const float4 s4 = *reinterpret_cast<const float4*>(ss + j);
+#pragma unroll
+            for (int i = 0; i < EPT; ++i) {
+                const float4 f = *reinterpret_cast<const float4*>(rows[i] + j);
+                const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const unsigned long long ff = f2pack(fv[r], fv[r]);
+                    a2[i][0] = f2fma(ff, f2pack(h[r][0].x, h[r][0].y), a2[i][0]);
+                    a2[i][1] = f2fma(ff, f2pack(h[r][0].z, h[r][0].w), a2[i][1]);
+                    a2[i][2] = f2fma(ff, f2pack(h[r][1].x, h[r][1].y), a2[i][2]);
+                    a2[i][3] = f2fma(ff, f2pack(h[r][1].z, h[r][1].w), a2[i][3]);
+                }
+                d0[i] = fmaf(f.x, s4.x, d0[i]); d1[i] = fmaf(f.y, s4.y, d1[i]);
+                d0[i] = fmaf(f.z, s4.z, d0[i]); d1[i] = fmaf(f.w, s4.w, d1[i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < EPT; ++i) {
+            const int li = ty + i * TY;
+            float pt = 0.f;
+            if (li < cnt) {
+                float acc[CPT];
+#pragma unroll
+                for (int u = 0; u < CPT / 2; ++u) f2unpack(a2[i][u], acc[2 * u], acc[2 * u + 1]);
+                const float dn = d0[i] + d1[i];
+                const TIn* vr = vb + (size_t)li * CW + CPT * tx;
+                const float4 va = load4(vr), vc = load4(vr + 4);
+                const float vf[CPT] = {va.x, va.y, va.z, va.w, vc.x, vc.y, vc.z, vc.w};
+                float pr[CPT];
+#pragma unroll
+                for (int u = 0; u < CPT; ++u) pr[u] = 0.f;
+                if (dn > 0.f) {
+                    const float rdn = 1.f / dn;
+#pragma unroll
+                    for (int u = 0; u < CPT; ++u) pr[u] = acc[u] * rdn;
+                }
+#pragma unroll
+                for (int u = 0; u < CPT; ++u) { const float r = pr[u] - vf[u]; pt = fmaf(r, r, pt); }
+            }
+#pragma unroll
+            for (int off = TX / 2; off > 0; off >>= 1) pt += __shfl_xor_sync(0xffffffffu, pt, off);
+            if (tx == 0 && li < cnt) mypart[e0 + li] = pt;
+        }
+    };
+
+    int pb = 0;
+    for (int c = 0; c < a.nc; ++c) {
+        const int t0 = a.t_start + c * C;
+        const int n_g = min(lam, max(0, t0 - eta));
+        const int l_lo = max(0, t0 - eta), n_l = max(0, t0 + C - eta) - l_lo;
+        const int n = n_g + n_l;
+        const bool scored = n_l > 0 && n > lam;
+        if (n_l > 0 && !scored) {
+            for (int i = tid; i < n_l; i += NT) slot_pos[n_g + i] = l_lo + i;   // all join (notes §2.4)
+        } else if (scored) {
+            for (int e = tid; e < n; e += NT) cand_pos[e] = e < n_g ? slot_pos[e] : l_lo + (e - n_g);
+            __syncthreads();
+            float* mypart = part + pb * N4;
+            if (lam > 0) {
+                const int ntile = (n + TL - 1) / TL;
+                load_tile(0, min(TL, n), [](int i) { return i; });
+                for (int t = 0; t < ntile; ++t) {
+                    if (t + 1 < ntile)
+                        load_tile((t + 1) & 1, min(TL, n - (t + 1) * TL), [t](int i) { return (t + 1) * TL + i; });
+                    else
+                        umma::cp_async_commit();
+                    umma::cp_async_wait<1>();                  // tile t has landed
+                    __syncthreads();
+                    sre_tile_cg(t & 1, t * TL, min(TL, n - t * TL), mypart);
+                    __syncthreads();                           // tile t's buffer is free again
+                }
+                cluster.sync();                                // partials visible cluster-wide
+                constexpr int GPW = 32 / NCL, KB = 4;
+                const int r = lane % NCL, gs = lane / NCL;
+                const float4* src = reinterpret_cast<const float4*>(cluster.map_shared_rank(mypart, r));
+                const int G4 = (n + 3) / 4;
+                for (int gw = warp * GPW; gw < G4; gw += KB * NW * GPW) {     // warp-uniform trip count
+                    float4 x[KB];
+#pragma unroll
+                    for (int k = 0; k < KB; ++k) {
+                        const int gi = gw + k * NW * GPW + gs;
+                        x[k] = gi < G4 ? src[gi] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int k = 0; k < KB; ++k) {
+#pragma unroll
+                        for (int off = NCL / 2; off > 0; off >>= 1) {
+                            x[k].x += __shfl_xor_sync(0xffffffffu, x[k].x, off);
+                            x[k].y += __shfl_xor_sync(0xffffffffu, x[k].y, off);
+                            x[k].z += __shfl_xor_sync(0xffffffffu, x[k].z, off);
+                            x[k].w += __shfl_xor_sync(0xffffffffu, x[k].w, off);
+                        }
+                        const int gi = gw + k * NW * GPW + gs;
+                        if (r == 0 && gi < G4) reinterpret_cast<float4*>(score)[gi] = x[k];
+                    }
+                }
+                pb ^= 1;
+                __syncthreads();
+            }
+            if (warp == 0) {
+                const int nfo = select_and_place<kCgKmax, false>(
+                    score, cand_pos, nullptr, n, n_g, n_l, lam, l_lo, nullptr, nullptr, slot_pos, fold_e,
+                    nullptr, 0, P, free_slots, hist, eq_list, keep);
+                if (lane == 0) tmp[0] = nfo;
+            }
+            __syncthreads();
+            const int nf = tmp[0];
+            // fold (notes §2.4, Eqs. 12-13), folded rows streamed through the tiles: a
+            // thread owns ITEMS x (row j, 8 columns) of H; column group 0 also carries s[j]
+            unsigned long long h2[ITEMS][4];
+            float sacc[ITEMS];
+#pragma unroll
+            for (int k = 0; k < ITEMS; ++k) {
+                const int it = tid + k * NT;
+                sacc[k] = 0.f;
+                if (it < HI) {
+                    const float* hp = Hs + (it % D) * CW + (it / D) * 8;
+                    const float4 h0 = *reinterpret_cast<const float4*>(hp), h1 = *reinterpret_cast<const float4*>(hp + 4);
+                    h2[k][0] = f2pack(h0.x, h0.y); h2[k][1] = f2pack(h0.z, h0.w);
+                    h2[k][2] = f2pack(h1.x, h1.y); h2[k][3] = f2pack(h1.z, h1.w);
+                }
+            }
+            const int nft = (nf + TL - 1) / TL;
+            if (nft > 0) load_tile(0, min(TL, nf), [&](int i) { return fold_e[i]; });
+            for (int t = 0; t < nft; ++t) {
+                if (t + 1 < nft)
+                    load_tile((t + 1) & 1, min(TL, nf - (t + 1) * TL), [&, t](int i) { return fold_e[(t + 1) * TL + i]; });
+                else
+                    umma::cp_async_commit();
+                umma::cp_async_wait<1>();
+                __syncthreads();
+                const float* ph = tphi + (size_t)(t & 1) * TL * LD;
+                const TIn* vb = tv + (size_t)(t & 1) * TL * CW;
+                const int cnt = min(TL, nf - t * TL);
+#pragma unroll
+                for (int k = 0; k < ITEMS; ++k) {
+                    const int it = tid + k * NT;
+                    if (it >= HI) continue;
+                    const int j = it % D, c8 = (it / D) * 8;
+                    for (int q = 0; q < cnt; ++q) {
+                        const float p0 = ph[(size_t)q * LD + j];
+                        const float4 va = load4(vb + (size_t)q * CW + c8), vc = load4(vb + (size_t)q * CW + c8 + 4);
+                        const unsigned long long pp = f2pack(p0, p0);
+                        h2[k][0] = f2fma(pp, f2pack(va.x, va.y), h2[k][0]);
+                        h2[k][1] = f2fma(pp, f2pack(va.z, va.w), h2[k][1]);
+                        h2[k][2] = f2fma(pp, f2pack(vc.x, vc.y), h2[k][2]);
+                        h2[k][3] = f2fma(pp, f2pack(vc.z, vc.w), h2[k][3]);
+                        sacc[k] += p0;
+                    }
+                }
+                __syncthreads();
+            }
+            {
+                float* sH = snapH(c + 1);
+                float* sS = a.snap_s + ((size_t)st * snaps + (c + 1)) * D;
+#pragma unroll
+                for (int k = 0; k < ITEMS; ++k) {
+                    const int it = tid + k * NT;
+                    if (it >= HI) continue;
+                    const int j = it % D, c8 = (it / D) * 8;
+                    float hv[8];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) f2unpack(h2[k][u], hv[2 * u], hv[2 * u + 1]);
+                    float* hp = Hs + j * CW + c8;
+                    *reinterpret_cast<float4*>(hp) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+                    *reinterpret_cast<float4*>(hp + 4) = make_float4(hv[4], hv[5], hv[6], hv[7]);
+                    float* dst = sH + (size_t)(col0 + c8) * D + j;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) dst[(size_t)u * D] = hv[u];
+                    if (c8 == 0) {
+                        const float sj = ss[j] + sacc[k];
+                        ss[j] = sj;
+                        if (rank == 0) sS[j] = sj;
+                    }
+                }
+            }
+            publish_pos_s(c + 1, false);
+        }
+        __syncthreads();
+        if (!scored) {
+            publish_H(c + 1);
+            publish_pos_s(c + 1, true);
+        }
+    }
+    float* Ho = a.sp.H + (size_t)st * D * DV;
+    for (int i = tid; i < D * CW; i += NT) Ho[(size_t)(i / CW) * DV + col0 + i % CW] = Hs[i];
+    if (rank == 0)
+        for (int i = tid; i < D; i += NT) a.sp.s[(size_t)st * D + i] = ss[i];
+    umma::cp_async_wait<0>();
+    cluster.sync();                                             // peers may still read our partials
+}
+
+size_t scan_cg_smem_bytes(const Dims& dm, int CW) {
+    return (size_t)cg_offsets(dm.D, CW, dm.lam, dm.C, dm.esize).total * 4;
 }
 
 size_t scan_cl_smem_bytes(const Dims& dm, int CW) {
@@ -911,6 +1258,50 @@ static int pick_cluster(const Dims& dm, int num_sms) {
     return 0;
 }
 
+template <int D, int DV, int NCL, typename TIn>
+static cudaError_t launch_scan_cg_t(const PrefillArgs& a, cudaStream_t s) {
+    const size_t bytes = scan_cg_smem_bytes(a.dm, DV / NCL);
+    auto kern = scan_cg_kernel<D, DV, NCL, TIn>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && NCL > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.dm.S * NCL);
+    cfg.blockDim = dim3(kClThreads);
+    cfg.dynamicSmemBytes = bytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = NCL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nclusters = 0;
+    e = cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg);
+    if (e != cudaSuccess || nclusters < a.dm.S) { (void)cudaGetLastError(); return cudaErrorNotSupported; }
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <int D, typename TIn>
+static cudaError_t launch_scan_cg_d(const PrefillArgs& a, int ncl, cudaStream_t s) {
+    if (a.dm.d == 128) {
+        switch (ncl) {
+            case 2: return launch_scan_cg_t<D, 128, 2, TIn>(a, s);
+            case 4: return launch_scan_cg_t<D, 128, 4, TIn>(a, s);
+            case 8: return launch_scan_cg_t<D, 128, 8, TIn>(a, s);
+        }
+    } else if (a.dm.d == 64) {
+        switch (ncl) {
+            case 2: return launch_scan_cg_t<D, 64, 2, TIn>(a, s);
+            case 4: return launch_scan_cg_t<D, 64, 4, TIn>(a, s);
+        }
+    }
+    return cudaErrorNotSupported;
+}
+
 static int g_num_sms = 0;
 
 cudaError_t launch_scan(const PrefillArgs& a, cudaStream_t s) {
@@ -928,6 +1319,20 @@ cudaError_t launch_scan(const PrefillArgs& a, cudaStream_t s) {
         else
             e = a.dm.dtype == 1 ? launch_scan_cl_d<64, __nv_bfloat16>(a, ncl, s) : launch_scan_cl_d<64, float>(a, ncl, s);
         if (e != cudaErrorNotSupported) return e;                // launched (or a real error)
+    }
+    // rows left in global memory: the largest cluster with whole 16-column slices
+    if (a.dm.lam + a.dm.C <= 32 * kCgKmax) {
+        for (int ncl = 8; ncl >= 2; ncl >>= 1) {
+            const int cw = a.dm.d / ncl;
+            if (cw < 16 || cw > 64 || a.dm.S * ncl > g_num_sms) continue;
+            if (scan_cg_smem_bytes(a.dm, cw) > 227 * 1024) continue;
+            cudaError_t e;
+            if (a.dm.D == 128)
+                e = a.dm.dtype == 1 ? launch_scan_cg_d<128, __nv_bfloat16>(a, ncl, s) : launch_scan_cg_d<128, float>(a, ncl, s);
+            else
+                e = a.dm.dtype == 1 ? launch_scan_cg_d<64, __nv_bfloat16>(a, ncl, s) : launch_scan_cg_d<64, float>(a, ncl, s);
+            if (e != cudaErrorNotSupported) return e;
+        }
     }
     return a.dm.dtype == 1 ? launch_scan_d<__nv_bfloat16>(a, s) : launch_scan_d<float>(a, s);
 }

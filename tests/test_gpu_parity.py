@@ -100,6 +100,10 @@ SMALL = {
     "all-equal-pairs": dict(base=2, B=1, Hkv=2, Hq=4, T=512, eta=64, lam=64, chunk=64, dup_every=1),
     # a third of the pairs identical, among distinct ones
     "dup-thirds": dict(base=2, B=1, Hkv=2, Hq=4, T=768, eta=64, lam=96, chunk=64, dup_every=3),
+    # lambda + C beyond a shared-memory row pool: candidate rows streamed from global memory
+    "rows-global-d128": dict(base=3, B=1, Hkv=2, Hq=4, T=1024, eta=64, lam=480, chunk=64),
+    "rows-global-d64": dict(base=5, B=1, Hkv=2, Hq=4, T=1280, eta=64, lam=768, chunk=64),
+    "rows-global-f32": dict(base=2, B=1, Hkv=2, Hq=4, T=1024, eta=64, lam=480, chunk=64, dtype="f32"),
 }
 
 
