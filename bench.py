@@ -3,6 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lola|reference]
                     [--workload 2] [--no-decode]
+    python bench.py --sweep [--steps K]     # single-layer latency over (eta, lambda)
 
 A step is one pass of the whole layer over one batch of synthetic input:
 reset the memories, then chunkwise prefill of B x T tokens (window advance,
@@ -275,6 +276,73 @@ def run_reference(args, w, rank):
     return 0
 
 
+# The pages' single-layer forward latencies (App. B, Tables 7-8; RTX 4090, batch 2,
+# 4096 tokens, 32 heads, emb 4096, precision not stated): context only.
+PAGES_LAYER_MS_RTX4090 = {"eta512": {"lambda0": 4.2, "lambda512": 9.7},
+                          "eta64": {"lambda0": 18.3, "lambda512": 35.5}}
+
+
+def run_sweep(args):
+    """Per-layer prefill latency over the (eta, lambda) grid: one JSON line."""
+    import torch
+    import sparse_kv_caching_b200 as lola
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w0 = synth.sweep_workload(synth.SWEEP_ETAS[0], synth.SWEEP_LAMBDAS[0])
+    full = synth.full_arrays(w0)          # the same inputs at every grid point
+
+    def to_dev(x):
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(x).to(dev)
+
+    q, k, v, W = (to_dev(full[x]) for x in ("q", "k", "v", "W"))
+    y = torch.empty((w0.B, w0.T, w0.Hq, w0.d), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    points = []
+    for eta in synth.SWEEP_ETAS:
+        for lam in synth.SWEEP_LAMBDAS:
+            w = synth.sweep_workload(eta, lam)
+            cfg = lola.make_config(w.B, w.Hq, w.Hkv, w.d, w.Dh, w.eta, w.lam, w.chunk, w.dtype, w.T)
+            layer = lola.LolaLayer(cfg, W, device=dev)
+            for _ in range(args.warmup):
+                layer.reset()
+                layer.prefill(q, k, v, y)
+            torch.cuda.synchronize()
+            layer.profile(True)
+            total = 0.0
+            for _ in range(args.steps):
+                flush.zero_()
+                ev0 = torch.cuda.Event(enable_timing=True)
+                ev1 = torch.cuda.Event(enable_timing=True)
+                ev0.record(stream)
+                layer.reset()
+                layer.prefill(q, k, v, y)
+                ev1.record(stream)
+                ev1.synchronize()
+                total += ev0.elapsed_time(ev1)
+            prof = layer.profile_read()
+            layer.profile(False)
+            ms = total / args.steps
+            kern = {kk: round(prof[kk][0] / max(1, prof[kk][1]), 4) for kk in ("phi", "scan", "output", "finalize")}
+            points.append({"eta": eta, "lambda": lam, "ms": round(ms, 4),
+                           "tokens_per_s": w.B * w.T / (ms / 1e3), "kernel_ms": kern})
+            layer.close()
+            del layer
+    line = {"metric": "single-layer prefill latency over the (eta, lambda) grid", "unit": "ms",
+            "higher_is_better": False, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "layer-sweep", "B": w0.B, "T": w0.T, "Hq": w0.Hq, "Hkv": w0.Hkv, "d": w0.d,
+                       "phi_dim": w0.D, "chunk": w0.chunk, "input_dtype": w0.dtype,
+                       "l2": "flushed between timed steps (256 MB write)"},
+            "sweep": points,
+            "context": {"pages_single_layer_ms_rtx4090": PAGES_LAYER_MS_RTX4090}}
+    print(json.dumps(line))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -284,9 +352,12 @@ def main():
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work (cpu_baseline)")
+    ap.add_argument("--sweep", action="store_true", help="single-layer latency over the (eta, lambda) grid")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.sweep:
+        return run_sweep(args)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

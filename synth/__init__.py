@@ -94,6 +94,20 @@ WORKLOADS = {
 }
 
 
+# Per-layer (eta, lambda) grid at the single-layer shape of the App. B latency
+# tables (batch 2, 4096 tokens, 32 heads, head dim 128), Llama-3.1-8B grouping
+# 32/8, values drawn as in workload 2.  The recipe does not depend on (eta,
+# lambda), so every grid point sees the same q, k, v and W.
+SWEEP_ETAS = (64, 128, 256, 512)
+SWEEP_LAMBDAS = (0, 64, 128, 256, 512)
+
+
+def sweep_workload(eta: int, lam: int) -> Workload:
+    """One point of the per-layer (eta, lambda) grid."""
+    return Workload(f"layer-e{eta}-l{lam}", B=2, Hq=32, Hkv=8, T=4096, d=128, Dh=64, eta=eta, lam=lam,
+                    chunk=64, dtype="bf16", cluster_frac=0.2, n_clusters=64, cluster_std=0.05, wid=6)
+
+
 def workload(i: int, **overrides) -> Workload:
     """Workload `i` (1..5), optionally with fields replaced (smaller T, B, ...)."""
     w = WORKLOADS[i]

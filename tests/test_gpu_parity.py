@@ -255,7 +255,18 @@ def _sample_rows(w, rng):
 @pytest.mark.slow
 @pytest.mark.parametrize("cfg", [2, 3, 5])
 def test_fullsize_prefill_sampled(cfg):
-    w = synth.workload(cfg)
+    _sampled_prefill_check(synth.workload(cfg), cfg)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("eta,lam", [(64, 512), (512, 256)])
+def test_layer_sweep_sampled(eta, lam):
+    """Corners of the per-layer (eta, lambda) grid that bench.py --sweep times."""
+    _sampled_prefill_check(synth.sweep_workload(eta, lam), eta + lam)
+
+
+def _sampled_prefill_check(w, seed):
+    cfg = w.name
     full = synth.full_arrays(w)
     dev = P.to_device(w, full)
     layer = P.make_layer(w, dev["W"], max_tokens=w.T)
@@ -264,7 +275,7 @@ def test_fullsize_prefill_sampled(cfg):
     ex = layer.export()
     tr = ex["trace_pos"].cpu().numpy()
     assert torch.isfinite(y).all()
-    rng = np.random.default_rng(cfg)
+    rng = np.random.default_rng(seed)
     streams = [(0, 0), (w.B - 1, w.Hkv - 1)]
     tol = P.TOL[w.dtype]
     ties = 0
