@@ -95,6 +95,14 @@ def decode_step_flops(w: synth.Workload) -> int:
 # ---------------------------------------------------------------------------
 # helpers
 # ---------------------------------------------------------------------------
+SM_MAX_MHZ = 1965          # clocks.max.sm of the B200s here
+
+
+def fp32_alu_peak_tflops(num_sms: int) -> float:
+    """FP32 FMA peak of the CUDA cores: SMs x 128 lanes x 2 FLOP x max SM clock."""
+    return num_sms * 128 * 2 * SM_MAX_MHZ * 1e6 / 1e12
+
+
 def load_peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -353,6 +361,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work (cpu_baseline)")
     ap.add_argument("--sweep", action="store_true", help="single-layer latency over the (eta, lambda) grid")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="sequences of the decode leg (default: the workload's 64; smaller for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -447,10 +457,19 @@ def main():
     fl = work[dom]["flops"]
     achieved = fl / (dom_ms / 1e3) / 1e12
     peak = peaks["bf16_tflops"]
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
-                "traffic": traffic_for(dom, w.name),
-                "flops_per_launch": fl, "ms_per_launch": dom_ms}
+    if dom == "scan":
+        # the memory-update chain runs fp32 FMAs on the CUDA cores, not the tensor cores
+        alu = fp32_alu_peak_tflops(props.multi_processor_count)
+        roofline = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": alu, "unit": "TFLOP/s",
+                    "frac": achieved / alu,
+                    "peak_kind": f"derived fp32 FMA: {props.multi_processor_count} SMs x 128 lanes x 2 FLOP x "
+                                 f"{SM_MAX_MHZ} MHz",
+                    "traffic": traffic_for(dom, w.name), "flops_per_launch": fl, "ms_per_launch": dom_ms}
+    else:
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
+                    "traffic": traffic_for(dom, w.name),
+                    "flops_per_launch": fl, "ms_per_launch": dom_ms}
     shares = {kk: round(prof[kk][0] / max(1e-9, sum(p[0] for p in prof.values())), 4) for kk in prof}
     layer_roof_ms = max(work["total_flops"] / (peak * 1e12), 0.0) * 1e3
     # ---- e2e through the host-buffer entry point ------------------------------
@@ -506,7 +525,7 @@ def main():
 
     # ---- decode workload ----------------------------------------------------
     if not args.no_decode:
-        wd = synth.workload(4)
+        wd = synth.workload(4) if args.decode_batch is None else synth.workload(4, B=args.decode_batch)
         fd = synth.full_arrays(wd)
         qd, kd, vd, Wd = (to_dev(fd[x]) for x in ("q", "k", "v", "W"))
         del fd
