@@ -453,7 +453,10 @@ def main():
     work = prefill_work(w)
     # dominant kernel by measured time
     dom = max(("phi", "scan", "output"), key=lambda kk: prof[kk][0])
-    dom_ms = prof[dom][0] / max(1, prof[dom][1])
+    # per step: a call may launch a kernel class several times (the chain runs in
+    # chunk segments), so work and time are both summed over the step's launches
+    dom_ms = prof[dom][0] / args.steps
+    dom_launches = prof[dom][1] / args.steps
     fl = work[dom]["flops"]
     achieved = fl / (dom_ms / 1e3) / 1e12
     peak = peaks["bf16_tflops"]
@@ -464,12 +467,13 @@ def main():
                     "frac": achieved / alu,
                     "peak_kind": f"derived fp32 FMA: {props.multi_processor_count} SMs x 128 lanes x 2 FLOP x "
                                  f"{SM_MAX_MHZ} MHz",
-                    "traffic": traffic_for(dom, w.name), "flops_per_launch": fl, "ms_per_launch": dom_ms}
+                    "traffic": traffic_for(dom, w.name), "flops_per_step": fl, "kernel_ms_per_step": dom_ms,
+                    "launches_per_step": dom_launches}
     else:
         roofline = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
                     "traffic": traffic_for(dom, w.name),
-                    "flops_per_launch": fl, "ms_per_launch": dom_ms}
+                    "flops_per_step": fl, "kernel_ms_per_step": dom_ms, "launches_per_step": dom_launches}
     shares = {kk: round(prof[kk][0] / max(1e-9, sum(p[0] for p in prof.values())), 4) for kk in prof}
     layer_roof_ms = max(work["total_flops"] / (peak * 1e12), 0.0) * 1e3
     # ---- e2e through the host-buffer entry point ------------------------------

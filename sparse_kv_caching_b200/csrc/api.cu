@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <string>
 #include <vector>
@@ -37,11 +38,23 @@ struct lola_state {
     bool resid_ok = true;     // per-slot decode residuals match (H, s)
     std::vector<lola_prof_mark> marks;
     std::vector<cudaEvent_t> pool;
+    // Prefill overlap: the chain runs on a high-priority stream in chunk segments,
+    // each segment's output on a low-priority stream as soon as its snapshots exist
+    // (null when the state was built without them: one stream, one segment).
+    cudaStream_t s_chain = nullptr, s_out = nullptr;
+    cudaEvent_t ev_fork = nullptr, ev_seg = nullptr, ev_join_chain = nullptr, ev_join_out = nullptr;
+    // Host-buffer prefill: copies in and out on their own streams, overlapped with
+    // the compute of neighbouring segments (double-buffered staging).
+    cudaStream_t s_in = nullptr, s_back = nullptr;
+    cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_done[2] = {nullptr, nullptr}, ev_back[2] = {nullptr, nullptr};
 };
 
 namespace {
 
 thread_local std::string g_err;
+constexpr int kSplitMinChunks = 32;   // calls with fewer chunks run in one segment
+constexpr int kSplitSegments = 4;
+constexpr int kHostSegments = 4;      // host-buffer prefill: copies overlap compute per segment
 std::atomic<long long> g_launches{0};
 
 cudaEvent_t take_event(lola_state* st) {
@@ -212,6 +225,26 @@ int lola_state_init(const lola_config* cfg, const void* W, void* dev_buf, size_t
     if (e != cudaSuccess) { delete st; return cuda_fail(e, "copying W"); }
     rc = clear_state(st, s);
     if (rc) { delete st; return rc; }
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&st->s_chain, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&st->s_out, cudaStreamNonBlocking, least) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_seg, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_join_chain, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_join_out, cudaEventDisableTiming) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&st->s_in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&st->s_back, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_in[0], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_in[1], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_done[0], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_done[1], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_back[0], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&st->ev_back[1], cudaEventDisableTiming) != cudaSuccess) {
+        e = cudaGetLastError();
+        lola_state_free(st);
+        return cuda_fail(e, "creating the prefill streams");
+    }
     *out = st;
     return LOLA_OK;
 }
@@ -225,6 +258,11 @@ int lola_state_free(lola_state* st) {
     if (st) {
         for (auto& m : st->marks) { cudaEventDestroy(m.a); cudaEventDestroy(m.b); }
         for (auto e : st->pool) cudaEventDestroy(e);
+        for (cudaEvent_t e : {st->ev_fork, st->ev_seg, st->ev_join_chain, st->ev_join_out, st->ev_in[0],
+                              st->ev_in[1], st->ev_done[0], st->ev_done[1], st->ev_back[0], st->ev_back[1]})
+            if (e) cudaEventDestroy(e);
+        for (cudaStream_t q : {st->s_chain, st->s_out, st->s_in, st->s_back})
+            if (q) cudaStreamDestroy(q);
     }
     delete st;
     return LOLA_OK;
@@ -289,6 +327,8 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
     a.T = T;
     a.t_start = (int)st->t;
     a.nc = T / dm.C;
+    a.c_begin = 0;
+    a.c_end = a.nc;
     a.phik_new = (float*)(st->base + st->L.phik_new);
     a.snap_pos = (int*)(st->base + st->L.snap_pos);
     a.snap_H = (float*)(st->base + st->L.snap_H);
@@ -298,12 +338,37 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
     cudaError_t e;
     if ((e = traced(st, 0, 1, s, [&] { return lola::launch_phi_keys(a, s); })) != cudaSuccess)
         return cuda_fail(e, "feature-map kernel");
-    if ((e = traced(st, 1, 1, s, [&] { return lola::launch_scan(a, s); })) != cudaSuccess)
-        return cuda_fail(e, "scan kernel");
-    if ((e = traced(st, 2, 1, s, [&] {
-             return dm.dtype == LOLA_DTYPE_BF16 ? lola::launch_output_tc(a, s) : lola::launch_output(a, s);
-         })) != cudaSuccess)
-        return cuda_fail(e, "output kernel");
+    auto output = [&](cudaStream_t q) {
+        return dm.dtype == LOLA_DTYPE_BF16 ? lola::launch_output_tc(a, q) : lola::launch_output(a, q);
+    };
+    const int seg = a.nc >= kSplitMinChunks ? (a.nc + kSplitSegments - 1) / kSplitSegments : a.nc;
+    if (st->s_chain && seg < a.nc) {
+        // The chain of segment i and the output of segment i-1 run at the same time:
+        // the chain holds one cluster per stream, the output fills the other SMs.
+        if ((e = cudaEventRecord(st->ev_fork, s)) || (e = cudaStreamWaitEvent(st->s_chain, st->ev_fork, 0)) ||
+            (e = cudaStreamWaitEvent(st->s_out, st->ev_fork, 0)))
+            return cuda_fail(e, "forking the prefill streams");
+        for (int c0 = 0; c0 < a.nc; c0 += seg) {
+            a.c_begin = c0;
+            a.c_end = std::min(a.nc, c0 + seg);
+            if ((e = traced(st, 1, 1, st->s_chain, [&] { return lola::launch_scan(a, st->s_chain); })) != cudaSuccess)
+                return cuda_fail(e, "scan kernel");
+            if ((e = cudaEventRecord(st->ev_seg, st->s_chain)) || (e = cudaStreamWaitEvent(st->s_out, st->ev_seg, 0)))
+                return cuda_fail(e, "ordering a prefill segment");
+            if ((e = traced(st, 2, 1, st->s_out, [&] { return output(st->s_out); })) != cudaSuccess)
+                return cuda_fail(e, "output kernel");
+        }
+        a.c_begin = 0;
+        a.c_end = a.nc;
+        if ((e = cudaEventRecord(st->ev_join_chain, st->s_chain)) || (e = cudaEventRecord(st->ev_join_out, st->s_out)) ||
+            (e = cudaStreamWaitEvent(s, st->ev_join_chain, 0)) || (e = cudaStreamWaitEvent(s, st->ev_join_out, 0)))
+            return cuda_fail(e, "joining the prefill streams");
+    } else {
+        if ((e = traced(st, 1, 1, s, [&] { return lola::launch_scan(a, s); })) != cudaSuccess)
+            return cuda_fail(e, "scan kernel");
+        if ((e = traced(st, 2, 1, s, [&] { return output(s); })) != cudaSuccess)
+            return cuda_fail(e, "output kernel");
+    }
     if ((e = traced(st, 3, dm.lam > 0 ? 2 : 1, s, [&] { return lola::launch_finalize(a, s); })) != cudaSuccess)
         return cuda_fail(e, "finalize kernels");
     st->last_nc = a.nc;
@@ -345,18 +410,69 @@ int lola_prefill_chunked_host(lola_state* st, const void* q, const void* k, cons
     if (T < 1 || T % dm.C || T > dm.max_tokens)
         return fail(LOLA_ERR_INVALID_ARG, "T=%d must be a positive multiple of chunk and <= max_tokens", T);
     cudaStream_t s = (cudaStream_t)stream;
-    const size_t nq = (size_t)dm.B * T * dm.Hq * dm.d, nk = (size_t)dm.B * T * dm.Hkv * dm.d;
     char* b = st->base;
     cudaError_t e;
-    if ((e = cudaMemcpyAsync(b + st->L.io_q, q, nq * dm.esize, cudaMemcpyHostToDevice, s)) ||
-        (e = cudaMemcpyAsync(b + st->L.io_k, k, nk * dm.esize, cudaMemcpyHostToDevice, s)) ||
-        (e = cudaMemcpyAsync(b + st->L.io_v, v, nk * dm.esize, cudaMemcpyHostToDevice, s)))
-        return cuda_fail(e, "host-to-device copy");
-    int rc = lola_prefill_chunked(st, b + st->L.io_q, b + st->L.io_k, b + st->L.io_v, T,
-                                  (float*)(b + st->L.io_y), stream);
-    if (rc) return rc;
-    if ((e = cudaMemcpyAsync(y, b + st->L.io_y, nq * 4, cudaMemcpyDeviceToHost, s)))
-        return cuda_fail(e, "device-to-host copy");
+    const int nc = T / dm.C;
+    if (!st->s_in || nc < 2 * kHostSegments) {
+        const size_t nq = (size_t)dm.B * T * dm.Hq * dm.d, nk = (size_t)dm.B * T * dm.Hkv * dm.d;
+        if ((e = cudaMemcpyAsync(b + st->L.io_q, q, nq * dm.esize, cudaMemcpyHostToDevice, s)) ||
+            (e = cudaMemcpyAsync(b + st->L.io_k, k, nk * dm.esize, cudaMemcpyHostToDevice, s)) ||
+            (e = cudaMemcpyAsync(b + st->L.io_v, v, nk * dm.esize, cudaMemcpyHostToDevice, s)))
+            return cuda_fail(e, "host-to-device copy");
+        int rc = lola_prefill_chunked(st, b + st->L.io_q, b + st->L.io_k, b + st->L.io_v, T,
+                                      (float*)(b + st->L.io_y), stream);
+        if (rc) return rc;
+        if ((e = cudaMemcpyAsync(y, b + st->L.io_y, nq * 4, cudaMemcpyDeviceToHost, s)))
+            return cuda_fail(e, "device-to-host copy");
+        return LOLA_OK;
+    }
+    // Pipelined: the call is split at chunk boundaries into kHostSegments calls (a
+    // split call equals one call).  Segment i's inputs are copied in on s_in while
+    // segment i-1 computes on s and segment i-2's output is copied back on s_back;
+    // staging is double-buffered inside the io region (two segments fit because a
+    // segment is at most half of max_tokens).
+    const int seg_chunks = (nc + kHostSegments - 1) / kHostSegments;
+    const int Ts = seg_chunks * dm.C;
+    const size_t rq = (size_t)dm.Hq * dm.d, rk = (size_t)dm.Hkv * dm.d;      // elements per token
+    const size_t half_q = (size_t)dm.B * Ts * rq, half_k = (size_t)dm.B * Ts * rk;
+    if ((e = cudaEventRecord(st->ev_fork, s)) || (e = cudaStreamWaitEvent(st->s_in, st->ev_fork, 0)) ||
+        (e = cudaStreamWaitEvent(st->s_back, st->ev_fork, 0)))
+        return cuda_fail(e, "ordering the host-buffer copies");
+    int nseg = 0;
+    for (int t0 = 0; t0 < T; t0 += Ts, ++nseg) {
+        const int bi = nseg & 1, Tl = std::min(Ts, T - t0);
+        char* sq = b + st->L.io_q + bi * half_q * dm.esize;
+        char* sk = b + st->L.io_k + bi * half_k * dm.esize;
+        char* sv = b + st->L.io_v + bi * half_k * dm.esize;
+        float* sy = (float*)(b + st->L.io_y) + bi * half_q;
+        // inputs of this segment, once the compute that last used this buffer is done
+        if (nseg >= 2 && (e = cudaStreamWaitEvent(st->s_in, st->ev_done[bi], 0))) return cuda_fail(e, "ordering");
+        const size_t wq = Tl * rq * dm.esize, wk = Tl * rk * dm.esize;
+        if ((e = cudaMemcpy2DAsync(sq, wq, (const char*)q + t0 * rq * dm.esize, (size_t)T * rq * dm.esize, wq, dm.B,
+                                   cudaMemcpyHostToDevice, st->s_in)) ||
+            (e = cudaMemcpy2DAsync(sk, wk, (const char*)k + t0 * rk * dm.esize, (size_t)T * rk * dm.esize, wk, dm.B,
+                                   cudaMemcpyHostToDevice, st->s_in)) ||
+            (e = cudaMemcpy2DAsync(sv, wk, (const char*)v + t0 * rk * dm.esize, (size_t)T * rk * dm.esize, wk, dm.B,
+                                   cudaMemcpyHostToDevice, st->s_in)) ||
+            (e = cudaEventRecord(st->ev_in[bi], st->s_in)))
+            return cuda_fail(e, "host-to-device copy");
+        // compute, once the inputs are in and the output buffer has been copied back
+        if ((e = cudaStreamWaitEvent(s, st->ev_in[bi], 0)) ||
+            (nseg >= 2 && (e = cudaStreamWaitEvent(s, st->ev_back[bi], 0))))
+            return cuda_fail(e, "ordering");
+        int rc = lola_prefill_chunked(st, sq, sk, sv, Tl, sy, stream);
+        if (rc) return rc;
+        if ((e = cudaEventRecord(st->ev_done[bi], s)) || (e = cudaStreamWaitEvent(st->s_back, st->ev_done[bi], 0)))
+            return cuda_fail(e, "ordering");
+        const size_t wy = Tl * rq * 4;
+        if ((e = cudaMemcpy2DAsync((char*)y + t0 * rq * 4, (size_t)T * rq * 4, sy, wy, wy, dm.B,
+                                   cudaMemcpyDeviceToHost, st->s_back)) ||
+            (e = cudaEventRecord(st->ev_back[bi], st->s_back)))
+            return cuda_fail(e, "device-to-host copy");
+    }
+    // the caller's stream resumes after the last copies back
+    for (int bi = 0; bi < std::min(nseg, 2); ++bi)
+        if ((e = cudaStreamWaitEvent(s, st->ev_back[bi], 0))) return cuda_fail(e, "joining the copy streams");
     return LOLA_OK;
 }
 

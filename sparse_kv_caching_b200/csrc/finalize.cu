@@ -14,6 +14,13 @@ namespace lola {
 
 constexpr int kSlotsPerBlock = 32;
 
+// A row of the state is copied as 16-byte pieces: k and v (d elements each) then
+// phi(k) (D floats); all rows start on 16-byte boundaries.
+struct RowPieces {
+    int kp, fp, per;                  // pieces of k (= of v), of phi, of a whole row
+    __device__ RowPieces(const Dims& dm) : kp(dm.d * dm.esize / 16), fp(dm.D / 4), per(2 * kp + fp) {}
+};
+
 template <typename TIn>
 __global__ void __launch_bounds__(256) finalize_cache_kernel(const __grid_constant__ PrefillArgs a) {
     const Dims& dm = a.dm;
@@ -22,17 +29,22 @@ __global__ void __launch_bounds__(256) finalize_cache_kernel(const __grid_consta
     const int j0 = blockIdx.y * kSlotsPerBlock, nj = min(kSlotsPerBlock, lam - j0);
     const size_t snaps = (size_t)dm.nc_max + 1;
     const int* fin = a.snap_pos + ((size_t)st * snaps + a.nc) * lam;
-    const int per = 2 * d + D;
-    for (int idx = threadIdx.x; idx < nj * per; idx += 256) {
-        const int j = j0 + idx / per, x = idx % per;
+    const RowPieces rp(dm);
+    for (int idx = threadIdx.x; idx < nj * rp.per; idx += 256) {
+        const int j = j0 + idx / rp.per, x = idx % rp.per;
         const int p = fin[j];
         const size_t cs = (size_t)st * lam + j;
         if (x == 0) a.sp.cache_pos[cs] = p;
         if (p < 0 || p < a.t_start - eta) continue;      // empty, or cached before this call
         const PairRef<TIn> r = pair_ref<TIn>(a, st, b, g, p, j);
-        if (x < d) ((TIn*)a.sp.cache_k)[cs * d + x] = r.k[x];
-        else if (x < 2 * d) ((TIn*)a.sp.cache_v)[cs * d + (x - d)] = r.v[x - d];
-        else a.sp.cache_phik[cs * D + (x - 2 * d)] = r.phik[x - 2 * d];
+        if (x < rp.kp)
+            reinterpret_cast<uint4*>((TIn*)a.sp.cache_k + cs * d)[x] = reinterpret_cast<const uint4*>(r.k)[x];
+        else if (x < 2 * rp.kp)
+            reinterpret_cast<uint4*>((TIn*)a.sp.cache_v + cs * d)[x - rp.kp] =
+                reinterpret_cast<const uint4*>(r.v)[x - rp.kp];
+        else
+            reinterpret_cast<float4*>(a.sp.cache_phik + cs * D)[x - 2 * rp.kp] =
+                reinterpret_cast<const float4*>(r.phik)[x - 2 * rp.kp];
     }
 }
 
@@ -45,15 +57,20 @@ __global__ void __launch_bounds__(256) finalize_window_kernel(const __grid_const
     const int p_lo = max(a.t_start, t_end - eta);
     const int p0 = p_lo + blockIdx.y * kSlotsPerBlock;
     const int np = min(kSlotsPerBlock, t_end - p0);
-    const int per = 2 * d + D;
-    for (int idx = threadIdx.x; idx < np * per; idx += 256) {
-        const int p = p0 + idx / per, x = idx % per;
+    const RowPieces rp(dm);
+    for (int idx = threadIdx.x; idx < np * rp.per; idx += 256) {
+        const int p = p0 + idx / rp.per, x = idx % rp.per;
         const size_t i = (size_t)(p - a.t_start);
         const size_t off = (((size_t)b * a.T + i) * dm.Hkv + g) * d;
         const size_t ws = (size_t)st * eta + (size_t)(p % eta);
-        if (x < d) ((TIn*)a.sp.win_k)[ws * d + x] = ((const TIn*)a.k)[off + x];
-        else if (x < 2 * d) ((TIn*)a.sp.win_v)[ws * d + (x - d)] = ((const TIn*)a.v)[off + (x - d)];
-        else a.sp.win_phik[ws * D + (x - 2 * d)] = a.phik_new[((size_t)st * dm.max_tokens + i) * D + (x - 2 * d)];
+        if (x < rp.kp)
+            reinterpret_cast<uint4*>((TIn*)a.sp.win_k + ws * d)[x] = reinterpret_cast<const uint4*>((const TIn*)a.k + off)[x];
+        else if (x < 2 * rp.kp)
+            reinterpret_cast<uint4*>((TIn*)a.sp.win_v + ws * d)[x - rp.kp] =
+                reinterpret_cast<const uint4*>((const TIn*)a.v + off)[x - rp.kp];
+        else
+            reinterpret_cast<float4*>(a.sp.win_phik + ws * D)[x - 2 * rp.kp] =
+                reinterpret_cast<const float4*>(a.phik_new + ((size_t)st * dm.max_tokens + i) * D)[x - 2 * rp.kp];
     }
 }
 

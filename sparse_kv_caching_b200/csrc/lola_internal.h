@@ -61,6 +61,7 @@ struct PrefillArgs {
     int T;                 // tokens in this call
     int t_start;           // position of the first token of the call
     int nc;                // chunks in this call
+    int c_begin, c_end;    // chunks [c_begin, c_end) of the call served by this launch (scan, output)
     float* phik_new;       // [S][max_tokens][D]
     int* snap_pos;         // [S][nc_max+1][lambda]
     float* snap_H;         // [S][nc_max+1][d][D] (H_c transposed)

@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(256) output_kernel(const __grid_constant__ Pre
     float* Ws = Kt;                                   // W is only needed before the key loop
     const Dims& dm = a.dm;
     const int nqb = (dm.C + QB - 1) / QB;
-    const int c = blockIdx.x / nqb, qb = blockIdx.x % nqb;
+    const int c = a.c_begin + (int)blockIdx.x / nqb, qb = blockIdx.x % nqb;
     const int h = blockIdx.y, b = blockIdx.z;
     const int g = h / dm.Gq, st = b * dm.Hkv + g;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -211,7 +211,7 @@ static cudaError_t launch_out_t(const PrefillArgs& a, cudaStream_t s) {
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     const int nqb = (a.dm.C + Sh::QB - 1) / Sh::QB;
-    dim3 grid(a.nc * nqb, a.dm.Hq, a.dm.B);
+    dim3 grid((a.c_end - a.c_begin) * nqb, a.dm.Hq, a.dm.B);
     output_kernel<DIM, DH, TIn><<<grid, 256, bytes, s>>>(a);
     return cudaGetLastError();
 }

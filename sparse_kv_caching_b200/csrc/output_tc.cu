@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(128, 2) output_tc_kernel(const __grid_constant
     const Dims& dm = a.dm;
     const int rows_total = dm.Gq * dm.C;
     const int nrb = (rows_total + ROWS - 1) / ROWS;
-    const int c = blockIdx.x / nrb, rb = blockIdx.x % nrb;
+    const int c = a.c_begin + (int)blockIdx.x / nrb, rb = blockIdx.x % nrb;
     const int g = blockIdx.y, b = blockIdx.z, st = b * dm.Hkv + g;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int t0 = a.t_start + c * dm.C;
@@ -356,7 +356,7 @@ static cudaError_t launch_tc_t(const PrefillArgs& a, cudaStream_t s) {
                                          Sh::total);
     if (e != cudaSuccess) return e;
     const int nrb = (a.dm.Gq * a.dm.C + Sh::ROWS - 1) / Sh::ROWS;
-    dim3 grid(a.nc * nrb, a.dm.Hkv, a.dm.B);
+    dim3 grid((a.c_end - a.c_begin) * nrb, a.dm.Hkv, a.dm.B);
     output_tc_kernel<DIM, DH><<<grid, 128, Sh::total, s>>>(a);
     return cudaGetLastError();
 }

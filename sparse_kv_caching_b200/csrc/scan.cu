@@ -56,6 +56,14 @@ __host__ __device__ inline ScanOffsets scan_offsets(int D, int DV, int lam, int 
     return o;
 }
 
+// Slot positions entering chunk a.c_begin: the cache at the start of the call, or
+// the snapshot a previous launch of the same call published for that chunk.
+__device__ __forceinline__ const int* entering_slots(const PrefillArgs& a, int st) {
+    const Dims& dm = a.dm;
+    return a.c_begin == 0 ? a.sp.cache_pos + (size_t)st * dm.lam
+                          : a.snap_pos + ((size_t)st * (dm.nc_max + 1) + a.c_begin) * dm.lam;
+}
+
 // keep[i] = 1 for the lam candidates with the largest (score, -position);
 // exact: a 4-pass MSB radix select over the fp32 score bits (scores >= 0, so
 // the bit pattern orders like the value), then the candidates equal to the
@@ -151,7 +159,8 @@ __global__ void __launch_bounds__(kThreads, 1) scan_kernel(PrefillArgs a) {
     for (int i = tid; i < D * DV / 4; i += kThreads)
         reinterpret_cast<float4*>(Hs)[i] = reinterpret_cast<const float4*>(Hg)[i];
     for (int i = tid; i < D; i += kThreads) ss[i] = sg[i];
-    for (int j = tid; j < lam; j += kThreads) slot_pos[j] = a.sp.cache_pos[(size_t)st * lam + j];
+    const int* slots_in = entering_slots(a, st);
+    for (int j = tid; j < lam; j += kThreads) slot_pos[j] = slots_in[j];
     __syncthreads();
 
     auto publish = [&](int c) {
@@ -168,13 +177,13 @@ __global__ void __launch_bounds__(kThreads, 1) scan_kernel(PrefillArgs a) {
         }
         for (int i = tid; i < D; i += kThreads) sS[i] = ss[i];
     };
-    publish(0);
+    if (a.c_begin == 0) publish(0);
 
     // fold-phase thread layout: rows ty*RPT.., columns 4tx..4tx+3
     constexpr int TXF = DV / 4, TYF = kThreads / TXF, RPT = D / TYF, TF = 32, LDV = DV + 4;
     const int ftx = tid % TXF, fty = tid / TXF;
 
-    for (int c = 0; c < a.nc; ++c) {
+    for (int c = a.c_begin; c < a.c_end; ++c) {
         const int t0 = a.t_start + c * C;
         const int n_g = min(lam, max(0, t0 - eta));
         const int l_lo = max(0, t0 - eta), l_hi = max(0, t0 + C - eta);
@@ -560,9 +569,10 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
         umma::cp_async16(Hs + j * CW + 4 * u, Hg + (size_t)j * DV + col0 + 4 * u);
     }
     for (int i = tid; i < D / 4; i += NT) umma::cp_async16(ss + 4 * i, a.sp.s + (size_t)st * D + 4 * i);
-    const int n_g0 = min(lam, max(0, a.t_start - eta));
+    const int n_g0 = min(lam, max(0, a.t_start + a.c_begin * C - eta));
+    const int* slots_in = entering_slots(a, st);
     for (int j = tid; j < lam; j += NT) {
-        slot_pos[j] = a.sp.cache_pos[(size_t)st * lam + j];
+        slot_pos[j] = slots_in[j];
         slot_row[j] = j;
     }
     for (int k = tid; k < P - n_g0; k += NT) free_rows[k] = P - 1 - k;      // popped from the top
@@ -574,7 +584,7 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
     // always commits one cp.async group
     auto prefetch = [&](int c) {
         int n_l = 0, l_lo = 0;
-        if (c < a.nc) {
+        if (c < a.c_end) {
             const int t0 = a.t_start + c * C;
             l_lo = max(0, t0 - eta);
             n_l = max(0, t0 + C - eta) - l_lo;
@@ -584,7 +594,7 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
               [&](int i) { return free_rows[nfree - 1 - i]; });
         nfree -= n_l;
     };
-    prefetch(0);
+    prefetch(a.c_begin);
 
     const size_t snaps = (size_t)dm.nc_max + 1;
     auto snapH = [&](int c) { return a.snap_H + ((size_t)st * snaps + c) * D * DV; };   // H_c^T [DV][D]
@@ -608,8 +618,10 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
     };
     umma::cp_async_wait<1>();                                  // state and resident rows landed
     __syncthreads();
-    publish_H(0);
-    publish_pos_s(0, true);
+    if (a.c_begin == 0) {
+        publish_H(0);
+        publish_pos_s(0, true);
+    }
 
     // Partial SRE over this CTA's columns (notes §2.3, Eq. 10) of candidates [0, n):
     // for each candidate, den_e = phi_e . s and pred = H^T phi_e restricted to the
@@ -688,7 +700,7 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
     };
 
     int pb = 0;
-    for (int c = 0; c < a.nc; ++c) {
+    for (int c = a.c_begin; c < a.c_end; ++c) {
         const int t0 = a.t_start + c * C;
         const int n_g = min(lam, max(0, t0 - eta));
         const int l_lo = max(0, t0 - eta), n_l = max(0, t0 + C - eta) - l_lo;
@@ -921,7 +933,8 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cg_kernel(const __grid_con
     }
     for (int i = tid; i < D / 4; i += NT) umma::cp_async16(ss + 4 * i, a.sp.s + (size_t)st * D + 4 * i);
     umma::cp_async_commit();
-    for (int j = tid; j < lam; j += NT) slot_pos[j] = a.sp.cache_pos[(size_t)st * lam + j];
+    const int* slots_in = entering_slots(a, st);
+    for (int j = tid; j < lam; j += NT) slot_pos[j] = slots_in[j];
     umma::cp_async_wait<0>();
     __syncthreads();
 
@@ -944,8 +957,10 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cg_kernel(const __grid_con
             dst[0] = h.x; dst[D] = h.y; dst[2 * D] = h.z; dst[3 * D] = h.w;
         }
     };
-    publish_H(0);
-    publish_pos_s(0, true);
+    if (a.c_begin == 0) {
+        publish_H(0);
+        publish_pos_s(0, true);
+    }
 
     // partial SRE (notes §2.3, Eq. 10) of the cnt candidates e0.. held in tile bi;
     // thread (tx, ty) takes 8 columns of EPT rows, out-of-range rows repeat a valid one
@@ -1019,7 +1034,7 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cg_kernel(const __grid_con
     };
 
     int pb = 0;
-    for (int c = 0; c < a.nc; ++c) {
+    for (int c = a.c_begin; c < a.c_end; ++c) {
         const int t0 = a.t_start + c * C;
         const int n_g = min(lam, max(0, t0 - eta));
         const int l_lo = max(0, t0 - eta), n_l = max(0, t0 + C - eta) - l_lo;

@@ -126,6 +126,17 @@ def test_split_calls_match_single_call():
     _check_small(w, splits=[128, 448])
 
 
+def test_segmented_call_matches_unsegmented_calls():
+    """A call of >= 32 chunks runs its chain in segments with the outputs overlapped;
+    it must equal, bit for bit, calls of one segment each (which do not split)."""
+    w = P.small_workload(2, B=1, Hkv=2, Hq=4, T=2048, eta=64, lam=64, chunk=64)
+    _, y1, ex1, _, _ = _run_small(w)
+    _, y2, ex2, _, _ = _run_small(w, splits=[512, 1024, 1536])
+    assert torch.equal(y1, y2)
+    assert torch.equal(ex1["H"], ex2["H"]) and torch.equal(ex1["s"], ex2["s"])
+    assert torch.equal(ex1["cache_pos"], ex2["cache_pos"])
+
+
 def _decode_check(w, T_pre, steps, streams, chunk_pre=None):
     """Prefill T_pre tokens, then `steps` decode steps; compare sampled streams each step."""
     full = synth.full_arrays(w)
@@ -224,6 +235,27 @@ def test_host_buffer_entry_points_match_device():
                        dev["v"][:, t].cpu().pin_memory(), hyd)
         torch.cuda.synchronize()
         assert torch.equal(hyd, yd.cpu())
+
+
+@pytest.mark.parametrize("T,Tpad", [(640, 640), (2240, 2560)])
+def test_pipelined_host_prefill_matches_device(T, Tpad):
+    """Host-buffer prefill of >= 8 chunks runs as segments whose copies overlap the
+    compute (strided copies for B > 1, a short last segment, a state with spare
+    capacity); it must equal the device-buffer call bit for bit, state included."""
+    w = P.small_workload(2, B=2, Hkv=2, Hq=4, T=T, eta=64, lam=96, chunk=64)
+    full = synth.full_arrays(w)
+    dev = P.to_device(w, full)
+    l1 = P.make_layer(w, dev["W"], max_tokens=Tpad)
+    l2 = P.make_layer(w, dev["W"], max_tokens=Tpad)
+    y1 = l1.prefill(dev["q"], dev["k"], dev["v"])
+    hq, hk, hv = (dev[x].cpu().pin_memory() for x in ("q", "k", "v"))
+    hy = torch.full(y1.shape, float("nan"), dtype=torch.float32).pin_memory()
+    l2.prefill_host(hq, hk, hv, hy)
+    torch.cuda.synchronize()
+    assert torch.equal(hy, y1.cpu())
+    e1, e2 = l1.export(), l2.export()
+    for key in ("H", "s", "cache_pos", "cache_k", "cache_v", "win_k", "win_v"):
+        assert torch.equal(e1[key], e2[key]), key
 
 
 def test_invalid_arguments_are_errors():
