@@ -21,7 +21,9 @@
  *   - The caller owns every buffer.  The library allocates no device memory:
  *     persistent state and per-call scratch live in the caller's `dev_buf`,
  *     sized by lola_state_bytes().  The library owns only the small host
- *     handle returned by lola_state_init().
+ *     handle returned by lola_state_init() and, per handle, four CUDA
+ *     streams and a few events (no device memory), released by
+ *     lola_state_free().
  *   - Return value 0 = LOLA_OK; a negative value is one of the LOLA_ERR_*
  *     codes below and lola_last_error_string() describes it (thread-local).
  *     No entry point aborts the process or traps on the device.
@@ -132,7 +134,12 @@ int lola_state_free(lola_state* st);
  * cached (older position wins exact ties) and the rest are folded (Eqs.
  * 12-13).  q, k, v: device, layouts above; y: device float32 [B][T][Hq][d].
  * T must be a positive multiple of chunk and <= max_tokens.  Calls may split
- * a sequence at any chunk-aligned point; the result equals one call. */
+ * a sequence at any chunk-aligned point; the result equals one call.
+ * A call of >= 32 chunks runs the memory-update chain in four chunk segments
+ * on an internal high-priority stream and each segment's output on an
+ * internal low-priority stream, forked from and joined back into `stream`
+ * with events: the call stays stream-ordered on `stream` (and can be captured
+ * into a CUDA graph), and its results equal those of one segment. */
 int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const void* v,
                          int T, float* y, void* stream);
 
@@ -143,7 +150,10 @@ int lola_decode_step(lola_state* st, const void* q, const void* k, const void* v
 
 /* Same as lola_prefill_chunked / lola_decode_step, with pinned HOST buffers:
  * the inputs are copied into device staging inside dev_buf, the layer runs,
- * and y is copied back, all enqueued on `stream` (synchronise before reading y). */
+ * and y is copied back, all ordered on `stream` (synchronise before reading y).
+ * A prefill of >= 8 chunks runs as four chunk-aligned calls whose copies in
+ * and back run on internal streams, overlapped with the neighbouring
+ * segments' compute (double-buffered staging); the result equals one call. */
 int lola_prefill_chunked_host(lola_state* st, const void* q, const void* k, const void* v,
                               int T, float* y, void* stream);
 int lola_decode_step_host(lola_state* st, const void* q, const void* k, const void* v,
