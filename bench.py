@@ -334,9 +334,9 @@ def run_sweep(args):
             prof = layer.profile_read()
             layer.profile(False)
             ms = total / args.steps
-            kern = {kk: round(prof[kk][0] / max(1, prof[kk][1]), 4) for kk in ("phi", "scan", "output", "finalize")}
+            kern = {kk: round(prof[kk][0] / args.steps, 4) for kk in ("phi", "scan", "output", "finalize")}
             points.append({"eta": eta, "lambda": lam, "ms": round(ms, 4),
-                           "tokens_per_s": w.B * w.T / (ms / 1e3), "kernel_ms": kern})
+                           "tokens_per_s": w.B * w.T / (ms / 1e3), "kernel_ms_per_step": kern})
             layer.close()
             del layer
     line = {"metric": "single-layer prefill latency over the (eta, lambda) grid", "unit": "ms",

@@ -336,21 +336,32 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
     a.err = (int*)(st->base + st->L.err);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if ((e = traced(st, 0, 1, s, [&] { return lola::launch_phi_keys(a, s); })) != cudaSuccess)
-        return cuda_fail(e, "feature-map kernel");
     auto output = [&](cudaStream_t q) {
         return dm.dtype == LOLA_DTYPE_BF16 ? lola::launch_output_tc(a, q) : lola::launch_output(a, q);
     };
     const int seg = a.nc >= kSplitMinChunks ? (a.nc + kSplitSegments - 1) / kSplitSegments : a.nc;
     if (st->s_chain && seg < a.nc) {
         // The chain of segment i and the output of segment i-1 run at the same time:
-        // the chain holds one cluster per stream, the output fills the other SMs.
+        // the chain holds one cluster per stream, the output fills the other SMs.  The
+        // feature map of the first segment's keys runs first; the rest of the keys
+        // are mapped on the output stream while the first segment's chain runs.
+        a.c_end = seg;
+        if ((e = traced(st, 0, 1, s, [&] { return lola::launch_phi_keys(a, s); })) != cudaSuccess)
+            return cuda_fail(e, "feature-map kernel");
         if ((e = cudaEventRecord(st->ev_fork, s)) || (e = cudaStreamWaitEvent(st->s_chain, st->ev_fork, 0)) ||
             (e = cudaStreamWaitEvent(st->s_out, st->ev_fork, 0)))
             return cuda_fail(e, "forking the prefill streams");
+        a.c_begin = seg;
+        a.c_end = a.nc;
+        if ((e = traced(st, 0, 1, st->s_out, [&] { return lola::launch_phi_keys(a, st->s_out); })) != cudaSuccess)
+            return cuda_fail(e, "feature-map kernel");
+        if ((e = cudaEventRecord(st->ev_join_out, st->s_out)))
+            return cuda_fail(e, "ordering the feature map");
         for (int c0 = 0; c0 < a.nc; c0 += seg) {
             a.c_begin = c0;
             a.c_end = std::min(a.nc, c0 + seg);
+            if (c0 == seg && (e = cudaStreamWaitEvent(st->s_chain, st->ev_join_out, 0)))
+                return cuda_fail(e, "ordering the feature map");
             if ((e = traced(st, 1, 1, st->s_chain, [&] { return lola::launch_scan(a, st->s_chain); })) != cudaSuccess)
                 return cuda_fail(e, "scan kernel");
             if ((e = cudaEventRecord(st->ev_seg, st->s_chain)) || (e = cudaStreamWaitEvent(st->s_out, st->ev_seg, 0)))
@@ -364,6 +375,8 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
             (e = cudaStreamWaitEvent(s, st->ev_join_chain, 0)) || (e = cudaStreamWaitEvent(s, st->ev_join_out, 0)))
             return cuda_fail(e, "joining the prefill streams");
     } else {
+        if ((e = traced(st, 0, 1, s, [&] { return lola::launch_phi_keys(a, s); })) != cudaSuccess)
+            return cuda_fail(e, "feature-map kernel");
         if ((e = traced(st, 1, 1, s, [&] { return lola::launch_scan(a, s); })) != cudaSuccess)
             return cuda_fail(e, "scan kernel");
         if ((e = traced(st, 2, 1, s, [&] { return output(s); })) != cudaSuccess)

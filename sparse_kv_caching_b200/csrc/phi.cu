@@ -4,6 +4,7 @@
 // this library fixes the Hedgehog form with per-kv-head W.  fp32 FFMA with
 // W staged in shared memory, exact softmax via expf.  Output layout
 // phik_new [S][max_tokens][D] (row i = token t_start + i of stream st).
+// A launch covers the tokens of chunks [c_begin, c_end) of the call.
 #include "device_common.cuh"
 
 namespace lola {
@@ -20,9 +21,10 @@ __global__ void __launch_bounds__(256) phi_keys_kernel(PrefillArgs a) {
     const TIn* Wg = (const TIn*)a.sp.W + (size_t)g * DIM * DH;
     for (int i = threadIdx.x; i < DIM * DH; i += 256) Ws[i] = to_f32(Wg[i]);
     __syncthreads();
+    const int i_end = a.c_end * dm.C;
     for (int r = 0; r < ROWS_PER_WARP; ++r) {
-        const int i = (blockIdx.x * 8 + warp) * ROWS_PER_WARP + r;
-        if (i >= a.T) break;
+        const int i = a.c_begin * dm.C + (blockIdx.x * 8 + warp) * ROWS_PER_WARP + r;
+        if (i >= i_end) break;
         const TIn* x = (const TIn*)a.k + (((size_t)b * a.T + i) * dm.Hkv + g) * DIM;
         for (int j = lane; j < DIM; j += 32) xs[warp][j] = to_f32(x[j]);
         __syncwarp();
@@ -62,7 +64,8 @@ __global__ void __launch_bounds__(256) phi_keys_kernel(PrefillArgs a) {
 template <int DIM, int DH, typename TIn>
 static cudaError_t launch_phi_t(const PrefillArgs& a, cudaStream_t s) {
     const int rows_per_block = 8 * 4;
-    dim3 grid((a.T + rows_per_block - 1) / rows_per_block, a.dm.S);
+    const int rows = (a.c_end - a.c_begin) * a.dm.C;
+    dim3 grid((rows + rows_per_block - 1) / rows_per_block, a.dm.S);
     phi_keys_kernel<DIM, DH, TIn><<<grid, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
