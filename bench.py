@@ -123,13 +123,14 @@ def kernel_source_hash() -> str:
 
 
 def traffic_for(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernels."""
+    """DRAM bytes (per step for prefill kernel classes, per launch for decode) from the
+    committed ncu summary, if it was taken on the current kernels."""
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
         ent = t.get(f"{kernel}@{workload}")
         if ent and ent.get("source_hash") == kernel_source_hash():
-            return ent["dram_bytes_per_launch"]
+            return ent.get("dram_bytes_per_step", ent.get("dram_bytes_per_launch"))
     except Exception:
         pass
     return None
