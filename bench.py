@@ -98,6 +98,23 @@ def decode_step_flops(w: synth.Workload) -> int:
 SM_MAX_MHZ = 1965          # clocks.max.sm of the B200s here
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The maximum of x over all ranks (the collective runs on `device`: the rank's
+    GPU under nccl, the CPU under gloo)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms_max / 1e3)
+
+
 def fp32_alu_peak_tflops(num_sms: int) -> float:
     """FP32 FMA peak of the CUDA cores: SMs x 128 lanes x 2 FLOP x max SM clock."""
     return num_sms * 128 * 2 * SM_MAX_MHZ * 1e6 / 1e12
@@ -397,12 +414,8 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def ranks_max(x: float) -> float:
+        return max_over_ranks(x, world, dev)
 
     peaks, peaks_kind = load_peaks()
     props = torch.cuda.get_device_properties(dev)
@@ -447,9 +460,8 @@ def main():
     prof = layer.profile_read()
     layer.profile(False)
     clk = clocks.stop()
-    ms_step = max_over_ranks(total_ms / args.steps)
-    tokens = w.B * w.T * world
-    value = tokens / (ms_step / 1e3)
+    ms_step = ranks_max(total_ms / args.steps)
+    value = job_throughput(w.B * w.T, world, ms_step)
 
     work = prefill_work(w)
     # dominant kernel by measured time
@@ -498,7 +510,7 @@ def main():
         ev1.record(stream)
         ev1.synchronize()
         e2e_ms += ev0.elapsed_time(ev1)
-    e2e_ms = max_over_ranks(e2e_ms / e2e_steps)
+    e2e_ms = ranks_max(e2e_ms / e2e_steps)
     h2d = hq.numel() * hq.element_size() + hk.numel() * hk.element_size() + hv.numel() * hv.element_size()
     d2h = hy.numel() * 4
     # y and trace of the last device-path step, for the oracle match
@@ -553,7 +565,7 @@ def main():
             ld.decode(qs[i], ks[i], vs[i], yd)
         ev1.record(stream)
         ev1.synchronize()
-        dms = max_over_ranks(ev0.elapsed_time(ev1) / steps_d)
+        dms = ranks_max(ev0.elapsed_time(ev1) / steps_d)
         pd = ld.profile_read()
         kms = pd["decode"][0] / max(1, pd["decode"][1])
         by = decode_step_bytes(wd)
