@@ -534,7 +534,7 @@ def main():
             "kernel_time_share": shares,
             "gpu_launches": launches,
             "clocks": clk,
-            "e2e": {"value": tokens / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+            "e2e": {"value": job_throughput(w.B * w.T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             }
     del layer, full, q, k, v, y, hq, hk, hv, hy

@@ -205,6 +205,18 @@ __global__ void __launch_bounds__(128, 2) output_tc_kernel(const __grid_constant
     const int N = n_g + n_w + qi_max + 1;
     const int ntiles = (N + KT - 1) / KT;
     const int* cpos = a.snap_pos + ((size_t)st * snaps + c) * dm.lam;
+    // positions of a tile's keys, one thread per key (one load per cache key, all
+    // in parallel); the copies then read them from shared memory
+    auto stage_pos = [&](int it, int buf) {
+        if (tid < KT) {
+            const int gk = it * KT + tid;
+            int pos = 0x7fffffff;
+            if (gk < n_g) pos = cpos[gk];
+            else if (gk < n_g + n_w) pos = w_lo + (gk - n_g);
+            else if (gk < N) pos = t0 + (gk - n_g - n_w);
+            kpos[buf * KT + tid] = pos;
+        }
+    };
     auto issue_tile = [&](int it, int buf) {
         uint8_t* sK = sKV + buf * 2 * Sh::KVB;
         uint8_t* sV = sK + Sh::KVB;
@@ -214,30 +226,32 @@ __global__ void __launch_bounds__(128, 2) output_tc_kernel(const __grid_constant
             const int gk = k0 + kk;
             uint8_t* dk = sK + j * KT * 16 + kk * 16;
             uint8_t* dv = sV + j * KT * 16 + kk * 16;
-            int pos = 0x7fffffff;
             if (gk < N) {
-                int slot = 0;
-                if (gk < n_g) { slot = gk; pos = cpos[gk]; }
-                else if (gk < n_g + n_w) pos = w_lo + (gk - n_g);
-                else pos = t0 + (gk - n_g - n_w);
-                const PairRef<bf16> r = pair_ref<bf16>(a, st, b, g, pos, slot);
+                const PairRef<bf16> r = pair_ref<bf16>(a, st, b, g, kpos[buf * KT + kk], gk < n_g ? gk : 0);
                 umma::cp_async16(dk, r.k + 8 * j);
                 umma::cp_async16(dv, r.v + 8 * j);
             } else {
                 st_shared_v4(dk, 0u, 0u, 0u, 0u);
                 st_shared_v4(dv, 0u, 0u, 0u, 0u);
             }
-            if (j == 0) kpos[buf * KT + kk] = pos;
         }
         umma::cp_async_commit();
     };
     const float c2 = 1.4426950408889634f / sqrtf((float)DIM);   // log2(e) / sqrt(d)
     float m_ref = 0.f;
+    stage_pos(0, 0);
+    __syncthreads();
     issue_tile(0, 0);
     for (int it = 0; it < ntiles; ++it) {
         const int buf = it & 1;
-        if (it + 1 < ntiles) { issue_tile(it + 1, buf ^ 1); umma::cp_async_wait<1>(); }
-        else umma::cp_async_wait<0>();
+        if (it + 1 < ntiles) {
+            stage_pos(it + 1, buf ^ 1);            // buffer buf^1 was last read by tile it-1
+            __syncthreads();
+            issue_tile(it + 1, buf ^ 1);
+            umma::cp_async_wait<1>();
+        } else {
+            umma::cp_async_wait<0>();
+        }
         umma::fence_async_smem();
         umma::fence_before_sync();
         __syncthreads();
