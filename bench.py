@@ -129,13 +129,18 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# Sources a kernel class's counters depend on: its own files plus the shared headers.
+KERNEL_SOURCES = {"phi": ["phi.cu"], "scan": ["scan.cu"], "output": ["output_tc.cu", "output.cu"],
+                  "finalize": ["finalize.cu"], "decode": ["decode.cu"]}
+SHARED_SOURCES = ["device_common.cuh", "lola_internal.h", "umma.cuh"]
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "sparse_kv_caching_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + fh.read())
+    for f in sorted(KERNEL_SOURCES[kernel] + SHARED_SOURCES):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -146,7 +151,7 @@ def traffic_for(kernel: str, workload: str):
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
         ent = t.get(f"{kernel}@{workload}")
-        if ent and ent.get("source_hash") == kernel_source_hash():
+        if ent and ent.get("source_hash") == kernel_source_hash(kernel):
             return ent.get("dram_bytes_per_step", ent.get("dram_bytes_per_launch"))
     except Exception:
         pass
