@@ -31,12 +31,16 @@ struct TcShape {
     static constexpr int MBAR = KPOS + 2 * KT * 4;
     static constexpr int TPTR = MBAR + 16;
     static constexpr int total = TPTR + 16;
-    // prologue aliases inside the KV region
-    static constexpr int PHI = KV;                            // [128 rows x 32 j] f32
-    static constexpr int HT = KV + ROWS * 32 * 4;             // [DIM rows x 32 j] f32
-    static constexpr int SC = HT + DIM * 32 * 4;              // s_c [D] f32
+    // prologue aliases: all D/32 chunks of H_c^T in the KV region, the phi(q) chunk
+    // in the P region (after W has served the z product), s_c in the KPOS region
+    static constexpr int HT = KV;                             // [D/32][DIM rows x 32 j] f32
+    static constexpr int HTC = DIM * 32 * 4;                  // one chunk (bytes)
+    static constexpr int PHI = P;                             // [128 rows x 32 j] f32
+    static constexpr int SC = KPOS;                           // s_c [D] f32
     static constexpr int TMEM_COLS = (DIM + KT <= 128) ? 128 : 256;
-    static_assert(SC + D * 4 <= P, "prologue buffers must fit in the KV region");
+    static_assert(HT + (D / 32) * HTC <= P, "H_c^T must fit in the KV region");
+    static_assert(ROWS * 32 * 4 <= ROWS * KT * 2, "a phi chunk must fit in the P region");
+    static_assert(D * 4 <= 2 * KT * 4, "s_c must fit in the KPOS region");
     static_assert(DIM * DH * 2 <= ROWS * KT * 2, "W must fit in the P region");
 };
 
@@ -117,6 +121,11 @@ __global__ void __launch_bounds__(128, 2) output_tc_kernel(const __grid_constant
             umma::cp_async16(sP + n8 * DIM * 16 + k * 16, Wg + (size_t)k * DH + 8 * n8);
         }
         for (int idx = tid; idx < D / 4; idx += 128) umma::cp_async16(s_c + 4 * idx, sc_g + 4 * idx);
+        // every chunk of H_c^T at once: rows cc of 32 j each, 8 groups of 4 j
+        for (int idx = tid; idx < (D / 32) * DIM * 8; idx += 128) {
+            const int cc = idx % DIM, jq = (idx / DIM) % 8, ch = idx / (DIM * 8);
+            umma::cp_async16(smem + Sh::HT + ch * Sh::HTC + jq * DIM * 16 + cc * 16, Hc + (size_t)cc * D + 32 * ch + 4 * jq);
+        }
     }
     umma::cp_async_commit();
     umma::cp_async_wait<0>();
@@ -159,14 +168,9 @@ __global__ void __launch_bounds__(128, 2) output_tc_kernel(const __grid_constant
         for (int i = 0; i < DH; ++i) { sp += expf(z[i] - mx); sn += expf(mn - z[i]); }
         const float isp = 1.f / sp, isn = 1.f / sn;
         uint8_t* sPhi = smem + Sh::PHI;
-        uint8_t* sHt = smem + Sh::HT;
 #pragma unroll
         for (int jc = 0; jc < D; jc += 32) {
-            for (int idx = tid; idx < DIM * 8; idx += 128) {     // H_c^T rows, 8 chunks of 4 j
-                const int cc = idx % DIM, jq = idx / DIM;
-                umma::cp_async16(sHt + jq * DIM * 16 + cc * 16, Hc + (size_t)cc * D + jc + 4 * jq);
-            }
-            umma::cp_async_commit();
+            uint8_t* sHt = smem + Sh::HT + (jc / 32) * Sh::HTC;
 #pragma unroll
             for (int jq = 0; jq < 8; ++jq) {
                 float f[4];
@@ -179,7 +183,6 @@ __global__ void __launch_bounds__(128, 2) output_tc_kernel(const __grid_constant
                 st_shared_v4(sPhi + jq * ROWS * 16 + tid * 16, __float_as_uint(f[0]), __float_as_uint(f[1]),
                              __float_as_uint(f[2]), __float_as_uint(f[3]));
             }
-            umma::cp_async_wait<0>();
             umma::fence_async_smem();
             umma::fence_before_sync();
             __syncthreads();
