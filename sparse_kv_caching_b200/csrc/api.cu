@@ -139,6 +139,7 @@ lola::Layout make_layout(const lola::Dims& dm) {
     L.win_phik = take(S * dm.eta * dm.D * 4);
     L.cache_R = take(S * dm.lam * dm.d * 4);
     L.cache_den = take(S * dm.lam * 4);
+    L.cache_sc = take(S * dm.lam * 4);
     L.phik_new = take(S * T * dm.D * 4);
     L.snap_pos = take(S * snaps * dm.lam * 4);
     L.snap_H = take(S * snaps * dm.D * dm.d * 4);
@@ -167,6 +168,7 @@ lola::StatePtrs state_ptrs(const lola_state* st) {
     p.win_phik = (float*)(b + st->L.win_phik);
     p.cache_R = (float*)(b + st->L.cache_R);
     p.cache_den = (float*)(b + st->L.cache_den);
+    p.cache_sc = (float*)(b + st->L.cache_sc);
     return p;
 }
 

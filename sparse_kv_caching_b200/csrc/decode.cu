@@ -17,22 +17,22 @@
 // change of (H, s), after which R_e += k_e (v_f - v_e), den_e += k_e with
 // k_e = phi_e . phi_f: O(lambda (D + d)) work per step instead of
 // O(lambda D d), and no cancellation (the residual itself is stored).
-// residual_init_kernel computes them exactly from (H, s) after a prefill.
+// residual_init_kernel computes them exactly from (H, s) after a prefill.  The
+// pass that updates R_e also stores each member's SRE against the new state,
+// so the next step's scoring reads one float per member instead of R.
 #include "device_common.cuh"
 #include "umma.cuh"
 
 namespace lola {
 
 constexpr int kDecThreads = 256;
-constexpr int kDecBatch = 4;      // keys / residual rows a warp loads before consuming them
 constexpr int kDecSlotBatch = 8;  // slot rows per warp in flight while scoring
 
 struct DecOffsets {
     int Hs, ss, Ws, qs, phq, kn, vn, phk, phl, Pl, vf, phf, red, kp, sc, wm, R, part, total;
 };
 
-__host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int lam, int eta, bool r_smem,
-                                                  int esize) {
+__host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int lam, int eta, int esize) {
     const int D = 2 * DH, NK = lam + eta + 1, NW = kDecThreads / 32;
     DecOffsets o;
     int p = 0;
@@ -53,8 +53,8 @@ __host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int l
     o.kp = take(4 * NK);                   // key and value row pointers (64-bit each)
     o.sc = take(max(Gq * NK, lam + 1));    // slot scores (update phase)
     o.wm = take(NW * 8 * 2);               // per-warp softmax max and sum per head
-    // R [lam][DIM] (update phase) aliases the read-phase partial sums [NW][Gq][DIM]
-    o.R = take(max(max(r_smem ? lam * DIM : 0, NW * Gq * DIM), (DIM * DH * esize + 3) / 4 + (Gq + 1) * DH));
+    // the read-phase partial sums [NW][Gq][DIM] alias the z scratch and the staged W
+    o.R = take(max(NW * Gq * DIM, (DIM * DH * esize + 3) / 4 + (Gq + 1) * DH));
     o.part = o.R;
     o.Ws = o.R + (Gq + 1) * DH;           // after the z scratch rows
     o.total = p;
@@ -96,8 +96,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     const int Gq = dm.Gq, lam = dm.lam, eta = dm.eta, t = a.t;
     const int st = blockIdx.x, b = st / dm.Hkv, g = st % dm.Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const bool rsm = a.r_smem != 0;                 // residual rows staged in shared memory
-    const DecOffsets o = dec_offsets(DIM, DH, Gq, lam, eta, rsm, (int)sizeof(TIn));
+    const DecOffsets o = dec_offsets(DIM, DH, Gq, lam, eta, (int)sizeof(TIn));
     float* Hs = smem + o.Hs;
     float* ss = smem + o.ss;
     float* qs = smem + o.qs;
@@ -114,7 +113,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     float* sc = smem + o.sc;
     float* wm = smem + o.wm;
     float* Ws = smem + o.Ws;
-    float* Rs = smem + o.R;
     float* part = smem + o.part;
 
     float* Hg = a.sp.H + (size_t)st * D * DIM;
@@ -162,7 +160,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     if (leaving)
         for (int i = tid; i < D; i += NT) phl[i] = a.sp.win_phik[(wbase + rs) * D + i];
     __syncthreads();
-    float* zs = Rs;                                                   // scratch [Gq + 1][DH]
+    float* zs = smem + o.R;                                           // scratch [Gq + 1][DH]
     for (int idx = tid; idx < (Gq + 1) * DH; idx += NT) {
         const int r = idx / DH, col = idx % DH;
         const float* x = r < Gq ? qs + r * DIM : kn;
@@ -306,38 +304,22 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
             }
             for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
             if (tid == 0) { a.sp.cache_pos[cs] = lpos; deng[n_g] = den_l; }
-        } else {
-            // scores: slots from their residuals (one warp per slot), l from R_l
-            float* scs = red + 64;                                    // reuse as scratch for the argmin
-            {
-                constexpr int RQ = DIM / 4;
-                const int q4 = lane & 3, rq = lane >> 2;
-                for (int e0 = warp * 8; e0 < lam; e0 += NW * 8) {
-                    const int e = e0 + rq;
-                    float rv[RQ];
-                    float dn = 0.f;
-                    if (e < lam) { load_quarter<DIM>(Rg + (size_t)e * DIM, q4, rv); dn = deng[e]; }
-                    float q = 0.f;
-                    if (e < lam) {
-#pragma unroll
-                        for (int u = 0; u < RQ; ++u) q = fmaf(rv[u], rv[u], q);
-                        if (rsm)
-#pragma unroll
-                            for (int u = 0; u < RQ; ++u) Rs[e * DIM + qidx(q4, u)] = rv[u];
-                    }
-                    q = quad_sum(q);
-                    float vq = 0.f;
-                    if (e < lam && !(dn > 0.f)) {                     // empty memory: SRE = ||v||^2
-                        float vv[RQ];
-                        load_quarter<DIM>((const TIn*)a.sp.cache_v + (cbase + e) * DIM, q4, vv);
-#pragma unroll
-                        for (int u = 0; u < RQ; ++u) vq = fmaf(vv[u], vv[u], vq);
-                    }
-                    vq += __shfl_xor_sync(0xffffffffu, vq, 1);
-                    vq += __shfl_xor_sync(0xffffffffu, vq, 2);
-                    if (e < lam && q4 == 0) sc[e] = dn > 0.f ? q / (dn * dn) : vq;
+            if (warp == 0) {                                          // its SRE against the state
+                float q = 0.f, vq = 0.f;
+                for (int cc = lane; cc < DIM; cc += 32) {
+                    const float v = to_f32(vl[cc]);
+                    const float r = Pl[cc] - den_l * v;
+                    q = fmaf(r, r, q);
+                    vq = fmaf(v, v, vq);
                 }
+                q = warp_sum(q);
+                vq = warp_sum(vq);
+                if (lane == 0) a.sp.cache_sc[cs] = den_l > 0.f ? q / (den_l * den_l) : vq;
             }
+        } else {
+            // scores: members from the cache (stored when their residuals last changed), l from R_l
+            float* scs = red + 64;                                    // reuse as scratch for the argmin
+            for (int e = tid; e < lam; e += NT) sc[e] = a.sp.cache_sc[cbase + e];
             if (warp == 0) {
                 float q = 0.f, vq = 0.f;
                 for (int cc = lane; cc < DIM; cc += 32) {
@@ -394,12 +376,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                         load_quarter<D>(e < lam ? a.sp.cache_phik + (cbase + e) * D : phl, q4, pv);
                         load_quarter<DIM>(e < lam ? (const TIn*)a.sp.cache_v + (cbase + e) * DIM : vl, q4, vv);
                         if (e < lam) {
-                            if (rsm) {
-#pragma unroll
-                                for (int u = 0; u < RQ; ++u) r0[u] = Rs[e * DIM + qidx(q4, u)];
-                            } else {
-                                load_quarter<DIM>(Rg + (size_t)e * DIM, q4, r0);
-                            }
+                            load_quarter<DIM>(Rg + (size_t)e * DIM, q4, r0);
                             d0 = deng[e];
                         } else {
 #pragma unroll
@@ -413,17 +390,30 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                         for (int u = 0; u < PQ; ++u) kap = fmaf(pv[u], phf[qidx(q4, u)], kap);
                     }
                     kap = quad_sum(kap);
+                    float q = 0.f, vq = 0.f;
                     if (act) {
                         const int dst = e < lam ? e : f;   // its own slot, or f's slot for the newcomer l
                         float* rw = Rg + (size_t)dst * DIM;
 #pragma unroll
                         for (int u = 0; u < RQ; u += 4) {
                             const int c0 = qidx(q4, u);                       // 4 consecutive columns
-                            *reinterpret_cast<float4*>(rw + c0) = make_float4(
+                            const float4 r4 = make_float4(
                                 fmaf(kap, vf[c0] - vv[u], r0[u]), fmaf(kap, vf[c0 + 1] - vv[u + 1], r0[u + 1]),
                                 fmaf(kap, vf[c0 + 2] - vv[u + 2], r0[u + 2]), fmaf(kap, vf[c0 + 3] - vv[u + 3], r0[u + 3]));
+                            *reinterpret_cast<float4*>(rw + c0) = r4;
+                            q = fmaf(r4.x, r4.x, q); q = fmaf(r4.y, r4.y, q);
+                            q = fmaf(r4.z, r4.z, q); q = fmaf(r4.w, r4.w, q);
                         }
-                        if (q4 == 0) deng[dst] = d0 + kap;
+#pragma unroll
+                        for (int u = 0; u < RQ; ++u) vq = fmaf(vv[u], vv[u], vq);
+                    }
+                    q = quad_sum(q);
+                    vq = quad_sum(vq);
+                    if (act && q4 == 0) {
+                        const int dst = e < lam ? e : f;
+                        const float dn = d0 + kap;
+                        deng[dst] = dn;
+                        a.sp.cache_sc[cbase + dst] = dn > 0.f ? q / (dn * dn) : vq;   // SRE against the new state
                     }
                 }
             }
@@ -491,15 +481,26 @@ __global__ void __launch_bounds__(256) residual_init_kernel(const __grid_constan
         const float v = to_f32(((const TIn*)a.sp.cache_v)[(cbase + e0 + e) * DIM + cc]);
         a.sp.cache_R[(cbase + e0 + e) * DIM + cc] = x - den[e] * v;
     }
+    __syncthreads();
+    // each member's SRE against the state (warp per member), from the rows just written
+    for (int e = threadIdx.x >> 5; e < ne; e += 8) {
+        float q = 0.f, vq = 0.f;
+        for (int cc = threadIdx.x & 31; cc < DIM; cc += 32) {
+            const float r = a.sp.cache_R[(cbase + e0 + e) * DIM + cc];
+            const float v = to_f32(((const TIn*)a.sp.cache_v)[(cbase + e0 + e) * DIM + cc]);
+            q = fmaf(r, r, q);
+            vq = fmaf(v, v, vq);
+        }
+        q = warp_sum(q);
+        vq = warp_sum(vq);
+        if ((threadIdx.x & 31) == 0) a.sp.cache_sc[cbase + e0 + e] = den[e] > 0.f ? q / (den[e] * den[e]) : vq;
+    }
 }
 
 template <int DIM, int DH, typename TIn>
 static cudaError_t launch_dec_t(const DecodeArgs& a0, cudaStream_t s) {
-    DecodeArgs a = a0;
-    // two CTAs per SM hide more memory latency than staging the residual rows would save
-    const int es = (int)sizeof(TIn);
-    a.r_smem = dec_offsets(DIM, DH, a.dm.Gq, a.dm.lam, a.dm.eta, true, es).total * 4 <= 100 * 1024 ? 1 : 0;
-    const size_t bytes = (size_t)dec_offsets(DIM, DH, a.dm.Gq, a.dm.lam, a.dm.eta, a.r_smem != 0, es).total * 4;
+    const DecodeArgs& a = a0;
+    const size_t bytes = (size_t)dec_offsets(DIM, DH, a.dm.Gq, a.dm.lam, a.dm.eta, (int)sizeof(TIn)).total * 4;
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<DIM, DH, TIn>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
@@ -544,7 +545,7 @@ cudaError_t launch_residual_init(const DecodeArgs& a, cudaStream_t s) {
 }
 
 size_t decode_smem_bytes(const Dims& dm) {   // the smaller layout (residuals re-read from global)
-    return (size_t)dec_offsets(dm.d, dm.Dh, dm.Gq, dm.lam, dm.eta, false, dm.esize).total * 4;
+    return (size_t)dec_offsets(dm.d, dm.Dh, dm.Gq, dm.lam, dm.eta, dm.esize).total * 4;
 }
 
 }  // namespace lola

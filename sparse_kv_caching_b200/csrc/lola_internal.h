@@ -25,7 +25,7 @@ namespace lola {
 constexpr int kThreads = 512;
 
 struct Layout {            // byte offsets inside dev_buf (all 256-aligned)
-    size_t W, H, s, cache_k, cache_v, cache_phik, cache_pos, win_k, win_v, win_phik, cache_R, cache_den;
+    size_t W, H, s, cache_k, cache_v, cache_phik, cache_pos, win_k, win_v, win_phik, cache_R, cache_den, cache_sc;
     size_t phik_new, snap_pos, snap_H, snap_s, io_q, io_k, io_v, io_y, err;
     size_t total;
 };
@@ -49,6 +49,7 @@ struct StatePtrs {
     float* win_phik;
     float* cache_R;        // [S][lambda][d]  H^T phi_e - den_e v_e (kept by decode)
     float* cache_den;      // [S][lambda]     phi_e . s
+    float* cache_sc;       // [S][lambda]     SRE of each member against the current (H, s)
 };
 
 struct PrefillArgs {
@@ -78,7 +79,6 @@ struct DecodeArgs {
     float* y;              // [B][Hq][d]
     int t;                 // position of the new token
     int* err;              // device error word
-    int r_smem;            // set by the launcher: residual rows fit in shared memory
 };
 
 // Launchers (each returns cudaGetLastError() of its launch).
