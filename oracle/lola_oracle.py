@@ -33,19 +33,36 @@ reason, in the design notes of this repository):
       are per kv head and the selection is shared by the head group.
   R8  The output is Eq. 14 evaluated as written (no max-stabiliser: the fp64
       exponent stays far from overflow for these inputs; this is asserted).
+  R9  Read-branch masks (notes §4.8, App. I, Table 12): a hidden branch is
+      dropped from both the numerator and the shared denominator of Eq. 14;
+      the memories are updated exactly as without the mask.
+  R10 Update-first decode (the token equations of notes §2.4, Eqs. 11-14
+      taken literally): the new pair enters the window, the pair eta steps
+      back leaves it and is scored with the cache against the state, and
+      only then does the query read; it sees the eta most recent pairs,
+      itself included.  The memories evolve exactly as under R3.
+  R11 Stored-pair SRE map (notes §4.4, Fig. 3): at each state time (a block
+      boundary) every folded pair's SRE against that state; pairs not in the
+      state are 0.  Relative SRE (notes §4.4, Fig. 10, Eq. 26): that value
+      minus the pair's SRE at the first state time that held it.
 
 Parity status of every function here: pinned by the tests in
 tests/test_oracle_pins.py (closed forms, reductions to textbook softmax
 attention and to the window+linear hybrid, brute-force state, exhaustive
 pairwise check of the selection, identical-key closed form, partition
 invariant, decode == one-token blocks, split calls == one call, and the
-printed App. B / Table 10 memory counts).
+printed App. B / Table 10 memory counts).  The read masks, the update-first
+decode and the SRE map are pinned the same way (banded softmax, brute-force
+hybrids over the logged memories, the one-, two- and identical-pair closed
+forms of the map).
 """
 from __future__ import annotations
 
 import numpy as np
 
 TIE_REL = 1e-5   # relative band around the lambda-th SRE inside which swaps are valid
+HIDE_STATE = 1   # read mask bit: the queries do not read (H, s)            (R9)
+HIDE_SPARSE = 2  # read mask bit: the queries do not read the sparse cache G (R9)
 
 
 # ---------------------------------------------------------------------------
@@ -130,8 +147,9 @@ class LolaStream:
     index it; the memories themselves hold positions only.
     """
 
-    def __init__(self, W: np.ndarray, eta: int, lam: int):
+    def __init__(self, W: np.ndarray, eta: int, lam: int, read_mask: int = 0):
         self.W = np.asarray(W, np.float64)
+        self.read_mask = int(read_mask)
         self.d, self.Dh = self.W.shape
         self.D = 2 * self.Dh
         self.eta, self.lam = int(eta), int(lam)
@@ -176,14 +194,16 @@ class LolaStream:
         self.t += n
         return P
 
-    # -- read (Eq. 14 with the state entering the block; R3, R8) ----------
+    # -- read (Eq. 14 with the memories as they stand; R3, R8, R9) ---------
     def _read(self, Q: np.ndarray, P: list[int], rows: np.ndarray | None) -> np.ndarray:
+        """Eq. 14 for queries Q [Gq, n, d]; P = the block's own positions, read causally."""
         Gq, n, d = Q.shape
         y = np.full((Gq, n, d), np.nan)
-        exact = self.cache + self.window           # G and W entering the block
+        exact = ([] if self.read_mask & HIDE_SPARSE else self.cache) + self.window
+        read_state = not self.read_mask & HIDE_STATE
         Ke, Ve = self.K[exact], self.V[exact]
         Kb, Vb = self.K[P], self.V[P]
-        causal = np.tril(np.ones((n, n)))          # block key j visible to query i iff j <= i
+        causal = np.tril(np.ones((n, len(P))))     # block key j visible to query i iff j <= i
         scale = 1.0 / np.sqrt(d)
         for h in range(Gq):
             sel = np.arange(n) if rows is None else np.nonzero(rows[h])[0]
@@ -193,12 +213,15 @@ class LolaStream:
             le = (q @ Ke.T) * scale
             lb = (q @ Kb.T) * scale
             assert le.size == 0 or le.max() < 700.0
-            assert lb.max() < 700.0
+            assert lb.size == 0 or lb.max() < 700.0
             ae = np.exp(le)
             ab = np.exp(lb) * causal[sel]
-            phq = feature_map(q, self.W)
-            num = ae @ Ve + ab @ Vb + phq @ self.H
-            den = ae.sum(axis=1) + ab.sum(axis=1) + phq @ self.s
+            num = ae @ Ve + ab @ Vb
+            den = ae.sum(axis=1) + ab.sum(axis=1)
+            if read_state:
+                phq = feature_map(q, self.W)
+                num = num + phq @ self.H
+                den = den + phq @ self.s
             y[h, sel] = num / den[:, None]
         return y
 
@@ -216,6 +239,11 @@ class LolaStream:
             Q = Q[:, None, :]
         P = self._append(K, V)
         y = self._read(Q, P, rows)
+        self._update(P, choose)
+        return y
+
+    def _update(self, P: list[int], choose=None) -> None:
+        """Window advance, candidates, SRE, top-lambda and fold for the new positions P."""
         # advance the window: the block enters, the oldest pairs beyond eta leave (R2)
         self.window.extend(P)
         n_leave = max(0, len(self.window) - self.eta)
@@ -243,7 +271,6 @@ class LolaStream:
             self.cache = keep
             rec["fold"] = S
         self.log.append(rec)
-        return y
 
     def _fold(self, S: list[int]) -> None:
         """Eqs. 12-13: H += sum phi(k) v^T, s += sum phi(k) over the pairs S leaving E."""
@@ -262,6 +289,43 @@ class LolaStream:
             out.append(self.step(Q[:, c0:c0 + chunk], K[c0:c0 + chunk], V[c0:c0 + chunk], r, choose))
         return np.concatenate(out, axis=1)
 
-    def decode(self, q, k, v, choose=None) -> np.ndarray:
-        """Per-token decode step: one block of a single token (R3)."""
-        return self.step(np.asarray(q).reshape(-1, 1, self.d), k, v, None, choose)[:, 0]
+    def decode(self, q, k, v, choose=None, update_first: bool = False) -> np.ndarray:
+        """Per-token decode step: one block of a single token (R3), or update then read (R10)."""
+        Q = np.asarray(q, np.float64).reshape(-1, 1, self.d)
+        if not update_first:
+            return self.step(Q, k, v, None, choose)[:, 0]
+        P = self._append(k, v)
+        self._update(P, choose)
+        return self._read(Q, [], None)[:, 0]     # the new pair is now the newest window member
+
+
+# ---------------------------------------------------------------------------
+# Stored-pair SRE over time (notes §4.4: Fig. 3; Fig. 10 and Eq. 26; R11)
+# ---------------------------------------------------------------------------
+def sre_map(st: LolaStream, first_block: int = 0) -> tuple[np.ndarray, np.ndarray]:
+    """SRE of every folded pair at each state time, and its change since first write.
+
+    State time c (0 <= c <= n, n = logged blocks from `first_block` on) is the
+    state entering block first_block + c; c = n is the state after the last
+    block.  Returns (sre, rel), both [n + 1, t] fp64 over positions 0 .. t-1:
+      sre[c, i] = SRE(k_i, v_i | H_c, s_c) if pair i is folded at time c, else 0,
+      rel[c, i] = sre[c, i] - sre[c_i, i], c_i the first state time holding i.
+    H_c and s_c are summed again from their definition over the folded set
+    (Eqs. 12-13 accumulated), not taken from the running state.
+    """
+    recs = st.log[first_block:]
+    n_folded = [r["folded_before"] for r in recs] + [len(st.folded)]
+    sre = np.zeros((len(n_folded), st.t))
+    rel = np.zeros_like(sre)
+    first: dict[int, int] = {}
+    for c, nf in enumerate(n_folded):
+        F = st.folded[:nf]
+        if not F:
+            continue
+        H = st.phiK[F].T @ st.V[F]
+        s = st.phiK[F].sum(axis=0)
+        sre[c, F] = self_recall_error(st.phiK[F], st.V[F], H, s)
+        for i in F:
+            first.setdefault(i, c)
+            rel[c, i] = sre[c, i] - sre[first[i], i]
+    return sre, rel

@@ -220,3 +220,139 @@ def check_tie_order(top_fn) -> int:
              ([1, 2, 3, 4], [1.0, 3.0, 3.0, 0.0], 1, [2]),
              ([9, 4, 6, 2], [5.0, 1.0, 5.0, 1.0], 3, [2, 6, 9])]
     return sum(sorted(top_fn(E, np.array(s), lam)) != want for E, s, lam, want in cases)
+
+
+def _hybrid_ref(q, k, v, W, exact, F, read_state=True):
+    """Eq. 14 by brute force for one query: softmax terms over `exact`, linear terms over F."""
+    e = np.exp(k[exact] @ q / np.sqrt(len(q)))
+    num, den = e @ v[exact], e.sum()
+    if read_state and F:
+        kern = softmax_fm(k[F], W) @ softmax_fm(q[None], W)[0]     # phi(q)^T phi(k_i)
+        num, den = num + kern @ v[F], den + kern.sum()
+    return num / den
+
+
+# Read-branch masks, window only (notes §4.8, App. I): a banded causal softmax
+def check_mask_window_only(Stream) -> float:
+    w, a, W = small(T=48, eta=8, lam=6, C=4)
+    st = Stream(W, w.eta, w.lam)
+    st.read_mask = 3
+    y = st.prefill(a["q"], a["k"], a["v"], w.chunk)
+    q, k, v = (np.asarray(a[x], np.float64) for x in "qkv")
+    t = np.arange(w.T)
+    lo = np.maximum(0, (t // w.chunk) * w.chunk - w.eta)
+    allowed = (t[None, :] <= t[:, None]) & (t[None, :] >= lo[:, None])
+    sd = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k)[None].expand(q.shape[0], -1, -1),
+        torch.from_numpy(v)[None].expand(q.shape[0], -1, -1), attn_mask=torch.from_numpy(allowed)).numpy()
+    err = 0.0
+    for h in range(q.shape[0]):            # textbook loop beside the library routine
+        for tt in range(w.T):
+            l = k[lo[tt]:tt + 1] @ q[h, tt] / np.sqrt(w.d)
+            p = np.exp(l - l.max())
+            ref = (p / p.sum()) @ v[lo[tt]:tt + 1]
+            err = max(err, float(np.abs(ref - sd[h, tt]).max()), float(np.abs(ref - y[h, tt]).max()))
+    return err
+
+
+# Read-branch masks, one branch hidden: brute-force hybrids over the logged memories;
+# the memories themselves evolve exactly as in the unmasked run
+def check_mask_one_branch(Stream) -> float:
+    w, a, W = small(T=64, eta=8, lam=5, C=4)
+    q, k, v = (np.asarray(a[x], np.float64) for x in "qkv")
+    ref_st, _ = run(Stream, w, a, W)
+    err = 0.0
+    for mask in (1, 2):
+        st = Stream(W, w.eta, w.lam)
+        st.read_mask = mask
+        y = st.prefill(a["q"], a["k"], a["v"], w.chunk)
+        for rec in st.log:
+            t0 = rec["t0"]
+            G = [] if mask == 2 else rec["cache_before"]
+            F = st.folded[:rec["folded_before"]]
+            for h in range(q.shape[0]):
+                for t in range(t0, t0 + rec["n"]):
+                    ex = G + list(range(max(0, t0 - w.eta), t + 1))
+                    ref = _hybrid_ref(q[h, t], k, v, W, ex, F, read_state=(mask != 1))
+                    err = max(err, float(np.abs(ref - y[h, t]).max()))
+        if st.cache != ref_st.cache or st.folded != ref_st.folded:
+            return np.inf
+        err = max(err, float(np.abs(st.H - ref_st.H).max()), float(np.abs(st.s - ref_st.s).max()))
+    return err
+
+
+# Update-first decode (Eqs. 11-14 read literally): lambda = 0 gives a window of
+# the eta most recent pairs (self included) plus the linear state over all older
+# pairs; eta + lambda >= T gives causal softmax; the memories match read-first decode
+def check_update_first(Stream) -> float:
+    err = 0.0
+    for T, eta, lam in ((40, 6, 0), (24, 10, 16), (48, 8, 5)):
+        w, a, W = small(T=T, eta=eta, lam=lam, C=1)
+        q, k, v = (np.asarray(a[x], np.float64) for x in "qkv")
+        st = Stream(W, eta, lam)
+        rf = Stream(W, eta, lam)
+        for t in range(T):
+            y = st.decode(a["q"][:, t], a["k"][t], a["v"][t], update_first=True)
+            rf.decode(a["q"][:, t], a["k"][t], a["v"][t])
+            if st.cache != rf.cache or st.folded != rf.folded or st.window != rf.window:
+                return np.inf
+            err = max(err, float(np.abs(st.H - rf.H).max()))
+            lo = max(0, t - eta + 1)
+            if lam == 0:
+                for h in range(q.shape[0]):
+                    ref = _hybrid_ref(q[h, t], k, v, W, list(range(lo, t + 1)), list(range(lo)))
+                    err = max(err, float(np.abs(ref - y[h]).max()))
+            elif eta + lam >= T:
+                for h in range(q.shape[0]):
+                    l = k[:t + 1] @ q[h, t] / np.sqrt(w.d)
+                    p = np.exp(l - l.max())
+                    err = max(err, float(np.abs((p / p.sum()) @ v[:t + 1] - y[h]).max()))
+            else:                              # general case over the updated memories
+                for h in range(q.shape[0]):
+                    ref = _hybrid_ref(q[h, t], k, v, W, st.cache + list(range(lo, t + 1)), st.folded)
+                    err = max(err, float(np.abs(ref - y[h]).max()))
+    return err
+
+
+# Stored-pair SRE map (Fig. 3) and relative SRE (Eq. 26): closed forms
+def check_sre_map(Stream, map_fn) -> float:
+    err = 0.0
+    # one folded pair is recalled exactly; two folded pairs a, b:
+    # SRE_a = (k_ab / (k_aa + k_ab))^2 ||v_b - v_a||^2, k = phi^T phi
+    for C in (1, 2):
+        w, a, W = small(T=16, eta=4, lam=0, C=C)
+        st, _ = run(Stream, w, a, W)
+        sre, rel = map_fn(st)
+        n_folded = [r["folded_before"] for r in st.log] + [len(st.folded)]
+        c = n_folded.index(C)
+        v = np.asarray(a["v"], np.float64)
+        if C == 1:
+            err = max(err, abs(sre[c, 0]))
+        else:
+            pk = softmax_fm(a["k"][:2], W)
+            K = pk @ pk.T
+            for i, j in ((0, 1), (1, 0)):
+                want = (K[i, j] / (K[i, i] + K[i, j])) ** 2 * ((v[j] - v[i]) ** 2).sum()
+                err = max(err, abs(sre[c, i] - want) / want)
+        if np.any(sre[:c, :] != 0) or np.any(rel[c] != 0):
+            return np.inf
+    # identical keys: the state recalls the mean of the folded values
+    w, a, W = small(T=40, eta=4, lam=3, C=4)
+    a = dict(a, k=np.tile(a["k"][0], (w.T, 1)))
+    st, _ = run(Stream, w, a, W)
+    sre, rel = map_fn(st)
+    v = np.asarray(a["v"], np.float64)
+    bounds = [r["t0"] for r in st.log] + [w.T]
+    first = {}
+    for c, t in enumerate(bounds):
+        F = set(range(max(0, t - w.eta))) - set(st.log[c]["cache_before"] if c < len(st.log) else st.cache)
+        vbar = v[sorted(F)].mean(axis=0) if F else None
+        for i in range(w.T):
+            if i not in F:
+                if sre[c, i] != 0 or rel[c, i] != 0:
+                    return np.inf
+                continue
+            want = ((vbar - v[i]) ** 2).sum()
+            first.setdefault(i, want)
+            err = max(err, abs(sre[c, i] - want), abs(rel[c, i] - (want - first[i])))
+    return err

@@ -13,7 +13,7 @@ import pytest
 import torch
 
 import oracle.lola_oracle as lo
-from oracle import LolaStream, feature_map, self_recall_error, state_elements, full_elements
+from oracle import LolaStream, feature_map, self_recall_error, state_elements, full_elements, sre_map
 from tests import pins
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -57,6 +57,22 @@ def test_selection_exhaustive():
 
 def test_identical_keys_closed_form():
     assert pins.check_identical_keys(LolaStream) < 1e-12
+
+
+def test_mask_window_only_is_banded_softmax():
+    assert pins.check_mask_window_only(LolaStream) < 1e-12
+
+
+def test_mask_one_branch_hidden():
+    assert pins.check_mask_one_branch(LolaStream) < 1e-12
+
+
+def test_update_first_decode():
+    assert pins.check_update_first(LolaStream) < 1e-12
+
+
+def test_sre_map_closed_forms():
+    assert pins.check_sre_map(LolaStream, sre_map) < 1e-12
 
 
 def test_partition_invariant():
@@ -127,9 +143,13 @@ def test_golden_memory_count(row):
 # ---------------------------------------------------------------------------
 # Planted mistakes: each broken oracle must fail at least one pin.
 # ---------------------------------------------------------------------------
-def _all_pins_pass(Stream, sre_fn=None):
+def _all_pins_pass(Stream, sre_fn=None, map_fn=None):
     ok = True
     try:
+        ok &= pins.check_mask_window_only(Stream) < 1e-9
+        ok &= pins.check_mask_one_branch(Stream) < 1e-9
+        ok &= pins.check_update_first(Stream) < 1e-9
+        ok &= pins.check_sre_map(Stream, map_fn or lo.sre_map) < 1e-9
         ok &= pins.check_sre_closed_form(sre_fn or lo.self_recall_error) < 1e-9
         ok &= pins.check_full_softmax(Stream) < 1e-9
         ok &= pins.check_lambda0(Stream) < 1e-9
@@ -210,6 +230,47 @@ class _NoLinearRead(LolaStream):
             self.H, self.s = H, s
 
 
+class _MaskIgnored(LolaStream):
+    def _read(self, Q, P, rows):
+        m = self.read_mask
+        self.read_mask = 0
+        try:
+            return super()._read(Q, P, rows)
+        finally:
+            self.read_mask = m
+
+
+class _MaskHidesBothSums(LolaStream):         # hidden state dropped from the numerator only
+    def _read(self, Q, P, rows):
+        if not self.read_mask & lo.HIDE_STATE:
+            return super()._read(Q, P, rows)
+        H = self.H
+        self.H = np.zeros_like(H)
+        self.read_mask &= ~lo.HIDE_STATE
+        try:
+            return super()._read(Q, P, rows)
+        finally:
+            self.H = H
+            self.read_mask |= lo.HIDE_STATE
+
+
+class _UpdateFirstReadsEarly(LolaStream):
+    def decode(self, q, k, v, choose=None, update_first=False):
+        return super().decode(q, k, v, choose, False)
+
+
+def _map_state_off_by_one(st, first_block=0):
+    sre, rel = lo.sre_map(st, first_block)
+    return np.vstack([np.zeros((1, sre.shape[1])), sre[:-1]]), np.vstack([np.zeros((1, rel.shape[1])), rel[:-1]])
+
+
+def _map_rel_from_previous(st, first_block=0):
+    sre, _ = lo.sre_map(st, first_block)
+    rel = np.zeros_like(sre)
+    rel[1:] = np.where(sre[1:] != 0, sre[1:] - sre[:-1], 0)
+    return sre, rel
+
+
 class _WindowOffByOne(LolaStream):
     def __init__(self, W, eta, lam):
         super().__init__(W, eta + 1, lam)
@@ -217,10 +278,13 @@ class _WindowOffByOne(LolaStream):
 
 @pytest.mark.parametrize("name", ["sre_no_division", "sre_wrong_sign", "sre_transposed",
                                   "keep_lowest", "tie_rule", "feature_same_half", "no_s_update",
-                                  "fold_transposed", "no_linear_read", "window_off_by_one"])
+                                  "fold_transposed", "no_linear_read", "window_off_by_one",
+                                  "mask_ignored", "mask_numerator_only", "update_first_reads_early",
+                                  "map_state_off_by_one", "map_rel_from_previous"])
 def test_planted_mistakes_are_caught(monkeypatch, name):
     Stream = LolaStream
     sre_fn = None
+    map_fn = None
     if name == "sre_no_division":
         monkeypatch.setattr(lo, "self_recall_error", _sre_no_division); sre_fn = _sre_no_division
     elif name == "sre_wrong_sign":
@@ -242,4 +306,14 @@ def test_planted_mistakes_are_caught(monkeypatch, name):
         Stream = _NoLinearRead
     elif name == "window_off_by_one":
         Stream = _WindowOffByOne
-    assert not _all_pins_pass(Stream, sre_fn)
+    elif name == "mask_ignored":
+        Stream = _MaskIgnored
+    elif name == "mask_numerator_only":
+        Stream = _MaskHidesBothSums
+    elif name == "update_first_reads_early":
+        Stream = _UpdateFirstReadsEarly
+    elif name == "map_state_off_by_one":
+        map_fn = _map_state_off_by_one
+    elif name == "map_rel_from_previous":
+        map_fn = _map_rel_from_previous
+    assert not _all_pins_pass(Stream, sre_fn, map_fn)
