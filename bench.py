@@ -76,6 +76,18 @@ def prefill_work(w: synth.Workload) -> dict:
     }
 
 
+def sre_map_work(w: synth.Workload) -> tuple[int, int]:
+    """(pairs, FLOPs) of one SRE-map launch after a prefill of w.T tokens from position 0:
+    every folded pair at every state time costs H^T phi (2 D d), phi . s (2 D) and the
+    residual's divide, subtract and square-add (3 d)."""
+    pairs = 0
+    for c in range(w.T // w.chunk + 1):
+        left = max(0, c * w.chunk - w.eta)
+        pairs += left - min(w.lam, left)
+    pairs *= w.B * w.Hkv
+    return pairs, pairs * (2 * w.D * w.d + 2 * w.D + 3 * w.d)
+
+
 def decode_step_bytes(w: synth.Workload) -> int:
     """HBM bytes one decode step must move (all streams, steady state)."""
     e = 2 if w.dtype == "bf16" else 4
@@ -131,7 +143,7 @@ def load_peaks():
 
 # Sources a kernel class's counters depend on: its own files plus the shared headers.
 KERNEL_SOURCES = {"phi": ["phi.cu"], "scan": ["scan.cu"], "output": ["output_tc.cu", "output.cu"],
-                  "finalize": ["finalize.cu"], "decode": ["decode.cu"]}
+                  "finalize": ["finalize.cu"], "decode": ["decode.cu"], "sre_map": ["sre_map.cu"]}
 SHARED_SOURCES = ["device_common.cuh", "lola_internal.h", "umma.cuh"]
 
 
@@ -471,6 +483,8 @@ def main():
     work = prefill_work(w)
     # dominant kernel by measured time
     dom = max(("phi", "scan", "output"), key=lambda kk: prof[kk][0])
+    alu = fp32_alu_peak_tflops(props.multi_processor_count)
+    alu_kind = f"derived fp32 FMA: {props.multi_processor_count} SMs x 128 lanes x 2 FLOP x {SM_MAX_MHZ} MHz"
     # per step: a call may launch a kernel class several times (the chain runs in
     # chunk segments), so work and time are both summed over the step's launches
     dom_ms = prof[dom][0] / args.steps
@@ -480,11 +494,8 @@ def main():
     peak = peaks["bf16_tflops"]
     if dom == "scan":
         # the memory-update chain runs fp32 FMAs on the CUDA cores, not the tensor cores
-        alu = fp32_alu_peak_tflops(props.multi_processor_count)
         roofline = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": alu, "unit": "TFLOP/s",
-                    "frac": achieved / alu,
-                    "peak_kind": f"derived fp32 FMA: {props.multi_processor_count} SMs x 128 lanes x 2 FLOP x "
-                                 f"{SM_MAX_MHZ} MHz",
+                    "frac": achieved / alu, "peak_kind": alu_kind,
                     "traffic": traffic_for(dom, w.name), "flops_per_step": fl, "kernel_ms_per_step": dom_ms,
                     "launches_per_step": dom_launches}
     else:
@@ -492,7 +503,8 @@ def main():
                     "frac": achieved / peak, "peak_kind": f"{peaks_kind} bf16 dense (burst)",
                     "traffic": traffic_for(dom, w.name),
                     "flops_per_step": fl, "kernel_ms_per_step": dom_ms, "launches_per_step": dom_launches}
-    shares = {kk: round(prof[kk][0] / max(1e-9, sum(p[0] for p in prof.values())), 4) for kk in prof}
+    shares = {kk: round(prof[kk][0] / max(1e-9, sum(p[0] for p in prof.values())), 4)
+              for kk in ("phi", "scan", "output", "finalize", "decode")}
     layer_roof_ms = max(work["total_flops"] / (peak * 1e12), 0.0) * 1e3
     # ---- e2e through the host-buffer entry point ------------------------------
     hq, hk, hv = (torch.from_numpy(full[x].view(np.int16) if full[x].dtype == np.uint16 else full[x])
@@ -522,6 +534,24 @@ def main():
     layer.reset()
     layer.prefill(q, k, v, y)
     torch.cuda.synchronize()
+    # ---- stored-pair SRE map of that prefill (analysis kernel, timed alone) ----
+    sre_buf, rel_buf = layer.sre_map(k, v)
+    for _ in range(2):
+        layer.sre_map(k, v, sre_buf, rel_buf)
+    layer.profile(True)
+    for _ in range(5):
+        flush.zero_()
+        layer.sre_map(k, v, sre_buf, rel_buf)
+    pm = layer.profile_read()["sre_map"]
+    layer.profile(False)
+    map_ms = pm[0] / max(1, pm[1])
+    map_pairs, map_fl = sre_map_work(w)
+    sre_map_line = {"workload": w.name, "ms_per_launch": map_ms, "pairs_per_launch": map_pairs,
+                    "roofline": {"bound": "alu", "kernel": "sre_map", "achieved": map_fl / (map_ms / 1e3) / 1e12,
+                                 "peak": alu, "unit": "TFLOP/s",
+                                 "frac": map_fl / (map_ms / 1e3) / 1e12 / alu, "peak_kind": alu_kind,
+                                 "flops_per_launch": map_fl, "traffic": traffic_for("sre_map", w.name)}}
+    del sre_buf, rel_buf
     ex = layer.export()
     trace = ex["trace_pos"].cpu().numpy() if w.lam > 0 else None
     y_host = y.cpu()
@@ -541,6 +571,7 @@ def main():
             "clocks": clk,
             "e2e": {"value": job_throughput(w.B * w.T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "sre_map": sre_map_line,
             }
     del layer, full, q, k, v, y, hq, hk, hv, hy
     torch.cuda.empty_cache()

@@ -159,16 +159,57 @@ int lola_prefill_chunked_host(lola_state* st, const void* q, const void* k, cons
 int lola_decode_step_host(lola_state* st, const void* q, const void* k, const void* v,
                           float* y, void* stream);
 
+/* Read options.  read_mask hides memory branches from every later read (the
+ * module-read ablation of notes §4.8, App. I, Table 12):
+ * LOLA_READ_HIDE_STATE drops phi(q)^T H and phi(q)^T s from the numerator
+ * and the shared denominator of Eq. 14, LOLA_READ_HIDE_SPARSE drops the
+ * cache members' softmax terms; with both, the queries read the window and
+ * their block's own causal keys only.  The memories are updated exactly as
+ * without a mask.  decode_update_first = 1 makes lola_decode_step take the
+ * token equations (notes §2.4, Eqs. 11-14) literally: the new pair enters the
+ * window, the pair eta steps back leaves it and is scored with the cache
+ * against the state (the lowest SRE is folded), and only then does the
+ * query read: the updated cache and state, and the eta most recent pairs,
+ * itself included.  The memories evolve identically under both orders; only
+ * y differs.  Prefill always reads first (the queries of a block share the
+ * state entering it, notes §2.6).  The options persist across
+ * lola_state_reset; 0, 0 restores the default.  LOLA_ERR_INVALID_ARG for
+ * other bits or values. */
+#define LOLA_READ_HIDE_STATE  1
+#define LOLA_READ_HIDE_SPARSE 2
+int lola_set_read_options(lola_state* st, int read_mask, int decode_update_first);
+
+/* Stored-pair SRE map of the last prefill call (notes §4.4: Fig. 3, and
+ * Fig. 10 / Eq. 26 for the relative form).  With n = the chunks of that call
+ * (trace_len - 1 of lola_state_export) and t_c = its first position + c *
+ * chunk, state time c in [0, n] is the state entering chunk c (c = n: the
+ * state after the call).  For every position i < T:
+ *   sre[b][g][c][i] = || H_c^T phi(k_i) / (phi(k_i)^T s_c) - v_i ||^2 when
+ *                     pair i is folded into the state at time c (it has left
+ *                     the window, i < t_c - eta, and is not cached), else 0;
+ *   rel[b][g][c][i] = sre[b][g][c][i] - sre[b][g][c_i][i], c_i the first state
+ *                     time of the map at which pair i is folded (0 where not
+ *                     folded).
+ * k, v: device [B][T][Hkv][d] in dtype, every position of the sequences from
+ * 0 (the same values the calls received); T must equal the tokens processed.
+ * sre, rel: device float32 [B][Hkv][n + 1][T]; rel may be NULL.  The last
+ * call on `st` must be a prefill (LOLA_ERR_INVALID_ARG after a decode step,
+ * a reset or no prefill).  For a host-buffer prefill of >= 8 chunks "the
+ * last call" is the last of its four chunk-aligned calls.  Reads the state's
+ * per-chunk snapshots and changes nothing; fp32 arithmetic. */
+int lola_sre_map(lola_state* st, const void* k, const void* v, int T, float* sre, float* rel,
+                 void* stream);
+
 /* Fill *out with device views of the state (no copy, no synchronisation). */
 int lola_state_export(const lola_state* st, lola_state_view* out);
 
 /* Tracing aid.  Kernel classes, in this order: 0 feature map, 1 scan (memory
- * update chain), 2 output, 3 finalize, 4 decode.  While enabled, every kernel
+ * update chain), 2 output, 3 finalize, 4 decode, 5 SRE map.  While enabled, every kernel
  * launch of `st` is bracketed by CUDA events recorded on its stream.
  * lola_profile_read waits for those events, adds their elapsed times (ms) and
- * launch counts into ms[0..4] and launches[0..4] (n >= 5 entries each) and
+ * launch counts into ms[0..5] and launches[0..5] (n >= 6 entries each) and
  * forgets them.  Enabling does not change what the kernels compute. */
-#define LOLA_KERNEL_CLASSES 5
+#define LOLA_KERNEL_CLASSES 6
 int lola_profile_enable(lola_state* st, int on);
 int lola_profile_read(lola_state* st, float* ms, long long* launches, int n);
 

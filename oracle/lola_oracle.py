@@ -14,7 +14,7 @@ top-lambda retention, fold), §2.5 (Eq. 14, shared normaliser), §2.6 (Eq. 15,
 Fig. 2, chunkwise inference) and §2.7 (App. B memory count).
 
 Readings taken where the pages leave a step open (each is listed, with its
-reason, in the design notes of this repository):
+reason and under the same number, in the design notes of this repository):
   R1  SRE is the squared L2 residual (the summaries' form); the ranking equals
       that of the unsquared norm of §2.3.
   R2  eta counts the exact pairs that precede the current block; the block's
@@ -33,15 +33,15 @@ reason, in the design notes of this repository):
       are per kv head and the selection is shared by the head group.
   R8  The output is Eq. 14 evaluated as written (no max-stabiliser: the fp64
       exponent stays far from overflow for these inputs; this is asserted).
-  R9  Read-branch masks (notes §4.8, App. I, Table 12): a hidden branch is
+  R15 Read-branch masks (notes §4.8, App. I, Table 12): a hidden branch is
       dropped from both the numerator and the shared denominator of Eq. 14;
       the memories are updated exactly as without the mask.
-  R10 Update-first decode (the token equations of notes §2.4, Eqs. 11-14
+  R16 Update-first decode (the token equations of notes §2.4, Eqs. 11-14
       taken literally): the new pair enters the window, the pair eta steps
       back leaves it and is scored with the cache against the state, and
       only then does the query read; it sees the eta most recent pairs,
       itself included.  The memories evolve exactly as under R3.
-  R11 Stored-pair SRE map (notes §4.4, Fig. 3): at each state time (a block
+  R17 Stored-pair SRE map (notes §4.4, Fig. 3): at each state time (a block
       boundary) every folded pair's SRE against that state; pairs not in the
       state are 0.  Relative SRE (notes §4.4, Fig. 10, Eq. 26): that value
       minus the pair's SRE at the first state time that held it.
@@ -61,8 +61,8 @@ from __future__ import annotations
 import numpy as np
 
 TIE_REL = 1e-5   # relative band around the lambda-th SRE inside which swaps are valid
-HIDE_STATE = 1   # read mask bit: the queries do not read (H, s)            (R9)
-HIDE_SPARSE = 2  # read mask bit: the queries do not read the sparse cache G (R9)
+HIDE_STATE = 1   # read mask bit: the queries do not read (H, s)            (R15)
+HIDE_SPARSE = 2  # read mask bit: the queries do not read the sparse cache G (R15)
 
 
 # ---------------------------------------------------------------------------
@@ -194,7 +194,7 @@ class LolaStream:
         self.t += n
         return P
 
-    # -- read (Eq. 14 with the memories as they stand; R3, R8, R9) ---------
+    # -- read (Eq. 14 with the memories as they stand; R3, R8, R15) --------
     def _read(self, Q: np.ndarray, P: list[int], rows: np.ndarray | None) -> np.ndarray:
         """Eq. 14 for queries Q [Gq, n, d]; P = the block's own positions, read causally."""
         Gq, n, d = Q.shape
@@ -290,7 +290,7 @@ class LolaStream:
         return np.concatenate(out, axis=1)
 
     def decode(self, q, k, v, choose=None, update_first: bool = False) -> np.ndarray:
-        """Per-token decode step: one block of a single token (R3), or update then read (R10)."""
+        """Per-token decode step: one block of a single token (R3), or update then read (R16)."""
         Q = np.asarray(q, np.float64).reshape(-1, 1, self.d)
         if not update_first:
             return self.step(Q, k, v, None, choose)[:, 0]
@@ -300,7 +300,7 @@ class LolaStream:
 
 
 # ---------------------------------------------------------------------------
-# Stored-pair SRE over time (notes §4.4: Fig. 3; Fig. 10 and Eq. 26; R11)
+# Stored-pair SRE over time (notes §4.4: Fig. 3; Fig. 10 and Eq. 26; R17)
 # ---------------------------------------------------------------------------
 def sre_map(st: LolaStream, first_block: int = 0) -> tuple[np.ndarray, np.ndarray]:
     """SRE of every folded pair at each state time, and its change since first write.

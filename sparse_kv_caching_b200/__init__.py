@@ -26,8 +26,9 @@ EXPORTS = ("lola_state_bytes", "lola_state_init", "lola_state_reset", "lola_stat
            "lola_prefill_chunked", "lola_decode_step", "lola_prefill_chunked_host",
            "lola_decode_step_host", "lola_state_export", "lola_profile_enable",
            "lola_profile_read", "lola_launch_count", "lola_prefill_once_noalloc", "lola_selftest_umma",
-           "lola_last_error_string")
-KERNEL_CLASSES = ("phi", "scan", "output", "finalize", "decode")
+           "lola_set_read_options", "lola_sre_map", "lola_last_error_string")
+KERNEL_CLASSES = ("phi", "scan", "output", "finalize", "decode", "sre_map")
+READ_HIDE_STATE, READ_HIDE_SPARSE = 1, 2
 
 
 class LolaConfig(ctypes.Structure):
@@ -73,6 +74,8 @@ def lib() -> ctypes.CDLL:
     L.lola_profile_read.argtypes = [vp, POINTER(ctypes.c_float), POINTER(c_longlong), c_int]
     L.lola_prefill_once_noalloc.argtypes = [POINTER(LolaConfig), vp, vp, vp, vp, c_int, vp, vp]
     L.lola_selftest_umma.argtypes = [c_int, vp, vp, vp, c_int, c_int, c_int, vp, vp]
+    L.lola_set_read_options.argtypes = [vp, c_int, c_int]
+    L.lola_sre_map.argtypes = [vp, vp, vp, c_int, vp, vp, vp]
     L.lola_launch_count.argtypes = []
     L.lola_launch_count.restype = c_longlong
     L.lola_last_error_string.argtypes = []
@@ -226,6 +229,31 @@ class LolaLayer:
         _check(lib().lola_decode_step_host(self.handle, c_void_p(q.data_ptr()), c_void_p(k.data_ptr()),
                                            c_void_p(v.data_ptr()), c_void_p(y.data_ptr()), _stream(stream)))
         return y
+
+    def set_read_options(self, read_mask: int = 0, decode_update_first: bool = False) -> None:
+        """Hide memory branches from later reads (READ_HIDE_* bits); update-first decode order."""
+        _check(lib().lola_set_read_options(self.handle, int(read_mask), 1 if decode_update_first else 0))
+
+    def sre_map(self, k, v, sre=None, rel=None, stream=None):
+        """SRE of every folded pair at each state time of the last prefill call, and its change
+        since first write: k/v [B,T,Hkv,d] (every position so far) -> sre, rel [B,Hkv,n+1,T] f32."""
+        c = self.cfg
+        T = k.shape[1]
+        _, sk = self._shapes(T)
+        self._check_tensor(k, sk, self.dtype, "k")
+        self._check_tensor(v, sk, self.dtype, "v")
+        v_ = LolaStateView()
+        _check(lib().lola_state_export(self.handle, byref(v_)))
+        shape = (c.B, c.Hkv, max(v_.trace_len, 1), T)
+        if sre is None:
+            sre = torch.empty(shape, dtype=torch.float32, device=self.device)
+        if rel is None:
+            rel = torch.empty(shape, dtype=torch.float32, device=self.device)
+        self._check_tensor(sre, shape, torch.float32, "sre")
+        self._check_tensor(rel, shape, torch.float32, "rel")
+        _check(lib().lola_sre_map(self.handle, c_void_p(k.data_ptr()), c_void_p(v.data_ptr()), T,
+                                  c_void_p(sre.data_ptr()), c_void_p(rel.data_ptr()), _stream(stream)))
+        return sre, rel
 
     def profile(self, on: bool = True) -> None:
         """Bracket every kernel launch of this layer with CUDA events (tracing aid)."""

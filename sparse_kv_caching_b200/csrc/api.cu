@@ -36,6 +36,8 @@ struct lola_state {
     long long last_t0;
     bool prof = false;
     bool resid_ok = true;     // per-slot decode residuals match (H, s)
+    int read_mask = 0;        // LOLA_READ_HIDE_* bits applied to every read
+    int update_first = 0;     // decode: update the memories before the read
     std::vector<lola_prof_mark> marks;
     std::vector<cudaEvent_t> pool;
     // Prefill overlap: the chain runs on a high-priority stream in chunk segments,
@@ -270,6 +272,46 @@ int lola_state_free(lola_state* st) {
     return LOLA_OK;
 }
 
+int lola_sre_map(lola_state* st, const void* k, const void* v, int T, float* sre, float* rel, void* stream) {
+    if (!st || !k || !v || !sre) return fail(LOLA_ERR_INVALID_ARG, "null argument");
+    if (misaligned(k) || misaligned(v) || misaligned(sre) || (rel && misaligned(rel)))
+        return fail(LOLA_ERR_INVALID_ARG, "k, v, sre and rel must be 16-byte aligned");
+    const lola::Dims& dm = st->dm;
+    if (st->last_nc < 0) return fail(LOLA_ERR_INVALID_ARG, "no prefill call since the state was initialised or reset");
+    if (st->t != st->last_t0 + (long long)st->last_nc * dm.C)
+        return fail(LOLA_ERR_INVALID_ARG, "decode steps followed the last prefill call; its snapshots no longer "
+                    "describe the state");
+    if ((long long)T != st->t)
+        return fail(LOLA_ERR_INVALID_ARG, "T=%d must equal the tokens processed (%lld)", T, st->t);
+    lola::SreMapArgs a{};
+    a.dm = dm;
+    a.k = k; a.v = v;
+    a.W = st->base + st->L.W;
+    a.snap_H = (const float*)(st->base + st->L.snap_H);
+    a.snap_s = (const float*)(st->base + st->L.snap_s);
+    a.snap_pos = (const int*)(st->base + st->L.snap_pos);
+    a.sre = sre; a.rel = rel;
+    a.T = T;
+    a.t0 = (int)st->last_t0;
+    a.nc = st->last_nc;
+    cudaStream_t s = (cudaStream_t)stream;
+    const cudaError_t e = traced(st, 5, 1, s, [&] { return lola::launch_sre_map(a, s); });
+    if (e != cudaSuccess) return cuda_fail(e, "SRE map kernel");
+    return LOLA_OK;
+}
+
+int lola_set_read_options(lola_state* st, int read_mask, int decode_update_first) {
+    if (!st) return fail(LOLA_ERR_INVALID_ARG, "null state");
+    if (read_mask & ~(LOLA_READ_HIDE_STATE | LOLA_READ_HIDE_SPARSE))
+        return fail(LOLA_ERR_INVALID_ARG, "read_mask=%d has bits other than LOLA_READ_HIDE_STATE | LOLA_READ_HIDE_SPARSE",
+                    read_mask);
+    if (decode_update_first != 0 && decode_update_first != 1)
+        return fail(LOLA_ERR_INVALID_ARG, "decode_update_first=%d must be 0 or 1", decode_update_first);
+    st->read_mask = read_mask;
+    st->update_first = decode_update_first;
+    return LOLA_OK;
+}
+
 int lola_profile_enable(lola_state* st, int on) {
     if (!st) return fail(LOLA_ERR_INVALID_ARG, "null state");
     st->prof = on != 0;
@@ -331,6 +373,7 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
     a.nc = T / dm.C;
     a.c_begin = 0;
     a.c_end = a.nc;
+    a.read_mask = st->read_mask;
     a.phik_new = (float*)(st->base + st->L.phik_new);
     a.snap_pos = (int*)(st->base + st->L.snap_pos);
     a.snap_H = (float*)(st->base + st->L.snap_H);
@@ -404,6 +447,8 @@ int lola_decode_step(lola_state* st, const void* q, const void* k, const void* v
     a.sp = state_ptrs(st);
     a.q = q; a.k = k; a.v = v; a.y = y;
     a.t = (int)st->t;
+    a.read_mask = st->read_mask;
+    a.update_first = st->update_first;
     a.err = (int*)(st->base + st->L.err);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;

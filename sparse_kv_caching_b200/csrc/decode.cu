@@ -132,24 +132,34 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     const TIn* vg = (const TIn*)a.v + ((size_t)b * dm.Hkv + g) * DIM;
     for (int i = tid; i < DIM; i += NT) { kn[i] = to_f32(kg[i]); vn[i] = to_f32(vg[i]); }
     const int n_g = min(lam, max(0, t - eta));
-    const int w_lo = max(0, t - eta);
-    const int n_w = t - w_lo;
-    const int NK = n_g + n_w + 1;
     const size_t cbase = (size_t)st * lam, wbase = (size_t)st * eta;
-    // key row pointers: cache slots, window (ring slot p % eta), then the token itself
-    for (int i = tid; i < NK; i += NT) {
-        const TIn* p;
-        if (i < n_g) p = (const TIn*)a.sp.cache_k + (cbase + i) * DIM;
-        else if (i < n_g + n_w) p = (const TIn*)a.sp.win_k + (wbase + (size_t)((w_lo + i - n_g) % eta)) * DIM;
-        else p = kg;
-        kp[2 * i] = p;
-        // the value row sits at the same offset of the matching value array
-        const TIn* pv;
-        if (i < n_g) pv = (const TIn*)a.sp.cache_v + (cbase + i) * DIM;
-        else if (i < n_g + n_w) pv = (const TIn*)a.sp.win_v + (wbase + (size_t)((w_lo + i - n_g) % eta)) * DIM;
-        else pv = vg;
-        kp[2 * i + 1] = pv;
-    }
+    const bool hide_state = (a.read_mask & 1) != 0, hide_sparse = (a.read_mask & 2) != 0;
+    // key row pointers of the read: cache slots [0, rg), window positions [rlo, t)
+    // (ring slot p % eta), then the token itself; returns the key count
+    auto fill_kp = [&](int rg, int rlo) -> int {
+        const int rw = t - rlo, nk = rg + rw + 1;
+        for (int i = tid; i < nk; i += NT) {
+            const TIn* p;
+            const TIn* pv;        // the value row sits at the same offset of the matching value array
+            if (i < rg) {
+                p = (const TIn*)a.sp.cache_k + (cbase + i) * DIM;
+                pv = (const TIn*)a.sp.cache_v + (cbase + i) * DIM;
+            } else if (i < rg + rw) {
+                const size_t ws = wbase + (size_t)((rlo + i - rg) % eta);
+                p = (const TIn*)a.sp.win_k + ws * DIM;
+                pv = (const TIn*)a.sp.win_v + ws * DIM;
+            } else {
+                p = kg;
+                pv = vg;
+            }
+            kp[2 * i] = p;
+            kp[2 * i + 1] = pv;
+        }
+        return nk;
+    };
+    // read first: the memories entering the step (the window holds [t - eta, t));
+    // update first reads after the update (see the end of the kernel)
+    const int NK = a.update_first ? 0 : fill_kp(hide_sparse ? 0 : n_g, max(0, t - eta));
     umma::cp_async_wait<0>();
     __syncthreads();
 
@@ -191,7 +201,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     __syncthreads();
 
     // ---- read: scores (a quad per key), softmax per head, P V (lane owns columns) ----
-    {
+    // Eq. 14 over the NK keys of kp and, unless hidden, the state (H, s) in shared memory
+    auto read_phase = [&](const int NK) {
         constexpr int KQ = DIM / 4;                                  // key elements per quad lane
         const int q4 = lane & 3, rq = lane >> 2;                     // lane in quad, quad in warp
         const float scale = 1.0f / sqrtf((float)DIM);
@@ -221,7 +232,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
             for (int i = lane; i < NK; i += 32) { const float e = expf(sc[hh * NK + i] - mx); sc[hh * NK + i] = e; sum += e; }
             sum = warp_sum(sum);
             float dl = 0.f;
-            for (int j = lane; j < D; j += 32) dl = fmaf(phq[hh * D + j], ss[j], dl);
+            if (!hide_state)
+                for (int j = lane; j < D; j += 32) dl = fmaf(phq[hh * D + j], ss[j], dl);
             dl = warp_sum(dl);
             if (lane == 0) { red[hh] = mx; red[8 + hh] = sum; red[16 + hh] = dl; }
         }
@@ -267,180 +279,196 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
             float A = 0.f;
             for (int w = 0; w < NW; ++w) A += part[(w * Gq + hh) * DIM + cc];
             float L = 0.f;
-            for (int j = 0; j < D; ++j) L = fmaf(phq[hh * D + j], Hs[j * DIM + cc], L);
+            if (!hide_state)
+                for (int j = 0; j < D; ++j) L = fmaf(phq[hh * D + j], Hs[j * DIM + cc], L);
             const float em = expf(-red[hh]);
             a.y[((size_t)b * dm.Hq + (size_t)g * Gq + hh) * DIM + cc] = (A + em * L) / (red[8 + hh] + em * red[16 + hh]);
         }
         __syncthreads();
-    }
+    };
 
-    // ---- update ----
-    if (leaving) {
-        const size_t wsl = wbase + rs;
-        const TIn* vl = (const TIn*)a.sp.win_v + wsl * DIM;
-        // P_l = H^T phi_l, den_l = phi_l . s, R_l = P_l - den_l v_l (pre-fold state)
-        for (int cc = tid; cc < DIM; cc += NT) {
-            float x = 0.f;
-            for (int j = 0; j < D; ++j) x = fmaf(phl[j], Hs[j * DIM + cc], x);
-            Pl[cc] = x;
-        }
-        if (warp == 0) {
-            float x = 0.f;
-            for (int j = lane; j < D; j += 32) x = fmaf(phl[j], ss[j], x);
-            x = warp_sum(x);
-            if (lane == 0) red[32] = x;
-        }
-        __syncthreads();
-        const float den_l = red[32];
-        float* Rg = a.sp.cache_R + cbase * DIM;
-        float* deng = a.sp.cache_den + cbase;
-        if (n_g < lam) {
-            // l joins the next free slot (fewer than lambda candidates: keep all)
-            const size_t cs = cbase + n_g;
-            for (int i = tid; i < DIM; i += NT) {
-                ((TIn*)a.sp.cache_k)[cs * DIM + i] = ((const TIn*)a.sp.win_k)[wsl * DIM + i];
-                ((TIn*)a.sp.cache_v)[cs * DIM + i] = vl[i];
-                Rg[(size_t)n_g * DIM + i] = Pl[i] - den_l * to_f32(vl[i]);
+    // ---- update (Eqs. 11-13 with one leaving pair l = t - eta) ----
+    auto update_phase = [&]() {
+        if (leaving) {
+            const size_t wsl = wbase + rs;
+            const TIn* vl = (const TIn*)a.sp.win_v + wsl * DIM;
+            // P_l = H^T phi_l, den_l = phi_l . s, R_l = P_l - den_l v_l (pre-fold state)
+            for (int cc = tid; cc < DIM; cc += NT) {
+                float x = 0.f;
+                for (int j = 0; j < D; ++j) x = fmaf(phl[j], Hs[j * DIM + cc], x);
+                Pl[cc] = x;
             }
-            for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
-            if (tid == 0) { a.sp.cache_pos[cs] = lpos; deng[n_g] = den_l; }
-            if (warp == 0) {                                          // its SRE against the state
-                float q = 0.f, vq = 0.f;
-                for (int cc = lane; cc < DIM; cc += 32) {
-                    const float v = to_f32(vl[cc]);
-                    const float r = Pl[cc] - den_l * v;
-                    q = fmaf(r, r, q);
-                    vq = fmaf(v, v, vq);
-                }
-                q = warp_sum(q);
-                vq = warp_sum(vq);
-                if (lane == 0) a.sp.cache_sc[cs] = den_l > 0.f ? q / (den_l * den_l) : vq;
-            }
-        } else {
-            // scores: members from the cache (stored when their residuals last changed), l from R_l
-            float* scs = red + 64;                                    // reuse as scratch for the argmin
-            for (int e = tid; e < lam; e += NT) sc[e] = a.sp.cache_sc[cbase + e];
             if (warp == 0) {
-                float q = 0.f, vq = 0.f;
-                for (int cc = lane; cc < DIM; cc += 32) {
-                    const float v = to_f32(vl[cc]);
-                    const float r = Pl[cc] - den_l * v;
-                    q = fmaf(r, r, q);
-                    vq = fmaf(v, v, vq);
-                }
-                q = warp_sum(q);
-                vq = warp_sum(vq);
-                if (lane == 0) sc[lam] = den_l > 0.f ? q / (den_l * den_l) : vq;
+                float x = 0.f;
+                for (int j = lane; j < D; j += 32) x = fmaf(phl[j], ss[j], x);
+                x = warp_sum(x);
+                if (lane == 0) red[32] = x;
             }
             __syncthreads();
-            // the folded pair: lowest SRE, the newer position on exact ties (keys are unique)
-            auto cand_key = [&](int e) -> unsigned long long {
-                const int p = e < lam ? a.sp.cache_pos[cbase + e] : lpos;
-                return ((unsigned long long)__float_as_uint(sc[e]) << 32) | (unsigned long long)(~(unsigned)p);
-            };
-            unsigned long long best = ~0ull;
-            for (int e = tid; e <= lam; e += NT) { const unsigned long long kk = cand_key(e); best = kk < best ? kk : best; }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const unsigned long long o2 = __shfl_xor_sync(0xffffffffu, best, off);
-                best = o2 < best ? o2 : best;
-            }
-            unsigned long long* keys = reinterpret_cast<unsigned long long*>(scs);
-            if (lane == 0) keys[warp] = best;
-            __syncthreads();
-            unsigned long long bb = keys[0];
-            for (int w = 1; w < NW; ++w) bb = keys[w] < bb ? keys[w] : bb;
-            int* fsel = reinterpret_cast<int*>(red + 40);
-            for (int e = tid; e <= lam; e += NT)
-                if (cand_key(e) == bb) *fsel = e;
-            __syncthreads();
-            const int f = *fsel;
-            // stage the folded pair
-            for (int i = tid; i < D; i += NT) phf[i] = f < lam ? a.sp.cache_phik[(cbase + f) * D + i] : phl[i];
-            for (int i = tid; i < DIM; i += NT) vf[i] = to_f32(f < lam ? ((const TIn*)a.sp.cache_v)[(cbase + f) * DIM + i] : vl[i]);
-            __syncthreads();
-            // fold (Eqs. 12-13): H += phi_f v_f^T, s += phi_f
-            for (int i = tid; i < D * DIM; i += NT) Hs[i] = fmaf(phf[i / DIM], vf[i % DIM], Hs[i]);
-            for (int i = tid; i < D; i += NT) ss[i] += phf[i];
-            // residuals of every remaining member follow the rank-1 change
-            // a quad per member: k_e = phi_e . phi_f, R_e += k_e (v_f - v_e), den_e += k_e
-            {
-                constexpr int PQ = D / 4, RQ = DIM / 4;
-                const int q4 = lane & 3, rq = lane >> 2;
-                for (int e0 = warp * 8; e0 <= lam; e0 += NW * 8) {
-                    const int e = e0 + rq;
-                    const bool act = e <= lam && e != f;
-                    float pv[PQ], vv[RQ], r0[RQ];
-                    float d0 = 0.f;
-                    if (act) {
-                        load_quarter<D>(e < lam ? a.sp.cache_phik + (cbase + e) * D : phl, q4, pv);
-                        load_quarter<DIM>(e < lam ? (const TIn*)a.sp.cache_v + (cbase + e) * DIM : vl, q4, vv);
-                        if (e < lam) {
-                            load_quarter<DIM>(Rg + (size_t)e * DIM, q4, r0);
-                            d0 = deng[e];
-                        } else {
-#pragma unroll
-                            for (int u = 0; u < RQ; ++u) r0[u] = Pl[qidx(q4, u)] - den_l * vv[u];
-                            d0 = den_l;
-                        }
-                    }
-                    float kap = 0.f;
-                    if (act) {
-#pragma unroll
-                        for (int u = 0; u < PQ; ++u) kap = fmaf(pv[u], phf[qidx(q4, u)], kap);
-                    }
-                    kap = quad_sum(kap);
-                    float q = 0.f, vq = 0.f;
-                    if (act) {
-                        const int dst = e < lam ? e : f;   // its own slot, or f's slot for the newcomer l
-                        float* rw = Rg + (size_t)dst * DIM;
-#pragma unroll
-                        for (int u = 0; u < RQ; u += 4) {
-                            const int c0 = qidx(q4, u);                       // 4 consecutive columns
-                            const float4 r4 = make_float4(
-                                fmaf(kap, vf[c0] - vv[u], r0[u]), fmaf(kap, vf[c0 + 1] - vv[u + 1], r0[u + 1]),
-                                fmaf(kap, vf[c0 + 2] - vv[u + 2], r0[u + 2]), fmaf(kap, vf[c0 + 3] - vv[u + 3], r0[u + 3]));
-                            *reinterpret_cast<float4*>(rw + c0) = r4;
-                            q = fmaf(r4.x, r4.x, q); q = fmaf(r4.y, r4.y, q);
-                            q = fmaf(r4.z, r4.z, q); q = fmaf(r4.w, r4.w, q);
-                        }
-#pragma unroll
-                        for (int u = 0; u < RQ; ++u) vq = fmaf(vv[u], vv[u], vq);
-                    }
-                    q = quad_sum(q);
-                    vq = quad_sum(vq);
-                    if (act && q4 == 0) {
-                        const int dst = e < lam ? e : f;
-                        const float dn = d0 + kap;
-                        deng[dst] = dn;
-                        a.sp.cache_sc[cbase + dst] = dn > 0.f ? q / (dn * dn) : vq;   // SRE against the new state
-                    }
-                }
-            }
-            if (f < lam) {                                            // l takes the folded member's slot
-                const size_t cs = cbase + f;
+            const float den_l = red[32];
+            float* Rg = a.sp.cache_R + cbase * DIM;
+            float* deng = a.sp.cache_den + cbase;
+            if (n_g < lam) {
+                // l joins the next free slot (fewer than lambda candidates: keep all)
+                const size_t cs = cbase + n_g;
                 for (int i = tid; i < DIM; i += NT) {
                     ((TIn*)a.sp.cache_k)[cs * DIM + i] = ((const TIn*)a.sp.win_k)[wsl * DIM + i];
                     ((TIn*)a.sp.cache_v)[cs * DIM + i] = vl[i];
+                    Rg[(size_t)n_g * DIM + i] = Pl[i] - den_l * to_f32(vl[i]);
                 }
                 for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
-                if (tid == 0) a.sp.cache_pos[cs] = lpos;
+                if (tid == 0) { a.sp.cache_pos[cs] = lpos; deng[n_g] = den_l; }
+                if (warp == 0) {                                          // its SRE against the state
+                    float q = 0.f, vq = 0.f;
+                    for (int cc = lane; cc < DIM; cc += 32) {
+                        const float v = to_f32(vl[cc]);
+                        const float r = Pl[cc] - den_l * v;
+                        q = fmaf(r, r, q);
+                        vq = fmaf(v, v, vq);
+                    }
+                    q = warp_sum(q);
+                    vq = warp_sum(vq);
+                    if (lane == 0) a.sp.cache_sc[cs] = den_l > 0.f ? q / (den_l * den_l) : vq;
+                }
+            } else {
+                // scores: members from the cache (stored when their residuals last changed), l from R_l
+                float* scs = red + 64;                                    // reuse as scratch for the argmin
+                for (int e = tid; e < lam; e += NT) sc[e] = a.sp.cache_sc[cbase + e];
+                if (warp == 0) {
+                    float q = 0.f, vq = 0.f;
+                    for (int cc = lane; cc < DIM; cc += 32) {
+                        const float v = to_f32(vl[cc]);
+                        const float r = Pl[cc] - den_l * v;
+                        q = fmaf(r, r, q);
+                        vq = fmaf(v, v, vq);
+                    }
+                    q = warp_sum(q);
+                    vq = warp_sum(vq);
+                    if (lane == 0) sc[lam] = den_l > 0.f ? q / (den_l * den_l) : vq;
+                }
+                __syncthreads();
+                // the folded pair: lowest SRE, the newer position on exact ties (keys are unique)
+                auto cand_key = [&](int e) -> unsigned long long {
+                    const int p = e < lam ? a.sp.cache_pos[cbase + e] : lpos;
+                    return ((unsigned long long)__float_as_uint(sc[e]) << 32) | (unsigned long long)(~(unsigned)p);
+                };
+                unsigned long long best = ~0ull;
+                for (int e = tid; e <= lam; e += NT) { const unsigned long long kk = cand_key(e); best = kk < best ? kk : best; }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const unsigned long long o2 = __shfl_xor_sync(0xffffffffu, best, off);
+                    best = o2 < best ? o2 : best;
+                }
+                unsigned long long* keys = reinterpret_cast<unsigned long long*>(scs);
+                if (lane == 0) keys[warp] = best;
+                __syncthreads();
+                unsigned long long bb = keys[0];
+                for (int w = 1; w < NW; ++w) bb = keys[w] < bb ? keys[w] : bb;
+                int* fsel = reinterpret_cast<int*>(red + 40);
+                for (int e = tid; e <= lam; e += NT)
+                    if (cand_key(e) == bb) *fsel = e;
+                __syncthreads();
+                const int f = *fsel;
+                // stage the folded pair
+                for (int i = tid; i < D; i += NT) phf[i] = f < lam ? a.sp.cache_phik[(cbase + f) * D + i] : phl[i];
+                for (int i = tid; i < DIM; i += NT) vf[i] = to_f32(f < lam ? ((const TIn*)a.sp.cache_v)[(cbase + f) * DIM + i] : vl[i]);
+                __syncthreads();
+                // fold (Eqs. 12-13): H += phi_f v_f^T, s += phi_f
+                for (int i = tid; i < D * DIM; i += NT) Hs[i] = fmaf(phf[i / DIM], vf[i % DIM], Hs[i]);
+                for (int i = tid; i < D; i += NT) ss[i] += phf[i];
+                // residuals of every remaining member follow the rank-1 change
+                // a quad per member: k_e = phi_e . phi_f, R_e += k_e (v_f - v_e), den_e += k_e
+                {
+                    constexpr int PQ = D / 4, RQ = DIM / 4;
+                    const int q4 = lane & 3, rq = lane >> 2;
+                    for (int e0 = warp * 8; e0 <= lam; e0 += NW * 8) {
+                        const int e = e0 + rq;
+                        const bool act = e <= lam && e != f;
+                        float pv[PQ], vv[RQ], r0[RQ];
+                        float d0 = 0.f;
+                        if (act) {
+                            load_quarter<D>(e < lam ? a.sp.cache_phik + (cbase + e) * D : phl, q4, pv);
+                            load_quarter<DIM>(e < lam ? (const TIn*)a.sp.cache_v + (cbase + e) * DIM : vl, q4, vv);
+                            if (e < lam) {
+                                load_quarter<DIM>(Rg + (size_t)e * DIM, q4, r0);
+                                d0 = deng[e];
+                            } else {
+#pragma unroll
+                                for (int u = 0; u < RQ; ++u) r0[u] = Pl[qidx(q4, u)] - den_l * vv[u];
+                                d0 = den_l;
+                            }
+                        }
+                        float kap = 0.f;
+                        if (act) {
+#pragma unroll
+                            for (int u = 0; u < PQ; ++u) kap = fmaf(pv[u], phf[qidx(q4, u)], kap);
+                        }
+                        kap = quad_sum(kap);
+                        float q = 0.f, vq = 0.f;
+                        if (act) {
+                            const int dst = e < lam ? e : f;   // its own slot, or f's slot for the newcomer l
+                            float* rw = Rg + (size_t)dst * DIM;
+#pragma unroll
+                            for (int u = 0; u < RQ; u += 4) {
+                                const int c0 = qidx(q4, u);                       // 4 consecutive columns
+                                const float4 r4 = make_float4(
+                                    fmaf(kap, vf[c0] - vv[u], r0[u]), fmaf(kap, vf[c0 + 1] - vv[u + 1], r0[u + 1]),
+                                    fmaf(kap, vf[c0 + 2] - vv[u + 2], r0[u + 2]), fmaf(kap, vf[c0 + 3] - vv[u + 3], r0[u + 3]));
+                                *reinterpret_cast<float4*>(rw + c0) = r4;
+                                q = fmaf(r4.x, r4.x, q); q = fmaf(r4.y, r4.y, q);
+                                q = fmaf(r4.z, r4.z, q); q = fmaf(r4.w, r4.w, q);
+                            }
+#pragma unroll
+                            for (int u = 0; u < RQ; ++u) vq = fmaf(vv[u], vv[u], vq);
+                        }
+                        q = quad_sum(q);
+                        vq = quad_sum(vq);
+                        if (act && q4 == 0) {
+                            const int dst = e < lam ? e : f;
+                            const float dn = d0 + kap;
+                            deng[dst] = dn;
+                            a.sp.cache_sc[cbase + dst] = dn > 0.f ? q / (dn * dn) : vq;   // SRE against the new state
+                        }
+                    }
+                }
+                if (f < lam) {                                            // l takes the folded member's slot
+                    const size_t cs = cbase + f;
+                    for (int i = tid; i < DIM; i += NT) {
+                        ((TIn*)a.sp.cache_k)[cs * DIM + i] = ((const TIn*)a.sp.win_k)[wsl * DIM + i];
+                        ((TIn*)a.sp.cache_v)[cs * DIM + i] = vl[i];
+                    }
+                    for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
+                    if (tid == 0) a.sp.cache_pos[cs] = lpos;
+                }
+                __syncthreads();
+                for (int i = tid; i < D * DIM / 4; i += NT)
+                    reinterpret_cast<float4*>(Hg)[i] = reinterpret_cast<const float4*>(Hs)[i];
+                for (int i = tid; i < D; i += NT) sg[i] = ss[i];
             }
-            __syncthreads();
-            for (int i = tid; i < D * DIM / 4; i += NT)
-                reinterpret_cast<float4*>(Hg)[i] = reinterpret_cast<const float4*>(Hs)[i];
-            for (int i = tid; i < D; i += NT) sg[i] = ss[i];
         }
-    }
-    __syncthreads();
-    // the new token enters the window ring
-    {
-        const size_t ws = wbase + (size_t)(t % eta);
-        for (int i = tid; i < DIM; i += NT) {
-            ((TIn*)a.sp.win_k)[ws * DIM + i] = kg[i];
-            ((TIn*)a.sp.win_v)[ws * DIM + i] = vg[i];
+        __syncthreads();
+        // the new token enters the window ring
+        {
+            const size_t ws = wbase + (size_t)(t % eta);
+            for (int i = tid; i < DIM; i += NT) {
+                ((TIn*)a.sp.win_k)[ws * DIM + i] = kg[i];
+                ((TIn*)a.sp.win_v)[ws * DIM + i] = vg[i];
+            }
+            for (int i = tid; i < D; i += NT) a.sp.win_phik[ws * D + i] = phk[i];
         }
-        for (int i = tid; i < D; i += NT) a.sp.win_phik[ws * D + i] = phk[i];
+    };
+
+    if (!a.update_first) {
+        read_phase(NK);
+        update_phase();
+    } else {
+        // the token equations read literally: update, then read the new memories
+        // (cache slots [0, min(lambda, t + 1 - eta)), window [t + 1 - eta, t), the token)
+        update_phase();
+        __syncthreads();
+        const int nk = fill_kp(hide_sparse ? 0 : min(lam, max(0, t + 1 - eta)), max(0, t + 1 - eta));
+        __syncthreads();
+        read_phase(nk);
     }
 }
 

@@ -63,6 +63,7 @@ struct PrefillArgs {
     int t_start;           // position of the first token of the call
     int nc;                // chunks in this call
     int c_begin, c_end;    // chunks [c_begin, c_end) of the call served by this launch (scan, output)
+    int read_mask;         // bit 0: queries do not read (H, s); bit 1: nor the sparse cache
     float* phik_new;       // [S][max_tokens][D]
     int* snap_pos;         // [S][nc_max+1][lambda]
     float* snap_H;         // [S][nc_max+1][d][D] (H_c transposed)
@@ -78,7 +79,25 @@ struct DecodeArgs {
     const void* v;
     float* y;              // [B][Hq][d]
     int t;                 // position of the new token
+    int read_mask;         // as PrefillArgs::read_mask
+    int update_first;      // 1: update the memories, then read them (token equations read literally)
     int* err;              // device error word
+};
+
+// Stored-pair SRE map of the last prefill call (analysis; reads the snapshots).
+struct SreMapArgs {
+    Dims dm;
+    const void* k;         // [B][T][Hkv][d]  every position of the sequence so far
+    const void* v;
+    const void* W;         // [Hkv][d][Dh]
+    const float* snap_H;   // [S][nc_max+1][d][D] (H_c transposed)
+    const float* snap_s;   // [S][nc_max+1][D]
+    const int* snap_pos;   // [S][nc_max+1][lambda]
+    float* sre;            // [S][nc+1][T]
+    float* rel;            // [S][nc+1][T] or null
+    int T;                 // positions covered
+    int t0;                // first position of the last prefill call
+    int nc;                // its chunks
 };
 
 // Launchers (each returns cudaGetLastError() of its launch).
@@ -88,6 +107,7 @@ cudaError_t launch_output(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_output_tc(const PrefillArgs& a, cudaStream_t s);   // bf16 on tcgen05
 cudaError_t launch_finalize(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_sre_map(const SreMapArgs& a, cudaStream_t s);
 cudaError_t launch_residual_init(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_clear(const Dims& dm, const StatePtrs& sp, cudaStream_t s);
 

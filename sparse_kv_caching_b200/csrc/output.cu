@@ -90,19 +90,21 @@ __global__ void __launch_bounds__(256) output_kernel(const __grid_constant__ Pre
     const size_t snaps = (size_t)dm.nc_max + 1;
     const float* Hc = a.snap_H + ((size_t)st * snaps + c) * D * DIM;
     const float* sc = a.snap_s + ((size_t)st * snaps + c) * D;
+    const bool read_state = !(a.read_mask & 1);
     float acc[QPW][CPL], m[QPW], l[QPW];
 #pragma unroll
     for (int qq = 0; qq < QPW; ++qq) {
         const int r = warp * QPW + qq;
         float x = 0.f;
-        for (int j = lane; j < D; j += 32) x = fmaf(Ph[r * D + j], sc[j], x);
+        if (read_state)
+            for (int j = lane; j < D; j += 32) x = fmaf(Ph[r * D + j], sc[j], x);
         l[qq] = warp_sum(x);
         m[qq] = l[qq] > 0.f ? 0.f : -INFINITY;
 #pragma unroll
         for (int u = 0; u < CPL; ++u) acc[qq][u] = 0.f;
     }
     constexpr int HT = KT;                            // H rows per tile (uses the Vs buffer)
-    for (int j0 = 0; j0 < D; j0 += HT) {
+    for (int j0 = 0; read_state && j0 < D; j0 += HT) {
         const int nj = min(HT, D - j0);
         __syncthreads();
         for (int idx = tid; idx < nj * DIM; idx += 256) {     // snapshot is H^T [d][D]
@@ -124,7 +126,7 @@ __global__ void __launch_bounds__(256) output_kernel(const __grid_constant__ Pre
     }
 
     // exact keys: cache slots, then the window, then the block up to the last query
-    const int n_g = min(dm.lam, max(0, t0 - dm.eta));
+    const int n_g = (a.read_mask & 2) ? 0 : min(dm.lam, max(0, t0 - dm.eta));
     const int w_lo = max(0, t0 - dm.eta);
     const int n_w = t0 - w_lo;
     const int n_c = qb * QB + nq;

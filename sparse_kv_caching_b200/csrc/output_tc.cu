@@ -94,7 +94,8 @@ __global__ void __launch_bounds__(128, 2) output_tc_kernel(const __grid_constant
     uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + Sh::MBAR);
     uint32_t* tptr = reinterpret_cast<uint32_t*>(smem + Sh::TPTR);
     const size_t snaps = (size_t)dm.nc_max + 1;
-    const bool has_lin = (t0 - dm.eta) > dm.lam;          // something was folded before block c
+    // something was folded before block c, and the state branch is read
+    const bool has_lin = (t0 - dm.eta) > dm.lam && !(a.read_mask & 1);
 
     if (warp == 0) umma::tmem_alloc(tptr, Sh::TMEM_COLS);
     if (tid == 0) { umma::mbar_init(&mbar[0], 1); umma::mbar_init(&mbar[1], 1); umma::fence_mbar_init(); }
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(128, 2) output_tc_kernel(const __grid_constant
     }
 
     // ---- exact keys: cache slots, window, block keys up to the last query of the CTA ----
-    const int n_g = min(dm.lam, max(0, t0 - dm.eta));
+    const int n_g = (a.read_mask & 2) ? 0 : min(dm.lam, max(0, t0 - dm.eta));
     const int w_lo = max(0, t0 - dm.eta);
     const int n_w = t0 - w_lo;
     const int N = n_g + n_w + qi_max + 1;
