@@ -254,7 +254,7 @@ def oracle_sample(w: synth.Workload, streams, budget_s: float, gpu=None):
             gset = exp.get(rec["t0"])
             if gset is None or gset == rec["keep"]:
                 return None
-            if valid_alternative(rec["E"], rec["sre"], w.lam, gset):
+            if valid_alternative(rec["E"], rec["score"], w.lam, gset):
                 stats["ties"] += 1
                 return gset
             stats["hard"] += 1

@@ -5,8 +5,8 @@ cpu_baseline / reference leg of bench.py, never by the product library.
 """
 from .lola_oracle import (LolaStream, feature_map, self_recall_error, top_lambda,
                           valid_alternative, state_elements, full_elements, sre_map, TIE_REL,
-                          HIDE_STATE, HIDE_SPARSE)
+                          HIDE_STATE, HIDE_SPARSE, SCORERS)
 
 __all__ = ["LolaStream", "feature_map", "self_recall_error", "top_lambda",
            "valid_alternative", "state_elements", "full_elements", "sre_map", "TIE_REL",
-           "HIDE_STATE", "HIDE_SPARSE"]
+           "HIDE_STATE", "HIDE_SPARSE", "SCORERS"]

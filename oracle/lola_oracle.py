@@ -41,6 +41,16 @@ reason and under the same number, in the design notes of this repository):
       back leaves it and is scored with the cache against the state, and
       only then does the query read; it sees the eta most recent pairs,
       itself included.  The memories evolve exactly as under R3.
+  R18 Alternative scoring rules (notes §4.5, Table 4; App. F, whose Eqs.
+      22-25 the pages do not print): with a = exp(q.k / sqrt(d)) (the
+      exponential kernel of Eq. 14) and f = phi(q)^T phi(k) (the feature
+      kernel), a key's score is the sum over every query that reads it
+      exactly through the window or its own block (any head of the group) of
+      (a - f)^2 ("kernel_sq"), |a - f| ("kernel_abs"), f / a ("kernel_ratio":
+      keys the linear kernel over-weights score high) or a ("attn").  The sum
+      stops when the key leaves the window (the scores are accumulated while
+      the key is in the window, never from later queries) and is frozen while
+      the key is cached.  The lambda highest scores are kept, as for SRE.
   R17 Stored-pair SRE map (notes §4.4, Fig. 3): at each state time (a block
       boundary) every folded pair's SRE against that state; pairs not in the
       state are 0.  Relative SRE (notes §4.4, Fig. 10, Eq. 26): that value
@@ -63,6 +73,20 @@ import numpy as np
 TIE_REL = 1e-5   # relative band around the lambda-th SRE inside which swaps are valid
 HIDE_STATE = 1   # read mask bit: the queries do not read (H, s)            (R15)
 HIDE_SPARSE = 2  # read mask bit: the queries do not read the sparse cache G (R15)
+SCORERS = ("sre", "kernel_sq", "kernel_abs", "kernel_ratio", "attn")   # R1 and R18
+
+
+def window_score_terms(a: np.ndarray, f: np.ndarray, rule: str) -> np.ndarray:
+    """Per-(query, key) term of an alternative scoring rule (R18), a = exp kernel, f = feature kernel."""
+    if rule == "kernel_sq":
+        return (a - f) ** 2
+    if rule == "kernel_abs":
+        return np.abs(a - f)
+    if rule == "kernel_ratio":
+        return f / a
+    if rule == "attn":
+        return a
+    raise ValueError(f"unknown scoring rule {rule!r}")
 
 
 # ---------------------------------------------------------------------------
@@ -147,15 +171,19 @@ class LolaStream:
     index it; the memories themselves hold positions only.
     """
 
-    def __init__(self, W: np.ndarray, eta: int, lam: int, read_mask: int = 0):
+    def __init__(self, W: np.ndarray, eta: int, lam: int, read_mask: int = 0, scorer: str = "sre"):
         self.W = np.asarray(W, np.float64)
         self.read_mask = int(read_mask)
+        if scorer not in SCORERS:
+            raise ValueError(f"unknown scoring rule {scorer!r}")
+        self.scorer = scorer
         self.d, self.Dh = self.W.shape
         self.D = 2 * self.Dh
         self.eta, self.lam = int(eta), int(lam)
         self._K = np.zeros((0, self.d))
         self._V = np.zeros((0, self.d))
         self._phiK = np.zeros((0, self.D))
+        self._acc = np.zeros(0)         # accumulated window score of each key (R18)
         self.t = 0
         self.window: list[int] = []     # W: positions, oldest first
         self.cache: list[int] = []      # G: positions (sorted)
@@ -187,6 +215,10 @@ class LolaStream:
                 grown = np.zeros((cap, width))
                 grown[:self.t] = getattr(self, name)[:self.t]
                 setattr(self, name, grown)
+            acc = np.zeros(cap)
+            acc[:self.t] = self._acc[:self.t]
+            self._acc = acc
+        self._acc[self.t:self.t + n] = 0.0
         self._K[self.t:self.t + n] = k
         self._V[self.t:self.t + n] = v
         self._phiK[self.t:self.t + n] = feature_map(k, self.W)
@@ -226,6 +258,19 @@ class LolaStream:
         return y
 
     # -- one update interval (notes §2.4 and §2.6) -------------------------
+    def _accumulate(self, Q: np.ndarray, P: list[int], qpos: list[int]) -> None:
+        """R18: add every query's term to the keys it reads exactly through the window
+        or its own block (P, causally).  Q [Gq, n, d] are the queries at positions qpos."""
+        if self.scorer == "sre":
+            return
+        scale = 1.0 / np.sqrt(self.d)
+        for qi, t in enumerate(qpos):
+            keys = self.window + [j for j in P if j <= t]
+            q = np.asarray(Q[:, qi], np.float64)                     # [Gq, d]
+            a = np.exp((q @ self.K[keys].T) * scale)                  # [Gq, n_keys]
+            f = feature_map(q, self.W) @ self.phiK[keys].T
+            self._acc[keys] += window_score_terms(a, f, self.scorer).sum(axis=0)
+
     def step(self, Q, K, V, rows=None, choose=None) -> np.ndarray:
         """Process one block of new tokens: read, advance window, score, keep, fold.
 
@@ -239,29 +284,34 @@ class LolaStream:
             Q = Q[:, None, :]
         P = self._append(K, V)
         y = self._read(Q, P, rows)
+        self._accumulate(Q, P, P)
         self._update(P, choose)
         return y
 
     def _update(self, P: list[int], choose=None) -> None:
-        """Window advance, candidates, SRE, top-lambda and fold for the new positions P."""
+        """Window advance, candidates, scores (SRE or R18), top-lambda and fold for the new positions P."""
         # advance the window: the block enters, the oldest pairs beyond eta leave (R2)
         self.window.extend(P)
         n_leave = max(0, len(self.window) - self.eta)
         L, self.window = self.window[:n_leave], self.window[n_leave:]
         E = self.cache + L                          # candidate set E
-        rec = dict(t0=P[0], n=len(P), E=E, L=L, sre=None, keep=None, fold=[], adopted=False,
+        rec = dict(t0=P[0], n=len(P), E=E, L=L, sre=None, score=None, keep=None, fold=[], adopted=False,
                    cache_before=list(self.cache), window_after=list(self.window),
                    folded_before=len(self.folded))
         if len(E) <= self.lam:                      # R6
             self.cache = sorted(E)
         else:
-            sre = self_recall_error(self.phiK[E], self.V[E], self.H, self.s)   # pre-fold state
-            keep = top_lambda(E, sre, self.lam)
-            rec.update(sre=sre, keep=keep)
+            if self.scorer == "sre":
+                score = self_recall_error(self.phiK[E], self.V[E], self.H, self.s)   # pre-fold state
+                rec.update(sre=score)
+            else:
+                score = self._acc[E].copy()          # frozen window accumulations (R18)
+            keep = top_lambda(E, score, self.lam)
+            rec.update(score=score, keep=keep)
             if choose is not None:
                 alt = choose(rec)
                 if alt is not None and sorted(alt) != keep:
-                    if not valid_alternative(E, sre, self.lam, list(alt)):
+                    if not valid_alternative(E, score, self.lam, list(alt)):
                         raise ValueError("rejected retained set: not a top-lambda set up to ties")
                     keep = sorted(alt)
                     rec.update(keep=keep, adopted=True)
@@ -296,7 +346,8 @@ class LolaStream:
             return self.step(Q, k, v, None, choose)[:, 0]
         P = self._append(k, v)
         self._update(P, choose)
-        return self._read(Q, [], None)[:, 0]     # the new pair is now the newest window member
+        self._accumulate(Q, [], P)               # the new pair is now the newest window member
+        return self._read(Q, [], None)[:, 0]
 
 
 # ---------------------------------------------------------------------------

@@ -61,7 +61,7 @@ class ChainCheck:
         gpu = self.expected
         if gpu is None or gpu == rec["keep"]:
             return None
-        if valid_alternative(rec["E"], rec["sre"], self.lam, gpu):
+        if valid_alternative(rec["E"], rec["score"], self.lam, gpu):
             self.ties += 1
             return gpu
         self.hard += 1

@@ -356,3 +356,82 @@ def check_sre_map(Stream, map_fn) -> float:
             first.setdefault(i, want)
             err = max(err, abs(sre[c, i] - want), abs(rel[c, i] - (want - first[i])))
     return err
+
+
+# Alternative scoring rules (R18): a key's score sums one term per query that reads it
+# through the window or its own block.  Closed forms and a brute-force recount.
+_RULE_CONST = {"kernel_sq": lambda a, f: (a - f) ** 2, "kernel_abs": lambda a, f: abs(a - f),
+               "kernel_ratio": lambda a, f: f / a, "attn": lambda a, f: a}
+
+
+def _window_reads(i, eta, C, T):
+    """Queries that read key i exactly before it leaves the window (R2), by hand:
+    its own block from i on, then the blocks whose preceding eta pairs hold it."""
+    return list(range(i, min(T, ((i + eta) // C + 1) * C)))
+
+
+def check_scorers(Stream) -> float:
+    err = 0.0
+    for rule, term in _RULE_CONST.items():
+        # (1) q = 0: a = 1 and f = phi(0)^T phi(k) = 2 / Dh for every key (each half of phi sums to 1)
+        w, a, W = small(T=64, eta=8, lam=5, C=4)
+        a0 = dict(a, q=np.zeros_like(a["q"]))
+        st = Stream(W, w.eta, w.lam)
+        st.scorer = rule
+        st.prefill(a0["q"], a0["k"], a0["v"], w.chunk)
+        const = term(1.0, 2.0 / w.Dh)
+        n_scored = 0
+        for rec in st.log:
+            if rec["score"] is None:
+                continue
+            n_scored += 1
+            for e, sc in zip(rec["E"], rec["score"]):
+                want = w.Gq * const * len(_window_reads(e, w.eta, w.chunk, w.T))
+                err = max(err, abs(sc - want) / want)
+        if n_scored == 0:
+            return np.inf
+        # per-token decode: eta + 1 reads (read first) or eta reads (update first)
+        for uf in (False, True):
+            st = Stream(W, w.eta, w.lam)
+            st.scorer = rule
+            for t in range(40):
+                st.decode(a0["q"][:, t], a0["k"][t], a0["v"][t], update_first=uf)
+            for rec in st.log:
+                if rec["score"] is not None:
+                    for sc in rec["score"]:
+                        err = max(err, abs(sc - w.Gq * const * (w.eta + (0 if uf else 1))) / sc)
+        # (2) every key and query the same vector x: a = exp(|x|^2 / sqrt(d)), f = |phi(x)|^2
+        x = a["k"][3].astype(np.float64)
+        ax = dict(a, k=np.tile(x, (w.T, 1)), q=np.tile(x, (w.Gq, w.T, 1)))
+        st = Stream(W, w.eta, w.lam)
+        st.scorer = rule
+        st.prefill(ax["q"], ax["k"], ax["v"], w.chunk)
+        av = float(np.exp(np.linalg.norm(x) ** 2 / np.sqrt(w.d)))
+        fv = float(np.linalg.norm(softmax_fm(x[None], W)[0]) ** 2)
+        for rec in st.log:
+            if rec["score"] is not None:
+                for e, sc in zip(rec["E"], rec["score"]):
+                    want = w.Gq * term(av, fv) * len(_window_reads(e, w.eta, w.chunk, w.T))
+                    err = max(err, abs(sc - want) / want)
+        # (3) general inputs: scores recounted key by key; each kept key beats each folded one
+        st = Stream(W, w.eta, w.lam)
+        st.scorer = rule
+        st.prefill(a["q"], a["k"], a["v"], w.chunk)
+        q, k = np.asarray(a["q"], np.float64), np.asarray(a["k"], np.float64)
+        pk = softmax_fm(k, W)
+        for rec in st.log:
+            if rec["score"] is None:
+                continue
+            got = dict(zip(rec["E"], rec["score"]))
+            for e in rec["E"]:
+                want = 0.0
+                for t in _window_reads(e, w.eta, w.chunk, w.T):
+                    for h in range(w.Gq):
+                        want += term(np.exp(q[h, t] @ k[e] / np.sqrt(w.d)), softmax_fm(q[h, t][None], W)[0] @ pk[e])
+                err = max(err, abs(got[e] - want) / abs(want))
+            keep = set(rec["keep"])
+            for i in keep:
+                for j in rec["E"]:
+                    if j not in keep and not (got[i] > got[j] or (got[i] == got[j] and i < j)):
+                        return np.inf
+    return err

@@ -71,6 +71,10 @@ def test_update_first_decode():
     assert pins.check_update_first(LolaStream) < 1e-12
 
 
+def test_alternative_scorers():
+    assert pins.check_scorers(LolaStream) < 1e-12
+
+
 def test_sre_map_closed_forms():
     assert pins.check_sre_map(LolaStream, sre_map) < 1e-12
 
@@ -150,6 +154,7 @@ def _all_pins_pass(Stream, sre_fn=None, map_fn=None):
         ok &= pins.check_mask_one_branch(Stream) < 1e-9
         ok &= pins.check_update_first(Stream) < 1e-9
         ok &= pins.check_sre_map(Stream, map_fn or lo.sre_map) < 1e-9
+        ok &= pins.check_scorers(Stream) < 1e-9
         ok &= pins.check_sre_closed_form(sre_fn or lo.self_recall_error) < 1e-9
         ok &= pins.check_full_softmax(Stream) < 1e-9
         ok &= pins.check_lambda0(Stream) < 1e-9
@@ -259,6 +264,21 @@ class _UpdateFirstReadsEarly(LolaStream):
         return super().decode(q, k, v, choose, False)
 
 
+class _ScoreNoScale(LolaStream):               # exp kernel without the 1/sqrt(d)
+    def _accumulate(self, Q, P, qpos):
+        d = self.d
+        self.d = 1
+        try:
+            super()._accumulate(Q, P, qpos)
+        finally:
+            self.d = d
+
+
+class _ScoreSkipsBlock(LolaStream):           # the block's own causal keys are not credited
+    def _accumulate(self, Q, P, qpos):
+        super()._accumulate(Q, [], qpos)
+
+
 def _map_state_off_by_one(st, first_block=0):
     sre, rel = lo.sre_map(st, first_block)
     return np.vstack([np.zeros((1, sre.shape[1])), sre[:-1]]), np.vstack([np.zeros((1, rel.shape[1])), rel[:-1]])
@@ -280,7 +300,8 @@ class _WindowOffByOne(LolaStream):
                                   "keep_lowest", "tie_rule", "feature_same_half", "no_s_update",
                                   "fold_transposed", "no_linear_read", "window_off_by_one",
                                   "mask_ignored", "mask_numerator_only", "update_first_reads_early",
-                                  "map_state_off_by_one", "map_rel_from_previous"])
+                                  "map_state_off_by_one", "map_rel_from_previous",
+                                  "ratio_inverted", "score_no_scale", "score_skips_block"])
 def test_planted_mistakes_are_caught(monkeypatch, name):
     Stream = LolaStream
     sre_fn = None
@@ -316,4 +337,12 @@ def test_planted_mistakes_are_caught(monkeypatch, name):
         map_fn = _map_state_off_by_one
     elif name == "map_rel_from_previous":
         map_fn = _map_rel_from_previous
+    elif name == "ratio_inverted":
+        orig = lo.window_score_terms
+        monkeypatch.setattr(lo, "window_score_terms",
+                            lambda a, f, rule: a / f if rule == "kernel_ratio" else orig(a, f, rule))
+    elif name == "score_no_scale":
+        Stream = _ScoreNoScale
+    elif name == "score_skips_block":
+        Stream = _ScoreSkipsBlock
     assert not _all_pins_pass(Stream, sre_fn, map_fn)
