@@ -179,6 +179,28 @@ int lola_decode_step_host(lola_state* st, const void* q, const void* k, const vo
 #define LOLA_READ_HIDE_SPARSE 2
 int lola_set_read_options(lola_state* st, int read_mask, int decode_update_first);
 
+/* Scoring rule that ranks the leaving pairs and the cache members (notes
+ * §4.5, Table 4; App. F, whose Eqs. 22-25 the pages do not print).
+ * LOLA_SCORE_SRE (default) is Eq. 10 against the state.  The four
+ * alternatives score a key by a sum over every query that reads it exactly
+ * through the window or its own block (all heads of its kv group), with
+ * a = exp(q.k / sqrt(d)) and f = phi(q)^T phi(k):
+ *   LOLA_SCORE_KERNEL_SQ     (a - f)^2      LOLA_SCORE_KERNEL_ABS  |a - f|
+ *   LOLA_SCORE_KERNEL_RATIO  f / a          LOLA_SCORE_ATTN        a
+ * The sum stops when the key leaves the window and stays frozen while the
+ * key is cached; the lambda highest scores are kept (older position on exact
+ * ties), the rest folded, as for SRE.  Under decode_update_first a query
+ * credits the window it reads after the update.  The rule can change only
+ * while no token has been processed (after init or reset; it persists across
+ * resets); LOLA_ERR_INVALID_ARG otherwise or for another value.  Prefill
+ * with an alternative rule runs unsegmented on `stream`. */
+#define LOLA_SCORE_SRE          0
+#define LOLA_SCORE_KERNEL_SQ    1
+#define LOLA_SCORE_KERNEL_ABS   2
+#define LOLA_SCORE_KERNEL_RATIO 3
+#define LOLA_SCORE_ATTN         4
+int lola_set_scorer(lola_state* st, int scorer);
+
 /* Stored-pair SRE map of the last prefill call (notes §4.4: Fig. 3, and
  * Fig. 10 / Eq. 26 for the relative form).  With n = the chunks of that call
  * (trace_len - 1 of lola_state_export) and t_c = its first position + c *

@@ -26,9 +26,10 @@ EXPORTS = ("lola_state_bytes", "lola_state_init", "lola_state_reset", "lola_stat
            "lola_prefill_chunked", "lola_decode_step", "lola_prefill_chunked_host",
            "lola_decode_step_host", "lola_state_export", "lola_profile_enable",
            "lola_profile_read", "lola_launch_count", "lola_prefill_once_noalloc", "lola_selftest_umma",
-           "lola_set_read_options", "lola_sre_map", "lola_last_error_string")
+           "lola_set_read_options", "lola_sre_map", "lola_set_scorer", "lola_last_error_string")
 KERNEL_CLASSES = ("phi", "scan", "output", "finalize", "decode", "sre_map")
 READ_HIDE_STATE, READ_HIDE_SPARSE = 1, 2
+SCORERS = ("sre", "kernel_sq", "kernel_abs", "kernel_ratio", "attn")   # LOLA_SCORE_* in this order
 
 
 class LolaConfig(ctypes.Structure):
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
     L.lola_selftest_umma.argtypes = [c_int, vp, vp, vp, c_int, c_int, c_int, vp, vp]
     L.lola_set_read_options.argtypes = [vp, c_int, c_int]
     L.lola_sre_map.argtypes = [vp, vp, vp, c_int, vp, vp, vp]
+    L.lola_set_scorer.argtypes = [vp, c_int]
     L.lola_launch_count.argtypes = []
     L.lola_launch_count.restype = c_longlong
     L.lola_last_error_string.argtypes = []
@@ -233,6 +235,11 @@ class LolaLayer:
     def set_read_options(self, read_mask: int = 0, decode_update_first: bool = False) -> None:
         """Hide memory branches from later reads (READ_HIDE_* bits); update-first decode order."""
         _check(lib().lola_set_read_options(self.handle, int(read_mask), 1 if decode_update_first else 0))
+
+    def set_scorer(self, scorer) -> None:
+        """Scoring rule (a name from SCORERS or its LOLA_SCORE_* number); only before the first token."""
+        code = SCORERS.index(scorer) if isinstance(scorer, str) else int(scorer)
+        _check(lib().lola_set_scorer(self.handle, code))
 
     def sre_map(self, k, v, sre=None, rel=None, stream=None):
         """SRE of every folded pair at each state time of the last prefill call, and its change

@@ -38,6 +38,7 @@ struct lola_state {
     bool resid_ok = true;     // per-slot decode residuals match (H, s)
     int read_mask = 0;        // LOLA_READ_HIDE_* bits applied to every read
     int update_first = 0;     // decode: update the memories before the read
+    int scorer = 0;           // LOLA_SCORE_*: how leaving pairs and members are ranked
     std::vector<lola_prof_mark> marks;
     std::vector<cudaEvent_t> pool;
     // Prefill overlap: the chain runs on a high-priority stream in chunk segments,
@@ -142,7 +143,9 @@ lola::Layout make_layout(const lola::Dims& dm) {
     L.cache_R = take(S * dm.lam * dm.d * 4);
     L.cache_den = take(S * dm.lam * 4);
     L.cache_sc = take(S * dm.lam * 4);
+    L.win_sc = take(S * dm.eta * 4);
     L.phik_new = take(S * T * dm.D * 4);
+    L.key_sc = take(S * (dm.eta + T) * 4);
     L.snap_pos = take(S * snaps * dm.lam * 4);
     L.snap_H = take(S * snaps * dm.D * dm.d * 4);
     L.snap_s = take(S * snaps * dm.D * 4);
@@ -171,6 +174,7 @@ lola::StatePtrs state_ptrs(const lola_state* st) {
     p.cache_R = (float*)(b + st->L.cache_R);
     p.cache_den = (float*)(b + st->L.cache_den);
     p.cache_sc = (float*)(b + st->L.cache_sc);
+    p.win_sc = (float*)(b + st->L.win_sc);
     return p;
 }
 
@@ -300,6 +304,17 @@ int lola_sre_map(lola_state* st, const void* k, const void* v, int T, float* sre
     return LOLA_OK;
 }
 
+int lola_set_scorer(lola_state* st, int scorer) {
+    if (!st) return fail(LOLA_ERR_INVALID_ARG, "null state");
+    if (scorer < LOLA_SCORE_SRE || scorer > LOLA_SCORE_ATTN)
+        return fail(LOLA_ERR_INVALID_ARG, "scorer=%d is not one of the LOLA_SCORE_* rules", scorer);
+    if (st->t != 0 && scorer != st->scorer)
+        return fail(LOLA_ERR_INVALID_ARG, "the scoring rule can change only before the first token "
+                    "(after lola_state_init or lola_state_reset)");
+    st->scorer = scorer;
+    return LOLA_OK;
+}
+
 int lola_set_read_options(lola_state* st, int read_mask, int decode_update_first) {
     if (!st) return fail(LOLA_ERR_INVALID_ARG, "null state");
     if (read_mask & ~(LOLA_READ_HIDE_STATE | LOLA_READ_HIDE_SPARSE))
@@ -374,6 +389,8 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
     a.c_begin = 0;
     a.c_end = a.nc;
     a.read_mask = st->read_mask;
+    a.scorer = st->scorer;
+    a.key_sc = (float*)(st->base + st->L.key_sc);
     a.phik_new = (float*)(st->base + st->L.phik_new);
     a.snap_pos = (int*)(st->base + st->L.snap_pos);
     a.snap_H = (float*)(st->base + st->L.snap_H);
@@ -385,7 +402,20 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
         return dm.dtype == LOLA_DTYPE_BF16 ? lola::launch_output_tc(a, q) : lola::launch_output(a, q);
     };
     const int seg = a.nc >= kSplitMinChunks ? (a.nc + kSplitSegments - 1) / kSplitSegments : a.nc;
-    if (st->s_chain && seg < a.nc) {
+    if (st->scorer != LOLA_SCORE_SRE) {
+        // Alternative rules: every key's window score first (it needs the call's queries,
+        // not the state), then the chain ranks by those scores, then the output.
+        if ((e = traced(st, 0, 1, s, [&] { return lola::launch_phi_keys(a, s); })) != cudaSuccess)
+            return cuda_fail(e, "feature-map kernel");
+        if ((e = traced(st, 1, 1, s, [&] { return lola::launch_key_scores(a, s); })) != cudaSuccess)
+            return cuda_fail(e, "window-score kernel");
+        if ((e = traced(st, 1, 1, s, [&] { return lola::launch_scan(a, s); })) != cudaSuccess)
+            return cuda_fail(e, "scan kernel");
+        if ((e = traced(st, 2, 1, s, [&] { return output(s); })) != cudaSuccess)
+            return cuda_fail(e, "output kernel");
+        if ((e = traced(st, 3, 1, s, [&] { return lola::launch_finalize_scores(a, s); })) != cudaSuccess)
+            return cuda_fail(e, "window-score finalize kernel");
+    } else if (st->s_chain && seg < a.nc) {
         // The chain of segment i and the output of segment i-1 run at the same time:
         // the chain holds one cluster per stream, the output fills the other SMs.  The
         // feature map of the first segment's keys runs first; the rest of the keys
@@ -449,10 +479,11 @@ int lola_decode_step(lola_state* st, const void* q, const void* k, const void* v
     a.t = (int)st->t;
     a.read_mask = st->read_mask;
     a.update_first = st->update_first;
+    a.scorer = st->scorer;
     a.err = (int*)(st->base + st->L.err);
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (!st->resid_ok) {
+    if (!st->resid_ok && st->scorer == LOLA_SCORE_SRE) {
         if ((e = traced(st, 4, st->dm.lam > 0 ? 1 : 0, s, [&] { return lola::launch_residual_init(a, s); })) != cudaSuccess)
             return cuda_fail(e, "decode residual init kernel");
         st->resid_ok = true;

@@ -159,7 +159,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     };
     // read first: the memories entering the step (the window holds [t - eta, t));
     // update first reads after the update (see the end of the kernel)
-    const int NK = a.update_first ? 0 : fill_kp(hide_sparse ? 0 : n_g, max(0, t - eta));
+    const int rg0 = hide_sparse ? 0 : n_g, rlo0 = max(0, t - eta);
+    const int NK = a.update_first ? 0 : fill_kp(rg0, rlo0);
     umma::cp_async_wait<0>();
     __syncthreads();
 
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
 
     // ---- read: scores (a quad per key), softmax per head, P V (lane owns columns) ----
     // Eq. 14 over the NK keys of kp and, unless hidden, the state (H, s) in shared memory
-    auto read_phase = [&](const int NK) {
+    auto read_phase = [&](const int NK, const int rg, const int rlo) {
         constexpr int KQ = DIM / 4;                                  // key elements per quad lane
         const int q4 = lane & 3, rq = lane >> 2;                     // lane in quad, quad in warp
         const float scale = 1.0f / sqrtf((float)DIM);
@@ -224,6 +225,27 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
             }
         }
         __syncthreads();
+        if (a.scorer) {
+            // alternative rules: the query credits every window key it reads, and itself
+            for (int i = rg + warp; i < NK; i += NW) {
+                const bool self = i == NK - 1;
+                const size_t ws = wbase + (size_t)((self ? t : rlo + i - rg) % eta);
+                const float* pk = self ? phk : a.sp.win_phik + ws * D;
+                float term = 0.f;
+                for (int hh = 0; hh < Gq; ++hh) {
+                    float f = 0.f;
+                    for (int j = lane; j < D; j += 32) f = fmaf(phq[hh * D + j], pk[j], f);
+                    f = warp_sum(f);
+                    term += window_term(a.scorer, expf(sc[hh * NK + i]), f);
+                }
+                if (lane == 0) {
+                    if (!self) a.sp.win_sc[ws] += term;
+                    else if (a.update_first) a.sp.win_sc[ws] = term;   // the ring slot is already the token's
+                    else red[48] = term;                                 // stored with the token after the update
+                }
+            }
+            __syncthreads();
+        }
         for (int hh = warp; hh < Gq; hh += NW) {
             float mx = -INFINITY;
             for (int i = lane; i < NK; i += 32) mx = fmaxf(mx, sc[hh * NK + i]);
@@ -292,20 +314,22 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
         if (leaving) {
             const size_t wsl = wbase + rs;
             const TIn* vl = (const TIn*)a.sp.win_v + wsl * DIM;
-            // P_l = H^T phi_l, den_l = phi_l . s, R_l = P_l - den_l v_l (pre-fold state)
-            for (int cc = tid; cc < DIM; cc += NT) {
-                float x = 0.f;
-                for (int j = 0; j < D; ++j) x = fmaf(phl[j], Hs[j * DIM + cc], x);
-                Pl[cc] = x;
-            }
-            if (warp == 0) {
-                float x = 0.f;
-                for (int j = lane; j < D; j += 32) x = fmaf(phl[j], ss[j], x);
-                x = warp_sum(x);
-                if (lane == 0) red[32] = x;
+            // P_l = H^T phi_l, den_l = phi_l . s, R_l = P_l - den_l v_l (pre-fold state; SRE only)
+            if (!a.scorer) {
+                for (int cc = tid; cc < DIM; cc += NT) {
+                    float x = 0.f;
+                    for (int j = 0; j < D; ++j) x = fmaf(phl[j], Hs[j * DIM + cc], x);
+                    Pl[cc] = x;
+                }
+                if (warp == 0) {
+                    float x = 0.f;
+                    for (int j = lane; j < D; j += 32) x = fmaf(phl[j], ss[j], x);
+                    x = warp_sum(x);
+                    if (lane == 0) red[32] = x;
+                }
             }
             __syncthreads();
-            const float den_l = red[32];
+            const float den_l = a.scorer ? 0.f : red[32];
             float* Rg = a.sp.cache_R + cbase * DIM;
             float* deng = a.sp.cache_den + cbase;
             if (n_g < lam) {
@@ -314,11 +338,15 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                 for (int i = tid; i < DIM; i += NT) {
                     ((TIn*)a.sp.cache_k)[cs * DIM + i] = ((const TIn*)a.sp.win_k)[wsl * DIM + i];
                     ((TIn*)a.sp.cache_v)[cs * DIM + i] = vl[i];
-                    Rg[(size_t)n_g * DIM + i] = Pl[i] - den_l * to_f32(vl[i]);
+                    if (!a.scorer) Rg[(size_t)n_g * DIM + i] = Pl[i] - den_l * to_f32(vl[i]);
                 }
                 for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
-                if (tid == 0) { a.sp.cache_pos[cs] = lpos; deng[n_g] = den_l; }
-                if (warp == 0) {                                          // its SRE against the state
+                if (tid == 0) {
+                    a.sp.cache_pos[cs] = lpos;
+                    if (a.scorer) a.sp.cache_sc[cs] = a.sp.win_sc[wsl];        // its frozen window score
+                    else deng[n_g] = den_l;
+                }
+                if (!a.scorer && warp == 0) {                             // its SRE against the state
                     float q = 0.f, vq = 0.f;
                     for (int cc = lane; cc < DIM; cc += 32) {
                         const float v = to_f32(vl[cc]);
@@ -334,7 +362,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                 // scores: members from the cache (stored when their residuals last changed), l from R_l
                 float* scs = red + 64;                                    // reuse as scratch for the argmin
                 for (int e = tid; e < lam; e += NT) sc[e] = a.sp.cache_sc[cbase + e];
-                if (warp == 0) {
+                if (a.scorer) {
+                    if (tid == 0) sc[lam] = a.sp.win_sc[wsl];             // l's window score is complete
+                } else if (warp == 0) {
                     float q = 0.f, vq = 0.f;
                     for (int cc = lane; cc < DIM; cc += 32) {
                         const float v = to_f32(vl[cc]);
@@ -376,9 +406,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                 // fold (Eqs. 12-13): H += phi_f v_f^T, s += phi_f
                 for (int i = tid; i < D * DIM; i += NT) Hs[i] = fmaf(phf[i / DIM], vf[i % DIM], Hs[i]);
                 for (int i = tid; i < D; i += NT) ss[i] += phf[i];
-                // residuals of every remaining member follow the rank-1 change
+                // residuals of every remaining member follow the rank-1 change (SRE only)
                 // a quad per member: k_e = phi_e . phi_f, R_e += k_e (v_f - v_e), den_e += k_e
-                {
+                if (!a.scorer) {
                     constexpr int PQ = D / 4, RQ = DIM / 4;
                     const int q4 = lane & 3, rq = lane >> 2;
                     for (int e0 = warp * 8; e0 <= lam; e0 += NW * 8) {
@@ -438,7 +468,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                         ((TIn*)a.sp.cache_v)[cs * DIM + i] = vl[i];
                     }
                     for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
-                    if (tid == 0) a.sp.cache_pos[cs] = lpos;
+                    if (tid == 0) {
+                        a.sp.cache_pos[cs] = lpos;
+                        if (a.scorer) a.sp.cache_sc[cs] = sc[lam];
+                    }
                 }
                 __syncthreads();
                 for (int i = tid; i < D * DIM / 4; i += NT)
@@ -455,20 +488,22 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                 ((TIn*)a.sp.win_v)[ws * DIM + i] = vg[i];
             }
             for (int i = tid; i < D; i += NT) a.sp.win_phik[ws * D + i] = phk[i];
+            if (a.scorer && !a.update_first && tid == 0) a.sp.win_sc[ws] = red[48];
         }
     };
 
     if (!a.update_first) {
-        read_phase(NK);
+        read_phase(NK, rg0, rlo0);
         update_phase();
     } else {
         // the token equations read literally: update, then read the new memories
         // (cache slots [0, min(lambda, t + 1 - eta)), window [t + 1 - eta, t), the token)
         update_phase();
         __syncthreads();
-        const int nk = fill_kp(hide_sparse ? 0 : min(lam, max(0, t + 1 - eta)), max(0, t + 1 - eta));
+        const int rg1 = hide_sparse ? 0 : min(lam, max(0, t + 1 - eta)), rlo1 = max(0, t + 1 - eta);
+        const int nk = fill_kp(rg1, rlo1);
         __syncthreads();
-        read_phase(nk);
+        read_phase(nk, rg1, rlo1);
     }
 }
 

@@ -42,6 +42,18 @@ __device__ __forceinline__ unsigned long long f2fma(unsigned long long a, unsign
     return d;
 }
 
+// One query's term of an alternative scoring rule (LoLA notes §4.5, Table 4;
+// App. F): a = exp(q.k / sqrt(d)), f = phi(q)^T phi(k).
+// rule 1: (a - f)^2, 2: |a - f|, 3: f / a, 4: a.
+__device__ __forceinline__ float window_term(int rule, float a, float f) {
+    switch (rule) {
+        case 1: { const float x = a - f; return x * x; }
+        case 2: return fabsf(a - f);
+        case 3: return f / a;
+        default: return a;
+    }
+}
+
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

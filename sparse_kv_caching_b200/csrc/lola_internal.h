@@ -25,8 +25,9 @@ namespace lola {
 constexpr int kThreads = 512;
 
 struct Layout {            // byte offsets inside dev_buf (all 256-aligned)
-    size_t W, H, s, cache_k, cache_v, cache_phik, cache_pos, win_k, win_v, win_phik, cache_R, cache_den, cache_sc;
-    size_t phik_new, snap_pos, snap_H, snap_s, io_q, io_k, io_v, io_y, err;
+    size_t W, H, s, cache_k, cache_v, cache_phik, cache_pos, win_k, win_v, win_phik, cache_R, cache_den, cache_sc,
+        win_sc;
+    size_t phik_new, key_sc, snap_pos, snap_H, snap_s, io_q, io_k, io_v, io_y, err;
     size_t total;
 };
 
@@ -49,7 +50,9 @@ struct StatePtrs {
     float* win_phik;
     float* cache_R;        // [S][lambda][d]  H^T phi_e - den_e v_e (kept by decode)
     float* cache_den;      // [S][lambda]     phi_e . s
-    float* cache_sc;       // [S][lambda]     SRE of each member against the current (H, s)
+    float* cache_sc;       // [S][lambda]     each member's score: SRE against the current (H, s),
+                           //                 or its frozen window score under an alternative rule
+    float* win_sc;         // [S][eta]        window score accumulated so far (alternative rules; ring slot p % eta)
 };
 
 struct PrefillArgs {
@@ -64,6 +67,8 @@ struct PrefillArgs {
     int nc;                // chunks in this call
     int c_begin, c_end;    // chunks [c_begin, c_end) of the call served by this launch (scan, output)
     int read_mask;         // bit 0: queries do not read (H, s); bit 1: nor the sparse cache
+    int scorer;            // 0 SRE; 1..4 the alternative rules (window scores, see scores.cu)
+    float* key_sc;         // [S][eta + max_tokens] window scores of positions t_start - eta + i
     float* phik_new;       // [S][max_tokens][D]
     int* snap_pos;         // [S][nc_max+1][lambda]
     float* snap_H;         // [S][nc_max+1][d][D] (H_c transposed)
@@ -81,6 +86,7 @@ struct DecodeArgs {
     int t;                 // position of the new token
     int read_mask;         // as PrefillArgs::read_mask
     int update_first;      // 1: update the memories, then read them (token equations read literally)
+    int scorer;            // as PrefillArgs::scorer
     int* err;              // device error word
 };
 
@@ -108,6 +114,8 @@ cudaError_t launch_output_tc(const PrefillArgs& a, cudaStream_t s);   // bf16 on
 cudaError_t launch_finalize(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_sre_map(const SreMapArgs& a, cudaStream_t s);
+cudaError_t launch_key_scores(const PrefillArgs& a, cudaStream_t s);       // alternative rules: window scores
+cudaError_t launch_finalize_scores(const PrefillArgs& a, cudaStream_t s);  // ... kept for later calls
 cudaError_t launch_residual_init(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_clear(const Dims& dm, const StatePtrs& sp, cudaStream_t s);
 

@@ -16,7 +16,10 @@
 // score bits with exact ties broken towards the older position; slot
 // bookkeeping by block scans (kept incumbents stay in their slots, kept
 // newcomers fill the freed slots in slot order); the fold H += Phi_S^T V_S,
-// s += sum Phi_S with H held in registers.
+// s += sum Phi_S with H held in registers.  Under an alternative scoring rule
+// (notes §4.5, Table 4) the scores do not depend on the state: they come from
+// the window-score kernel (scores.cu) and the one-CTA chain only selects and
+// folds.
 #include <cooperative_groups.h>
 #include <type_traits>
 
@@ -62,6 +65,16 @@ __device__ __forceinline__ const int* entering_slots(const PrefillArgs& a, int s
     const Dims& dm = a.dm;
     return a.c_begin == 0 ? a.sp.cache_pos + (size_t)st * dm.lam
                           : a.snap_pos + ((size_t)st * (dm.nc_max + 1) + a.c_begin) * dm.lam;
+}
+
+// Score of candidate position p (held in cache slot `slot` if it was cached before
+// the call) under an alternative rule: its window score, computed for this call's
+// positions and the window entering it, else the frozen score kept with its slot.
+__device__ __forceinline__ float static_score(const PrefillArgs& a, int st, int p, int slot) {
+    const Dims& dm = a.dm;
+    if (p >= a.t_start - dm.eta)
+        return a.key_sc[(size_t)st * (dm.eta + dm.max_tokens) + (size_t)(p - a.t_start + dm.eta)];
+    return a.sp.cache_sc[(size_t)st * dm.lam + slot];
 }
 
 // keep[i] = 1 for the lam candidates with the largest (score, -position);
@@ -196,7 +209,11 @@ __global__ void __launch_bounds__(kThreads, 1) scan_kernel(PrefillArgs a) {
             for (int i = tid; i < n; i += kThreads) cand_pos[i] = i < n_g ? slot_pos[i] : l_lo + (i - n_g);
             __syncthreads();
             auto ref = [&](int e) { return pair_ref<TIn>(a, st, b, g, cand_pos[e], e); };
-            if (lam > 0) {
+            if (lam > 0 && a.scorer != 0) {
+                for (int e = tid; e < n; e += kThreads) score[e] = static_score(a, st, cand_pos[e], e);
+                __syncthreads();
+                select_top(score, cand_pos, n, lam, keep, sbits, hist, tmp, eq_list);
+            } else if (lam > 0) {
                 for (int e0 = 0; e0 < n; e0 += Sh::TE) {
                     const int ne = min(Sh::TE, n - e0);
                     load_phi_tile<D>(tile, ne, [&](int e) { return ref(e0 + e).phik; });
@@ -1320,6 +1337,9 @@ static cudaError_t launch_scan_cg_d(const PrefillArgs& a, int ncl, cudaStream_t 
 static int g_num_sms = 0;
 
 cudaError_t launch_scan(const PrefillArgs& a, cudaStream_t s) {
+    // alternative rules rank by precomputed window scores: one CTA per stream folds
+    if (a.scorer != 0)
+        return a.dm.dtype == 1 ? launch_scan_d<__nv_bfloat16>(a, s) : launch_scan_d<float>(a, s);
     if (g_num_sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);

@@ -1,10 +1,13 @@
-"""Parity of the read options and the SRE map (through the C ABI) with the CPU oracle.
+"""Parity of the read options, the scoring rules and the SRE map (through the C ABI)
+with the CPU oracle.
 
 Read-branch masks (LoLA notes §4.8, App. I, Table 12) on the prefill output
 kernels (bf16 tensor-core path and fp32 path) and on decode; update-first
-decode (the token equations of notes §2.4 read literally); the stored-pair SRE
-map and relative SRE (notes §4.4, Fig. 3, Fig. 10, Eq. 26) over the
-prefill's snapshots.  Every output element of the small cases is compared.
+decode (the token equations of notes §2.4 read literally); the alternative
+scoring rules of the scoring ablation (notes §4.5, Table 4; App. F) in
+prefill, across calls and in decode; the stored-pair SRE map and relative SRE
+(notes §4.4, Fig. 3, Fig. 10, Eq. 26) over the prefill's snapshots.  Every
+output element of the small cases is compared.
 """
 import numpy as np
 import pytest
@@ -37,10 +40,11 @@ def _prefill(w, layer, dev, cuts):
     return torch.cat(ys, dim=1), traces
 
 
-def _oracle_follow(w, b, g, cuts, traces, yg, mask=0):
+def _oracle_follow(w, b, g, cuts, traces, yg, mask=0, scorer="sre"):
     """Oracle stream for (b, g) stepped through the library's chunks and cache trace."""
     st = P.oracle_stream(w, g)
     st.read_mask = mask
+    st.scorer = scorer
     a = synth.stream_arrays(w, b, g)
     err = 0.0
     for ci, (t_lo, t_hi) in enumerate(zip(cuts[:-1], cuts[1:])):
@@ -81,21 +85,24 @@ def test_read_mask_prefill(case, mask):
     assert worst <= P.TOL[w.dtype], worst
 
 
-def _decode_variant(w, T_pre, steps, streams, mask, update_first):
+def _decode_variant(w, T_pre, steps, streams, mask, update_first, scorer="sre", cuts=None):
     dev = P.to_device(w, synth.full_arrays(w))
     layer = P.make_layer(w, dev["W"], max_tokens=max(T_pre, w.chunk))
     layer.set_read_options(mask, update_first)
+    layer.set_scorer(scorer)
     oracles = {}
     if T_pre:
-        y0, traces = _prefill(w, layer, dev, [0, T_pre])
+        cuts = cuts or [0, T_pre]
+        y0, traces = _prefill(w, layer, dev, cuts)
         for (b, g) in streams:
-            st, a, e = _oracle_follow(w, b, g, [0, T_pre], traces, P.gpu_stream_y(y0, w, b, g), mask)
+            st, a, e = _oracle_follow(w, b, g, cuts, traces, P.gpu_stream_y(y0, w, b, g), mask, scorer)
             assert e <= P.TOL[w.dtype]
             oracles[(b, g)] = (st, a)
     else:
         for (b, g) in streams:
             st = P.oracle_stream(w, g)
             st.read_mask = mask
+            st.scorer = scorer
             oracles[(b, g)] = (st, synth.stream_arrays(w, b, g))
     worst, ties = 0.0, 0
     for i in range(steps):
@@ -133,6 +140,67 @@ def test_update_first_decode_from_empty_state(mask):
     """Window filling, cache filling, then scoring, every step updating before the read."""
     w = P.small_workload(1, T=64, eta=16, lam=12, chunk=64, decode_steps=160)
     _decode_variant(w, 0, 160, [(0, 0)], mask, True)
+
+
+SCORE_CASES = {
+    # GQA 4, several key tiles; two calls so window scores carry across calls
+    "bf16-d128": (dict(base=2, B=1, Hkv=2, Hq=8, T=768, eta=128, lam=96, chunk=64), [320]),
+    # chunk 48, eta not a multiple of it, Gq = 2, fp32
+    "f32-d64": (dict(base=5, B=1, Hkv=2, Hq=4, T=480, eta=72, lam=80, chunk=48, dtype="f32"), None),
+}
+
+
+@pytest.mark.parametrize("rule", ["kernel_sq", "kernel_abs", "kernel_ratio", "attn"])
+@pytest.mark.parametrize("case", list(SCORE_CASES))
+def test_alternative_scorer_prefill(case, rule):
+    kw, splits = SCORE_CASES[case]
+    kw = dict(kw)
+    w = P.small_workload(kw.pop("base"), **kw)
+    cuts = [0] + (splits or []) + [w.T]
+    dev = P.to_device(w, synth.full_arrays(w))
+    layer = P.make_layer(w, dev["W"], max_tokens=max(b - a for a, b in zip(cuts[:-1], cuts[1:])))
+    layer.set_scorer(rule)
+    y, traces = _prefill(w, layer, dev, cuts)
+    ex = layer.export()
+    worst = 0.0
+    for b in range(w.B):
+        for g in range(w.Hkv):
+            st, _, e = _oracle_follow(w, b, g, cuts, traces, P.gpu_stream_y(y, w, b, g), 0, rule)
+            worst = max(worst, e)
+            S = b * w.Hkv + g
+            assert sorted(int(p) for p in ex["cache_pos"][S].cpu().numpy() if p >= 0) == sorted(st.cache)
+            if st.folded:
+                assert P.max_rel(ex["H"][S].double().cpu().numpy(), st.H) <= P.TOL[w.dtype]
+    assert worst <= P.TOL[w.dtype], worst
+
+
+@pytest.mark.parametrize("rule,update_first", [("kernel_sq", False), ("kernel_ratio", True), ("attn", False),
+                                               ("kernel_abs", True)])
+def test_alternative_scorer_decode_after_prefill(rule, update_first):
+    w = P.small_workload(4, B=2, Hkv=2, Hq=8, T=512, eta=64, lam=48, chunk=64, decode_steps=80)
+    _decode_variant(w, 512, 80, [(0, 0), (1, 1)], 0, update_first, rule, cuts=[0, 192, 512])
+
+
+@pytest.mark.parametrize("rule", ["kernel_sq", "attn"])
+def test_alternative_scorer_decode_from_empty_state(rule):
+    w = P.small_workload(1, T=64, eta=16, lam=12, chunk=64, decode_steps=120)
+    _decode_variant(w, 0, 120, [(0, 0)], 0, False, rule)
+
+
+def test_scorer_change_after_tokens_is_an_error():
+    import sparse_kv_caching_b200 as lola
+    w = P.small_workload(2, B=1, Hkv=2, Hq=4, T=128, eta=64, lam=64, chunk=64)
+    dev = P.to_device(w, synth.full_arrays(w))
+    layer = P.make_layer(w, dev["W"])
+    with pytest.raises(lola.LolaError, match="INVALID_ARG"):
+        layer.set_scorer(7)
+    layer.set_scorer("attn")
+    layer.prefill(dev["q"], dev["k"], dev["v"])
+    with pytest.raises(lola.LolaError, match="INVALID_ARG"):
+        layer.set_scorer("sre")
+    layer.reset()
+    layer.set_scorer("sre")
+    torch.cuda.synchronize()
 
 
 def _check_map(w, cuts):
