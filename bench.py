@@ -88,6 +88,17 @@ def sre_map_work(w: synth.Workload) -> tuple[int, int]:
     return pairs, pairs * (2 * w.D * w.d + 2 * w.D + 3 * w.d)
 
 
+def scorer_work(w: synth.Workload) -> int:
+    """FLOPs of one window-score launch (alternative rules) over a prefill of w.T tokens
+    from position 0: every (key, query, head) credit costs q.k (2 d), phi(q).phi(k) (2 D)
+    and the rule's term (3); every query row's feature map costs 2 d Dh once."""
+    credits = 0
+    for i in range(w.T):
+        credits += min(w.T, ((i + w.eta) // w.chunk + 1) * w.chunk) - i
+    S = w.B * w.Hkv
+    return S * (credits * w.Gq * (2 * w.d + 2 * w.D + 3) + w.T * w.Gq * 2 * w.d * w.Dh)
+
+
 def decode_step_bytes(w: synth.Workload) -> int:
     """HBM bytes one decode step must move (all streams, steady state)."""
     e = 2 if w.dtype == "bf16" else 4
@@ -143,7 +154,8 @@ def load_peaks():
 
 # Sources a kernel class's counters depend on: its own files plus the shared headers.
 KERNEL_SOURCES = {"phi": ["phi.cu"], "scan": ["scan.cu"], "output": ["output_tc.cu", "output.cu"],
-                  "finalize": ["finalize.cu"], "decode": ["decode.cu"], "sre_map": ["sre_map.cu"]}
+                  "finalize": ["finalize.cu"], "decode": ["decode.cu"], "sre_map": ["sre_map.cu"],
+                  "scores": ["scores.cu"]}
 SHARED_SOURCES = ["device_common.cuh", "lola_internal.h", "umma.cuh"]
 
 
@@ -555,6 +567,39 @@ def main():
     ex = layer.export()
     trace = ex["trace_pos"].cpu().numpy() if w.lam > 0 else None
     y_host = y.cpu()
+    # ---- the same prefill under each alternative scoring rule (one CTA chain per stream) ----
+    scorer_lines = {}
+    for rule in lola.SCORERS[1:]:
+        layer.reset()
+        layer.set_scorer(rule)
+        for _ in range(2):
+            layer.reset()
+            layer.prefill(q, k, v, y)
+        layer.profile(True)
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        sc_ms = 0.0
+        for _ in range(3):
+            flush.zero_()
+            ev0.record(stream)
+            layer.reset()
+            layer.prefill(q, k, v, y)
+            ev1.record(stream)
+            ev1.synchronize()
+            sc_ms += ev0.elapsed_time(ev1)
+        ps = layer.profile_read()
+        layer.profile(False)
+        ks_ms = ps["scores"][0] / max(1, ps["scores"][1])
+        ks_fl = scorer_work(w)
+        scorer_lines[rule] = {"ms_per_step": sc_ms / 3, "tokens_per_s": w.B * w.T / (sc_ms / 3 / 1e3),
+                              "window_score_ms": ks_ms, "chain_ms": ps["scan"][0] / max(1, ps["scan"][1]),
+                              "window_score_roofline": {"bound": "alu", "achieved": ks_fl / (ks_ms / 1e3) / 1e12,
+                                                        "peak": alu, "unit": "TFLOP/s",
+                                                        "frac": ks_fl / (ks_ms / 1e3) / 1e12 / alu,
+                                                        "flops_per_launch": ks_fl,
+                                                        "traffic": traffic_for("scores", w.name)}}
+    layer.reset()
+    layer.set_scorer("sre")
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -572,6 +617,7 @@ def main():
             "e2e": {"value": job_throughput(w.B * w.T, world, e2e_ms), "unit": "tokens/s", "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "sre_map": sre_map_line,
+            "scorers": scorer_lines,
             }
     del layer, full, q, k, v, y, hq, hk, hv, hy
     torch.cuda.empty_cache()

@@ -226,12 +226,13 @@ int lola_sre_map(lola_state* st, const void* k, const void* v, int T, float* sre
 int lola_state_export(const lola_state* st, lola_state_view* out);
 
 /* Tracing aid.  Kernel classes, in this order: 0 feature map, 1 scan (memory
- * update chain), 2 output, 3 finalize, 4 decode, 5 SRE map.  While enabled, every kernel
+ * update chain), 2 output, 3 finalize, 4 decode, 5 SRE map, 6 window scores of
+ * an alternative scoring rule.  While enabled, every kernel
  * launch of `st` is bracketed by CUDA events recorded on its stream.
  * lola_profile_read waits for those events, adds their elapsed times (ms) and
- * launch counts into ms[0..5] and launches[0..5] (n >= 6 entries each) and
+ * launch counts into ms[0..6] and launches[0..6] (n >= 7 entries each) and
  * forgets them.  Enabling does not change what the kernels compute. */
-#define LOLA_KERNEL_CLASSES 6
+#define LOLA_KERNEL_CLASSES 7
 int lola_profile_enable(lola_state* st, int on);
 int lola_profile_read(lola_state* st, float* ms, long long* launches, int n);
 

@@ -27,7 +27,7 @@ EXPORTS = ("lola_state_bytes", "lola_state_init", "lola_state_reset", "lola_stat
            "lola_decode_step_host", "lola_state_export", "lola_profile_enable",
            "lola_profile_read", "lola_launch_count", "lola_prefill_once_noalloc", "lola_selftest_umma",
            "lola_set_read_options", "lola_sre_map", "lola_set_scorer", "lola_last_error_string")
-KERNEL_CLASSES = ("phi", "scan", "output", "finalize", "decode", "sre_map")
+KERNEL_CLASSES = ("phi", "scan", "output", "finalize", "decode", "sre_map", "scores")
 READ_HIDE_STATE, READ_HIDE_SPARSE = 1, 2
 SCORERS = ("sre", "kernel_sq", "kernel_abs", "kernel_ratio", "attn")   # LOLA_SCORE_* in this order
 

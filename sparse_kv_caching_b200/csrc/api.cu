@@ -407,7 +407,7 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
         // not the state), then the chain ranks by those scores, then the output.
         if ((e = traced(st, 0, 1, s, [&] { return lola::launch_phi_keys(a, s); })) != cudaSuccess)
             return cuda_fail(e, "feature-map kernel");
-        if ((e = traced(st, 1, 1, s, [&] { return lola::launch_key_scores(a, s); })) != cudaSuccess)
+        if ((e = traced(st, 6, 1, s, [&] { return lola::launch_key_scores(a, s); })) != cudaSuccess)
             return cuda_fail(e, "window-score kernel");
         if ((e = traced(st, 1, 1, s, [&] { return lola::launch_scan(a, s); })) != cudaSuccess)
             return cuda_fail(e, "scan kernel");
