@@ -136,6 +136,7 @@ int lola_state_free(lola_state* st);
  * T must be a positive multiple of chunk and <= max_tokens.  Calls may split
  * a sequence at any chunk-aligned point; the result equals one call.
  * A call of >= 32 chunks runs the memory-update chain in four chunk segments
+ * (sized 2:2:2:1)
  * on an internal high-priority stream and each segment's output on an
  * internal low-priority stream, forked from and joined back into `stream`
  * with events: the call stays stream-ordered on `stream` (and can be captured

@@ -56,7 +56,13 @@ namespace {
 
 thread_local std::string g_err;
 constexpr int kSplitMinChunks = 32;   // calls with fewer chunks run in one segment
-constexpr int kSplitSegments = 4;
+// Relative chunk counts of the chain segments.  The output of segment i runs
+// beside the chain of segment i+1; only the last segment's output is exposed,
+// so the last segment is the shortest (2:2:2:1 measured 0.7 % faster than
+// four equal segments on the 8B-shaped 4096-token prefill; 1:1:1:1, 3:3:3:1,
+// 4:4:4:4:1 and 3:3:3:2:1 were tried).
+constexpr int kSegWeights[] = {2, 2, 2, 1};
+constexpr int kSplitSegments = sizeof(kSegWeights) / sizeof(kSegWeights[0]);
 constexpr int kHostSegments = 4;      // host-buffer prefill: copies overlap compute per segment
 std::atomic<long long> g_launches{0};
 
@@ -401,7 +407,19 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
     auto output = [&](cudaStream_t q) {
         return dm.dtype == LOLA_DTYPE_BF16 ? lola::launch_output_tc(a, q) : lola::launch_output(a, q);
     };
-    const int seg = a.nc >= kSplitMinChunks ? (a.nc + kSplitSegments - 1) / kSplitSegments : a.nc;
+    // chunk boundaries of the chain segments (one segment below kSplitMinChunks chunks)
+    int bounds[kSplitSegments + 1] = {0};
+    int nseg = 1;
+    bounds[1] = a.nc;
+    if (a.nc >= kSplitMinChunks) {
+        int wsum = 0, acc = 0;
+        for (int w : kSegWeights) wsum += w;
+        nseg = kSplitSegments;
+        for (int i = 0; i < nseg; ++i) {
+            acc += kSegWeights[i];
+            bounds[i + 1] = (int)(((long long)a.nc * acc + wsum - 1) / wsum);
+        }
+    }
     if (st->scorer != LOLA_SCORE_SRE) {
         // Alternative rules: every key's window score first (it needs the call's queries,
         // not the state), then the chain ranks by those scores, then the output.
@@ -415,27 +433,28 @@ int lola_prefill_chunked(lola_state* st, const void* q, const void* k, const voi
             return cuda_fail(e, "output kernel");
         if ((e = traced(st, 3, 1, s, [&] { return lola::launch_finalize_scores(a, s); })) != cudaSuccess)
             return cuda_fail(e, "window-score finalize kernel");
-    } else if (st->s_chain && seg < a.nc) {
+    } else if (st->s_chain && nseg > 1) {
         // The chain of segment i and the output of segment i-1 run at the same time:
         // the chain holds one cluster per stream, the output fills the other SMs.  The
         // feature map of the first segment's keys runs first; the rest of the keys
         // are mapped on the output stream while the first segment's chain runs.
-        a.c_end = seg;
+        a.c_end = bounds[1];
         if ((e = traced(st, 0, 1, s, [&] { return lola::launch_phi_keys(a, s); })) != cudaSuccess)
             return cuda_fail(e, "feature-map kernel");
         if ((e = cudaEventRecord(st->ev_fork, s)) || (e = cudaStreamWaitEvent(st->s_chain, st->ev_fork, 0)) ||
             (e = cudaStreamWaitEvent(st->s_out, st->ev_fork, 0)))
             return cuda_fail(e, "forking the prefill streams");
-        a.c_begin = seg;
+        a.c_begin = bounds[1];
         a.c_end = a.nc;
         if ((e = traced(st, 0, 1, st->s_out, [&] { return lola::launch_phi_keys(a, st->s_out); })) != cudaSuccess)
             return cuda_fail(e, "feature-map kernel");
         if ((e = cudaEventRecord(st->ev_join_out, st->s_out)))
             return cuda_fail(e, "ordering the feature map");
-        for (int c0 = 0; c0 < a.nc; c0 += seg) {
-            a.c_begin = c0;
-            a.c_end = std::min(a.nc, c0 + seg);
-            if (c0 == seg && (e = cudaStreamWaitEvent(st->s_chain, st->ev_join_out, 0)))
+        for (int i = 0; i < nseg; ++i) {
+            a.c_begin = bounds[i];
+            a.c_end = bounds[i + 1];
+            if (a.c_begin == a.c_end) continue;
+            if (i == 1 && (e = cudaStreamWaitEvent(st->s_chain, st->ev_join_out, 0)))
                 return cuda_fail(e, "ordering the feature map");
             if ((e = traced(st, 1, 1, st->s_chain, [&] { return lola::launch_scan(a, st->s_chain); })) != cudaSuccess)
                 return cuda_fail(e, "scan kernel");
