@@ -273,3 +273,77 @@ def test_sre_map_and_options_argument_errors():
     with pytest.raises(lola.LolaError, match="INVALID_ARG"):
         layer.sre_map(dev["k"][:, :257].contiguous(), dev["v"][:, :257].contiguous())    # decode followed
     torch.cuda.synchronize()
+
+
+# ---- the 8B-shaped 4096-token workload that bench.py times, on sampled streams ----
+
+def _fullsize_rows(w, rng):
+    rows = np.zeros((w.Gq, w.T), bool)
+    rows[:, rng.choice(w.T, size=96, replace=False)] = True
+    rows[:, -w.chunk:] = True
+    return rows
+
+
+def _fullsize_variant(mask=0, scorer="sre", with_map=False):
+    w = synth.workload(2)
+    dev = P.to_device(w, synth.full_arrays(w))
+    layer = P.make_layer(w, dev["W"], max_tokens=w.T)
+    layer.set_read_options(mask)
+    layer.set_scorer(scorer)
+    y = layer.prefill(dev["q"], dev["k"], dev["v"])
+    torch.cuda.synchronize()
+    ex = layer.export()
+    tr = ex["trace_pos"].cpu().numpy()
+    sre = rel = None
+    if with_map:
+        sre, rel = layer.sre_map(dev["k"], dev["v"])
+        torch.cuda.synchronize()
+    rng = np.random.default_rng(17)
+    for (b, g) in [(0, 0), (w.B - 1, w.Hkv - 1)]:
+        st = P.oracle_stream(w, g)
+        st.read_mask = mask
+        st.scorer = scorer
+        a = synth.stream_arrays(w, b, g)
+        e, chain = P.check_prefill_stream(w, st, a, 0, w.T, tr[b * w.Hkv + g], P.gpu_stream_y(y, w, b, g),
+                                          _fullsize_rows(w, rng))
+        assert chain.hard == 0 and chain.set_mismatch == 0, (b, g, chain.hard, chain.set_mismatch)
+        assert e <= P.TOL[w.dtype], (b, g, e)
+        S = b * w.Hkv + g
+        assert P.max_rel(ex["H"][S].double().cpu().numpy(), st.H) <= P.TOL[w.dtype]
+        if with_map:
+            so, ro = oracle_sre_map(st)
+            sg = sre[b, g].double().cpu().numpy()
+            rg = rel[b, g].double().cpu().numpy()
+            nfold = [r["folded_before"] for r in st.log] + [len(st.folded)]
+            M = np.zeros_like(so, dtype=bool)
+            for c, nf in enumerate(nfold):
+                M[c, st.folded[:nf]] = True
+            assert np.all(sg[~M] == 0) and np.all(rg[~M] == 0)
+            scale = np.abs(so).max()
+            assert np.abs(sg - so).max() / scale <= MAP_TOL
+            assert np.abs(rg - ro).max() / scale <= MAP_TOL
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("mask", [1, 2])
+def test_fullsize_read_mask_sampled(mask):
+    _fullsize_variant(mask=mask)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("rule", ["kernel_sq", "kernel_ratio"])
+def test_fullsize_alternative_scorer_sampled(rule):
+    _fullsize_variant(scorer=rule)
+
+
+@pytest.mark.slow
+def test_fullsize_sre_map_sampled():
+    """The map of the whole 4096-token prefill (65 state times), two streams element by element."""
+    _fullsize_variant(with_map=True)
+
+
+@pytest.mark.slow
+def test_fullsize_update_first_decode_sampled():
+    """Update-first decode after the 8B-shaped decode workload's 4096-token prefill."""
+    w = synth.workload(4)
+    _decode_variant(w, w.T, 48, [(0, 0), (w.B - 1, w.Hkv - 1)], 0, True)
