@@ -88,15 +88,6 @@ __device__ __forceinline__ void load_quarter(const __nv_bfloat16* row, int q, fl
     }
 }
 
-// Ask L2 to fetch a contiguous byte range (128-byte lines; no registers held, no
-// effect on what is computed): the rows a later phase reads arrive while the
-// earlier phases run.
-__device__ __forceinline__ void prefetch_l2_range(const void* p, size_t bytes, int tid, int nt) {
-    const char* c = static_cast<const char*>(p);
-    for (size_t off = (size_t)tid * 128; off < bytes; off += (size_t)nt * 128)
-        asm volatile("prefetch.global.L2 [%0];" ::"l"(c + off));
-}
-
 template <int DIM, int DH, typename TIn>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int D = 2 * DH, NT = kDecThreads, NW = NT / 32, CPL = DIM / 32;
@@ -142,15 +133,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     for (int i = tid; i < DIM; i += NT) { kn[i] = to_f32(kg[i]); vn[i] = to_f32(vg[i]); }
     const int n_g = min(lam, max(0, t - eta));
     const size_t cbase = (size_t)st * lam, wbase = (size_t)st * eta;
-    {   // the key and value rows any read of this step may touch: the cache slots that can
-        // be occupied after the update, and the whole window ring
-        const int ng_max = min(lam, max(0, t + 1 - eta));
-        const size_t krow = (size_t)DIM * sizeof(TIn);
-        prefetch_l2_range((const TIn*)a.sp.cache_k + cbase * DIM, ng_max * krow, tid, NT);
-        prefetch_l2_range((const TIn*)a.sp.cache_v + cbase * DIM, ng_max * krow, tid, NT);
-        prefetch_l2_range((const TIn*)a.sp.win_k + wbase * DIM, min(eta, t) * krow, tid, NT);
-        prefetch_l2_range((const TIn*)a.sp.win_v + wbase * DIM, min(eta, t) * krow, tid, NT);
-    }
     const bool hide_state = (a.read_mask & 1) != 0, hide_sparse = (a.read_mask & 2) != 0;
     // key row pointers of the read: cache slots [0, rg), window positions [rlo, t)
     // (ring slot p % eta), then the token itself; returns the key count
@@ -329,11 +311,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
 
     // ---- update (Eqs. 11-13 with one leaving pair l = t - eta) ----
     auto update_phase = [&]() {
-        if (leaving && !a.scorer && n_g == lam) {
-            // the members' phi rows and residuals, read by the rank-1 update below
-            prefetch_l2_range(a.sp.cache_phik + cbase * D, (size_t)lam * D * 4, tid, NT);
-            prefetch_l2_range(a.sp.cache_R + cbase * DIM, (size_t)lam * DIM * 4, tid, NT);
-        }
         if (leaving) {
             const size_t wsl = wbase + rs;
             const TIn* vl = (const TIn*)a.sp.win_v + wsl * DIM;
