@@ -347,3 +347,39 @@ def test_fullsize_update_first_decode_sampled():
     """Update-first decode after the 8B-shaped decode workload's 4096-token prefill."""
     w = synth.workload(4)
     _decode_variant(w, w.T, 48, [(0, 0), (w.B - 1, w.Hkv - 1)], 0, True)
+
+
+def test_scorer_host_prefill_matches_device():
+    """The pipelined host-buffer prefill (four chunk-aligned calls) carries the window
+    scores between its calls exactly as one device call does."""
+    w = P.small_workload(2, B=2, Hkv=2, Hq=4, T=640, eta=64, lam=96, chunk=64)
+    dev = P.to_device(w, synth.full_arrays(w))
+    l1 = P.make_layer(w, dev["W"])
+    l2 = P.make_layer(w, dev["W"])
+    for layer in (l1, l2):
+        layer.set_scorer("kernel_abs")
+    y1 = l1.prefill(dev["q"], dev["k"], dev["v"])
+    hq, hk, hv = (dev[x].cpu().pin_memory() for x in ("q", "k", "v"))
+    hy = torch.full(y1.shape, float("nan"), dtype=torch.float32).pin_memory()
+    l2.prefill_host(hq, hk, hv, hy)
+    torch.cuda.synchronize()
+    e1, e2 = l1.export(), l2.export()
+    assert torch.equal(e1["cache_pos"], e2["cache_pos"]) and torch.equal(e1["H"], e2["H"])
+    assert torch.allclose(hy, y1.cpu(), rtol=0, atol=1e-6 * float(y1.abs().max()))
+
+
+def test_sre_map_after_alternative_scorer():
+    """The map reads the snapshots whatever rule chose the cache."""
+    w = P.small_workload(2, B=1, Hkv=2, Hq=4, T=512, eta=64, lam=64, chunk=64)
+    dev = P.to_device(w, synth.full_arrays(w))
+    layer = P.make_layer(w, dev["W"])
+    layer.set_scorer("attn")
+    y, traces = _prefill(w, layer, dev, [0, w.T])
+    sre, rel = layer.sre_map(dev["k"], dev["v"])
+    torch.cuda.synchronize()
+    for g in range(w.Hkv):
+        st, _, e = _oracle_follow(w, 0, g, [0, w.T], traces, P.gpu_stream_y(y, w, 0, g), 0, "attn")
+        so, ro = oracle_sre_map(st)
+        scale = np.abs(so).max()
+        assert np.abs(sre[0, g].double().cpu().numpy() - so).max() / scale <= MAP_TOL
+        assert np.abs(rel[0, g].double().cpu().numpy() - ro).max() / scale <= MAP_TOL
