@@ -91,7 +91,7 @@ def window_score_terms(a: np.ndarray, f: np.ndarray, rule: str) -> np.ndarray:
 
 # ---------------------------------------------------------------------------
 # Feature map (notes §2.1 notation table: learned phi: R^{d_k} -> R^D; the
-# Hedgehog form [softmax(xW), softmax(-xW)] is the fixed choice of this build)
+# Hedgehog form [softmax(xW), softmax(-xW)] is the form fixed here)
 # ---------------------------------------------------------------------------
 def _softmax(z: np.ndarray) -> np.ndarray:
     e = np.exp(z - z.max(axis=-1, keepdims=True))
