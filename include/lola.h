@@ -218,8 +218,10 @@ int lola_set_scorer(lola_state* st, int scorer);
  * sre, rel: device float32 [B][Hkv][n + 1][T]; rel may be NULL.  The last
  * call on `st` must be a prefill (LOLA_ERR_INVALID_ARG after a decode step,
  * a reset or no prefill).  For a host-buffer prefill of >= 8 chunks "the
- * last call" is the last of its four chunk-aligned calls.  Reads the state's
- * per-chunk snapshots and changes nothing; fp32 arithmetic. */
+ * last call" is the last of its four chunk-aligned calls.  k, v, sre and rel
+ * must be 16-byte aligned (LOLA_ERR_INVALID_ARG otherwise); a failed launch
+ * returns LOLA_ERR_CUDA.  Reads the state's per-chunk snapshots and changes
+ * nothing; fp32 arithmetic, whatever scoring rule chose the cache. */
 int lola_sre_map(lola_state* st, const void* k, const void* v, int T, float* sre, float* rel,
                  void* stream);
 
