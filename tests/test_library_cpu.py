@@ -82,5 +82,8 @@ def test_null_arguments_rejected(L):
     assert L.lola_decode_step(None, None, None, None, None, None) == -1
     assert L.lola_state_export(None, None) == -1
     assert L.lola_state_free(None) == 0
+    assert L.lola_set_read_options(None, 0, 0) == -1
+    assert L.lola_set_scorer(None, 0) == -1
+    assert L.lola_sre_map(None, None, None, 64, None, None, None) == -1
     n = ctypes.c_size_t()
     assert L.lola_state_bytes(ctypes.byref(_cfg()), ctypes.byref(n)) == 0 and n.value > 0
