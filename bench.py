@@ -600,6 +600,26 @@ def main():
                                                         "traffic": traffic_for("scores", w.name)}}
     layer.reset()
     layer.set_scorer("sre")
+    # ---- the same prefill with memory branches hidden from the read (read-branch masks) ----
+    mask_lines = {}
+    for mask, label in ((1, "hide_state"), (2, "hide_sparse"), (3, "window_only")):
+        layer.set_read_options(mask)
+        for _ in range(2):
+            layer.reset()
+            layer.prefill(q, k, v, y)
+        m_ms = 0.0
+        for _ in range(3):
+            flush.zero_()
+            ev0 = torch.cuda.Event(enable_timing=True)
+            ev1 = torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            layer.reset()
+            layer.prefill(q, k, v, y)
+            ev1.record(stream)
+            ev1.synchronize()
+            m_ms += ev0.elapsed_time(ev1)
+        mask_lines[label] = {"ms_per_step": m_ms / 3, "tokens_per_s": w.B * w.T / (m_ms / 3 / 1e3)}
+    layer.set_read_options(0)
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -618,6 +638,7 @@ def main():
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "sre_map": sre_map_line,
             "scorers": scorer_lines,
+            "read_masks": mask_lines,
             }
     del layer, full, q, k, v, y, hq, hk, hv, hy
     torch.cuda.empty_cache()
@@ -660,7 +681,23 @@ def main():
                          "bytes_per_launch": by, "ms_per_launch": kms,
                          "peak_kind": f"{peaks_kind} HBM copy", "traffic": traffic_for("decode", wd.name)},
             "flops_per_step": decode_step_flops(wd)}
-        del ld, qd, kd, vd, qs, ks, vs
+        # the same sequences continued with update-first decode (the token equations read literally)
+        ld.profile(False)
+        ld.set_read_options(0, True)
+        t_uf = wd.T + args.warmup + steps_d
+        n_uf = min(50, wd.T + wd.decode_steps - t_uf)
+        quf = [(qd[:, t].contiguous(), kd[:, t].contiguous(), vd[:, t].contiguous()) for t in range(t_uf, t_uf + n_uf)]
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for qq, kk_, vv_ in quf:
+            ld.decode(qq, kk_, vv_, yd)
+        ev1.record(stream)
+        ev1.synchronize()
+        uf_ms = ranks_max(ev0.elapsed_time(ev1) / n_uf)
+        line["decode"]["update_first"] = {"ms_per_step": uf_ms, "value": wd.B * world / (uf_ms / 1e3),
+                                          "steps": n_uf}
+        del ld, qd, kd, vd, qs, ks, vs, quf
         torch.cuda.empty_cache()
 
     # ---- cpu_baseline: the oracle on a bounded sample, plus the oracle match ----
