@@ -18,8 +18,7 @@
 // newcomers fill the freed slots in slot order); the fold H += Phi_S^T V_S,
 // s += sum Phi_S with H held in registers.  Under an alternative scoring rule
 // (notes §4.5, Table 4) the scores do not depend on the state: they come from
-// the window-score kernel (scores.cu) and the one-CTA chain only selects and
-// folds.
+// the window-score kernel (scores.cu) and the chain only selects and folds.
 #include <cooperative_groups.h>
 #include <type_traits>
 
@@ -738,7 +737,11 @@ __global__ void __launch_bounds__(kClThreads, 1) scan_cl_kernel(const __grid_con
             float* mypart = part + pb * N4;
             umma::cp_async_wait<0>();                          // the newcomers have landed
             __syncthreads();
-            if (lam > 0) {
+            if (lam > 0 && a.scorer != 0) {
+                // alternative rules: the window scores, read alike by every CTA of the cluster
+                for (int e = tid; e < n; e += NT) score[e] = static_score(a, st, cand_pos[e], e);
+                __syncthreads();
+            } else if (lam > 0) {
                 sre_all(n, mypart);
                 cluster.sync();                                // partials visible cluster-wide
                 // score_e = sum of the cluster's partials, by a butterfly over NCL lanes
@@ -1337,9 +1340,6 @@ static cudaError_t launch_scan_cg_d(const PrefillArgs& a, int ncl, cudaStream_t 
 static int g_num_sms = 0;
 
 cudaError_t launch_scan(const PrefillArgs& a, cudaStream_t s) {
-    // alternative rules rank by precomputed window scores: one CTA per stream folds
-    if (a.scorer != 0)
-        return a.dm.dtype == 1 ? launch_scan_d<__nv_bfloat16>(a, s) : launch_scan_d<float>(a, s);
     if (g_num_sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
@@ -1356,7 +1356,8 @@ cudaError_t launch_scan(const PrefillArgs& a, cudaStream_t s) {
         if (e != cudaErrorNotSupported) return e;                // launched (or a real error)
     }
     // rows left in global memory: the largest cluster with whole 16-column slices
-    if (a.dm.lam + a.dm.C <= 32 * kCgKmax) {
+    // (SRE only; alternative rules take the one-CTA chain when no row pool fits)
+    if (a.scorer == 0 && a.dm.lam + a.dm.C <= 32 * kCgKmax) {
         for (int ncl = 8; ncl >= 2; ncl >>= 1) {
             const int cw = a.dm.d / ncl;
             if (cw < 16 || cw > 64 || a.dm.S * ncl > g_num_sms) continue;
