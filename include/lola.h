@@ -121,7 +121,8 @@ int lola_state_bytes(const lola_config* cfg, size_t* bytes);
 int lola_state_init(const lola_config* cfg, const void* W, void* dev_buf, size_t bytes,
                     void* stream, lola_state** out);
 
-/* Clear the memories again (t = 0) without touching W.  Enqueued on stream. */
+/* Clear the memories again (t = 0) without touching W; the read options and
+ * the scoring rule are kept.  Enqueued on stream. */
 int lola_state_reset(lola_state* st, void* stream);
 
 /* Release the host handle.  The caller still owns (and frees) dev_buf. */
@@ -130,7 +131,8 @@ int lola_state_free(lola_state* st);
 /* Chunkwise prefill (notes §2.6, Eq. 15): process T new tokens of every
  * sequence in blocks of `chunk`.  For each block, every query reads the
  * state entering the block (Eq. 14); then the window advances, the leaving
- * pairs and the cache are scored by SRE (Eq. 10), the top lambda stay
+ * pairs and the cache are scored by SRE (Eq. 10; or by the rule chosen with
+ * lola_set_scorer), the top lambda stay
  * cached (older position wins exact ties) and the rest are folded (Eqs.
  * 12-13).  q, k, v: device, layouts above; y: device float32 [B][T][Hq][d].
  * T must be a positive multiple of chunk and <= max_tokens.  Calls may split
