@@ -89,3 +89,19 @@ def test_prefill_chain_work_matches_scored_blocks():
             n, f = len(r["E"]), len(r["fold"])
             fl += 2 * n * D * d + 2 * n * D + 3 * n * d + 2 * f * D * d + f * D
         assert bench.prefill_work(w)["scan"]["flops"] == w.B * w.Hkv * fl
+
+
+def test_profile_summaries_give_runnable_commands():
+    """Every committed ncu summary names the command that made it, with the clocks
+    left alone, and runs committed files only."""
+    import glob
+    import json
+    mds = glob.glob(os.path.join(ROOT, "profiles", "*.md"))
+    assert mds
+    for p in mds:
+        txt = open(p).read()
+        assert "ncu " in txt and "--clock-control none" in txt, p
+        assert "_work" not in txt and "/root/" not in txt, p
+    traffic = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))
+    for key, ent in traffic.items():
+        assert "--clock-control none" in ent["capture"] and "_work" not in ent["capture"], key
