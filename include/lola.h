@@ -227,6 +227,16 @@ int lola_set_scorer(lola_state* st, int scorer);
 int lola_sre_map(lola_state* st, const void* k, const void* v, int T, float* sre, float* rel,
                  void* stream);
 
+/* Sync point for device-side failures: waits for `stream` (every call made
+ * on it so far) and reads the state's device error word.  Kernels never trap:
+ * a bounded wait (an mbarrier the tensor cores should complete, about 4 s of
+ * wall time) that gives up sets the word, finishes without that result and
+ * returns.  Returns LOLA_ERR_TIMEOUT if any kernel of this state has set it
+ * since the last init or reset (the outputs of those calls are not valid;
+ * lola_state_reset clears the word), LOLA_ERR_CUDA if the stream reports an
+ * error, LOLA_OK otherwise. */
+int lola_state_check(lola_state* st, void* stream);
+
 /* Fill *out with device views of the state (no copy, no synchronisation). */
 int lola_state_export(const lola_state* st, lola_state_view* out);
 
@@ -249,10 +259,15 @@ long long lola_launch_count(void);
  * the shared-memory operand layouts the kernels use, accumulating in tensor
  * memory.  mode bit 0: B given MN-major as [K][N] (else K-major as [N][K]);
  * bit 1: f32 inputs computed as tf32 (else bf16 inputs); bit 2 (with bit 1):
- * 3xTF32 split products.  A, B, C, err are device pointers (C f32 row-major,
- * *err set to 1 if the MMA completion wait gave up).  Requires M = 128,
- * 16 <= N <= 256 with N % 16 == 0, K a multiple of 16 (bf16) or 8 (tf32), and
- * operands that fit in shared memory. */
+ * 3xTF32 split products; bit 3 (with bit 1): A given MN-major as [K][M] (else
+ * [M][K]); bit 4 (with bit 1, not with bit 3): A read from tensor memory;
+ * bit 5: no MMA is issued and the completion wait gives up after about 1 ms
+ * (exercises the bounded-wait failure path: *err is set to 1 and C is filled
+ * with NaN).  A, B, C, err are device pointers (C f32 row-major, *err set to
+ * 1 if the MMA completion wait gave up).  Requires M = 128, 16 <= N <= 256
+ * with N % 16 == 0, K a multiple of 16 (bf16, or A in tensor memory) or 8
+ * (tf32), operands that fit in shared memory and at most 512 tensor-memory
+ * columns (N, plus K, or 2 K for 3xTF32, with A in tensor memory). */
 int lola_selftest_umma(int mode, const void* A, const void* B, float* C, int M, int N, int K,
                        int* err, void* stream);
 

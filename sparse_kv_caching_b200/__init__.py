@@ -26,7 +26,8 @@ EXPORTS = ("lola_state_bytes", "lola_state_init", "lola_state_reset", "lola_stat
            "lola_prefill_chunked", "lola_decode_step", "lola_prefill_chunked_host",
            "lola_decode_step_host", "lola_state_export", "lola_profile_enable",
            "lola_profile_read", "lola_launch_count", "lola_prefill_once_noalloc", "lola_selftest_umma",
-           "lola_set_read_options", "lola_sre_map", "lola_set_scorer", "lola_last_error_string")
+           "lola_set_read_options", "lola_sre_map", "lola_set_scorer", "lola_state_check",
+           "lola_last_error_string")
 KERNEL_CLASSES = ("phi", "scan", "output", "finalize", "decode", "sre_map", "scores")
 READ_HIDE_STATE, READ_HIDE_SPARSE = 1, 2
 SCORERS = ("sre", "kernel_sq", "kernel_abs", "kernel_ratio", "attn")   # LOLA_SCORE_* in this order
@@ -78,6 +79,7 @@ def lib() -> ctypes.CDLL:
     L.lola_set_read_options.argtypes = [vp, c_int, c_int]
     L.lola_sre_map.argtypes = [vp, vp, vp, c_int, vp, vp, vp]
     L.lola_set_scorer.argtypes = [vp, c_int]
+    L.lola_state_check.argtypes = [vp, vp]
     L.lola_launch_count.argtypes = []
     L.lola_launch_count.restype = c_longlong
     L.lola_last_error_string.argtypes = []
@@ -273,6 +275,11 @@ class LolaLayer:
         cnt = (c_longlong * n)()
         _check(lib().lola_profile_read(self.handle, ms, cnt, n))
         return {k: (float(ms[i]), int(cnt[i])) for i, k in enumerate(KERNEL_CLASSES)}
+
+    def check(self, stream=None) -> None:
+        """Sync point: wait for the stream and raise LolaError (LOLA_ERR_TIMEOUT) if a bounded
+        device-side wait of this state gave up since the last reset."""
+        _check(lib().lola_state_check(self.handle, _stream(stream)))
 
     def reset(self, stream=None) -> None:
         _check(lib().lola_state_reset(self.handle, _stream(stream)))

@@ -16,6 +16,7 @@
 namespace lola {
 size_t decode_smem_bytes(const Dims& dm);
 size_t selftest_smem(int mode, int M, int N, int K);
+int selftest_tmem_cols(int mode, int N, int K);
 cudaError_t launch_selftest(int mode, const void* A, const void* B, float* C, int M, int N, int K, int* err,
                             cudaStream_t s);
 }
@@ -137,6 +138,7 @@ lola::Layout make_layout(const lola::Dims& dm) {
     auto take = [&](size_t n) { size_t r = off; off = (off + n + 255) & ~(size_t)255; return r; };
     const size_t S = dm.S, e = dm.esize, snaps = (size_t)dm.nc_max + 1, T = dm.max_tokens;
     L.W = take((size_t)dm.Hkv * dm.d * dm.Dh * e);
+    L.err = take(256);     // device error word: before the host-I/O staging, which one-shot calls omit
     L.H = take(S * dm.D * dm.d * 4);
     L.s = take(S * dm.D * 4);
     L.cache_k = take(S * dm.lam * dm.d * e);
@@ -159,7 +161,6 @@ lola::Layout make_layout(const lola::Dims& dm) {
     L.io_k = take((size_t)dm.B * T * dm.Hkv * dm.d * e);
     L.io_v = take((size_t)dm.B * T * dm.Hkv * dm.d * e);
     L.io_y = take((size_t)dm.B * T * dm.Hq * dm.d * 4);
-    L.err = take(256);
     L.total = off;
     return L;
 }
@@ -364,9 +365,13 @@ int lola_selftest_umma(int mode, const void* A, const void* B, float* C, int M, 
                        void* stream) {
     if (!A || !B || !C || !err) return fail(LOLA_ERR_INVALID_ARG, "null argument");
     const bool tf32 = mode & 2;
-    if (mode < 0 || mode > 7 || ((mode & 4) && !tf32)) return fail(LOLA_ERR_INVALID_ARG, "mode=%d", mode);
+    if (mode < 0 || mode > 63 || ((mode & (4 | 8 | 16)) && !tf32) || ((mode & 8) && (mode & 16)))
+        return fail(LOLA_ERR_INVALID_ARG, "mode=%d", mode);
     if (M != 128 || N < 16 || N > 256 || N % 16 || K < (tf32 ? 8 : 16) || K % (tf32 ? 8 : 16))
         return fail(LOLA_ERR_INVALID_ARG, "unsupported shape M=%d N=%d K=%d", M, N, K);
+    if ((mode & 16) && K % 16) return fail(LOLA_ERR_INVALID_ARG, "A in tensor memory needs K %% 16 == 0");
+    if (lola::selftest_tmem_cols(mode, N, K) > 512)
+        return fail(LOLA_ERR_UNSUPPORTED, "accumulator and A need more than 512 tensor-memory columns");
     if (lola::selftest_smem(mode, M, N, K) > (size_t)kMaxSmem)
         return fail(LOLA_ERR_UNSUPPORTED, "operands do not fit in shared memory");
     cudaError_t e = lola::launch_selftest(mode, A, B, C, M, N, K, err, (cudaStream_t)stream);
@@ -606,6 +611,19 @@ int lola_decode_step_host(lola_state* st, const void* q, const void* k, const vo
     return LOLA_OK;
 }
 
+int lola_state_check(lola_state* st, void* stream) {
+    if (!st) return fail(LOLA_ERR_INVALID_ARG, "null state");
+    cudaStream_t s = (cudaStream_t)stream;
+    int word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, st->base + st->L.err, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (word != 0)
+        return fail(LOLA_ERR_TIMEOUT, "a bounded device-side wait gave up (error word 0x%x); the results of "
+                    "the calls since the last reset are not valid: reset the state", (unsigned)word);
+    return LOLA_OK;
+}
+
 int lola_state_export(const lola_state* st, lola_state_view* out) {
     if (!st || !out) return fail(LOLA_ERR_INVALID_ARG, "null argument");
     const lola::StatePtrs p = state_ptrs(st);
@@ -682,7 +700,11 @@ extern "C" int lola_prefill_once_noalloc(const lola_config* cfg, const void* W, 
         return fail(LOLA_ERR_INVALID_ARG, "T=%d must be a positive multiple of chunk=%d and <= max_tokens=%d",
                     T, dm.C, dm.max_tokens);
     const lola::Layout L = make_layout(dm);
-    const size_t need = L.io_q;          // state + prefill scratch; no host-I/O staging here
+    // state + prefill scratch + error word; the host-I/O staging, the only regions
+    // after io_q, is never touched by a device-buffer prefill
+    const size_t need = L.io_q;
+    if (L.err + 256 > need || L.snap_s >= need || L.key_sc >= need)
+        return fail(LOLA_ERR_CUDA, "internal layout error: a prefill region lies beyond the one-shot array's need");
     if (need > (size_t)LOLA_NOALLOC_SCRATCH_BYTES)
         return fail(LOLA_ERR_BUF_TOO_SMALL,
                     "this configuration needs %zu bytes of state and scratch; the built-in array holds %zu "

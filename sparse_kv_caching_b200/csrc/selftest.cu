@@ -3,7 +3,12 @@
 // layouts the kernels use, the accumulator in TMEM, read back by tcgen05.ld.
 // Modes: bit 0 = B is MN-major ([K][N] in global) rather than K-major
 // ([N][K]); bit 1 = tf32 operands (f32 in global) rather than bf16; bit 2 =
-// 3xTF32 (hi*hi + hi*lo + lo*hi, f32-accurate products).
+// 3xTF32 (hi*hi + hi*lo + lo*hi, f32-accurate products); bit 3 = A is
+// MN-major ([K][M] in global, tf32 only); bit 4 = A is read from tensor
+// memory (tf32 only; stored there by tcgen05.st, K-major); bit 5 = no MMA is
+// issued and the completion wait gives up after about a millisecond (the
+// bounded-wait failure path: *err is set, C is filled with NaN, the kernel
+// frees its tensor memory and returns).
 #include "device_common.cuh"
 #include "umma.cuh"
 
@@ -43,6 +48,7 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
     __shared__ uint64_t mbar;
     __shared__ uint32_t tbase;
     const bool bmn = a.mode & 1, tf32 = a.mode & 2, x3 = (a.mode & 4) && tf32;
+    const bool amn = (a.mode & 8) && tf32, ats = (a.mode & 16) && tf32, expire = a.mode & 32;
     const int M = a.M, N = a.N, K = a.K;
     const int es = tf32 ? 4 : 2;
     const size_t szA = (size_t)M * K * es, szB = (size_t)N * K * es;
@@ -54,8 +60,13 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
     if (tf32) {
         const float* A = (const float*)a.A;
         const float* B = (const float*)a.B;
-        fill_chunk_major<float>(sA, A, M, K, false, x3);
-        if (x3) fill_chunk_major<float>(sA2, A, M, K, true, false);
+        if (amn) {   // A given as [K][M]: rows = K, chunks along M
+            fill_chunk_major<float>(sA, A, K, M, false, x3);
+            if (x3) fill_chunk_major<float>(sA2, A, K, M, true, false);
+        } else if (!ats) {
+            fill_chunk_major<float>(sA, A, M, K, false, x3);
+            if (x3) fill_chunk_major<float>(sA2, A, M, K, true, false);
+        }
         if (bmn) {   // rows = K, chunks along N
             fill_chunk_major<float>(sB, B, K, N, false, x3);
             if (x3) fill_chunk_major<float>(sB2, B, K, N, true, false);
@@ -69,19 +80,43 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
         else fill_chunk_major<__nv_bfloat16>(sB, (const __nv_bfloat16*)a.B, N, K, false, false);
     }
     umma::fence_async_smem();
-    const uint32_t ncols = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+    // accumulator columns [0, N); with A in tensor memory, A (hi) at column N and A_lo after it
+    const int need_cols = N + (ats ? K * (x3 ? 2 : 1) : 0);
+    const uint32_t ncols = need_cols <= 32 ? 32 : need_cols <= 64 ? 64 : need_cols <= 128 ? 128
+                         : need_cols <= 256 ? 256 : 512;
     if (warp == 0) umma::tmem_alloc(&tbase, ncols);
     if (threadIdx.x == 0) { umma::mbar_init(&mbar, 1); umma::fence_mbar_init(); }
     umma::fence_before_sync();
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = tbase;
-    if (threadIdx.x == 0) {
-        const uint32_t id = umma::idesc(tf32 ? umma::kTF32 : umma::kBF16, M, N, false, bmn);
+    if (ats) {
+        // thread r of the 128 stores row r of A (and of A_lo) into lane r, one f32 per column
+        const float* A = (const float*)a.A;
+        const int r = threadIdx.x;
+        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+        for (int k0 = 0; k0 < K; k0 += 16) {
+            float hi[16], lo[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float x = r < M ? A[(size_t)r * K + k0 + i] : 0.f;
+                hi[i] = x3 ? umma::tf32_hi(x) : x;
+                lo[i] = x - umma::tf32_hi(x);
+            }
+            umma::tmem_st16(tmem + lane_off + N + k0, hi);
+            if (x3) umma::tmem_st16(tmem + lane_off + N + K + k0, lo);
+        }
+        umma::tmem_wait_st();
+        umma::fence_before_sync();
+        __syncthreads();
+        umma::fence_after_sync();
+    }
+    if (threadIdx.x == 0 && !expire) {
+        const uint32_t id = umma::idesc(tf32 ? umma::kTF32 : umma::kBF16, M, N, amn, bmn);
         const int kstep = tf32 ? 8 : 16;
         const uint32_t a0 = umma::smem_addr(sA), b0 = umma::smem_addr(sB);
         const uint32_t a1 = umma::smem_addr(sA2), b1 = umma::smem_addr(sB2);
-        const uint32_t lboA = M * 16, sboA = 128;
+        const uint32_t lboA = amn ? 128 : M * 16, sboA = amn ? K * 16 : 128;
         const uint32_t lboB = bmn ? 128 : N * 16, sboB = bmn ? K * 16 : 128;
         const int passes = x3 ? 3 : 1;
         uint32_t acc = 0;
@@ -89,18 +124,23 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
             const uint32_t abase = (p == 2) ? a1 : a0;   // pass 0: hi*hi, 1: hi*lo, 2: lo*hi
             const uint32_t bbase = (p == 1) ? b1 : b0;
             for (int ks = 0; ks < K / kstep; ++ks) {
-                const uint32_t aoff = ks * 2 * M * 16;
+                const uint32_t aoff = amn ? ks * kstep * 16 : ks * 2 * M * 16;
                 const uint32_t boff = bmn ? ks * kstep * 16 : ks * 2 * N * 16;
-                const uint64_t da = umma::sdesc(abase + aoff, lboA, sboA);
                 const uint64_t db = umma::sdesc(bbase + boff, lboB, sboB);
-                if (tf32) umma::mma_tf32(tmem, da, db, id, acc);
-                else umma::mma_bf16(tmem, da, db, id, acc);
+                if (ats) {
+                    const uint32_t ta = tmem + N + (p == 2 ? K : 0) + ks * kstep;
+                    umma::mma_tf32_ts(tmem, ta, db, id, acc);
+                } else {
+                    const uint64_t da = umma::sdesc(abase + aoff, lboA, sboA);
+                    if (tf32) umma::mma_tf32(tmem, da, db, id, acc);
+                    else umma::mma_bf16(tmem, da, db, id, acc);
+                }
                 acc = 1;
             }
         }
         umma::commit(&mbar);
     }
-    const bool ok = umma::mbar_wait(&mbar, 0);
+    const bool ok = umma::mbar_wait(&mbar, 0, expire ? 1000000ull : 4000000000ull);
     if (!ok && threadIdx.x == 0) atomicExch(a.err, 1);
     umma::fence_after_sync();
     const int row = 32 * (warp & 3) + (threadIdx.x & 31);
@@ -121,6 +161,11 @@ size_t selftest_smem(int mode, int M, int N, int K) {
     const size_t es = tf32 ? 4 : 2;
     size_t b = (size_t)M * K * es + (size_t)N * K * es;
     return x3 ? 2 * b : b;
+}
+
+int selftest_tmem_cols(int mode, int N, int K) {
+    const bool tf32 = mode & 2, x3 = (mode & 4) && tf32, ats = (mode & 16) && tf32;
+    return N + (ats ? K * (x3 ? 2 : 1) : 0);
 }
 
 cudaError_t launch_selftest(int mode, const void* A, const void* B, float* C, int M, int N, int K, int* err,

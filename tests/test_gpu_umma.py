@@ -1,6 +1,8 @@
 """Tensor-core building blocks (tcgen05 MMA from the library's shared-memory
 layouts, TMEM accumulators) checked through lola_selftest_umma against a
-float64 matrix product."""
+float64 matrix product, and the bounded-wait failure path: a completion wait
+that nothing will satisfy gives up, the kernel returns, and the state's sync
+point reports LOLA_ERR_TIMEOUT."""
 import ctypes
 
 import pytest
@@ -18,7 +20,7 @@ def _cuda():
     torch.cuda.set_device(0)
 
 
-def _run(mode, N, K, seed=0):
+def _run(mode, N, K, seed=0, err=None):
     g = torch.Generator(device="cpu").manual_seed(seed)
     tf32 = bool(mode & 2)
     A = torch.randn(128, K, generator=g)
@@ -26,15 +28,19 @@ def _run(mode, N, K, seed=0):
     if not tf32:
         A, B = A.bfloat16(), B.bfloat16()
     Bin = B if mode & 1 else B.t().contiguous()
-    Ad, Bd = A.cuda(), Bin.cuda()
+    Ain = A.t().contiguous() if mode & 8 else A
+    Ad, Bd = Ain.cuda(), Bin.cuda()
     C = torch.full((128, N), float("nan"), device="cuda")
-    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if err is None:
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
     L = lola.lib()
     rc = L.lola_selftest_umma(mode, ctypes.c_void_p(Ad.data_ptr()), ctypes.c_void_p(Bd.data_ptr()),
                               ctypes.c_void_p(C.data_ptr()), 128, N, K, ctypes.c_void_p(err.data_ptr()),
                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert rc == 0, L.lola_last_error_string().decode()
     torch.cuda.synchronize()
+    if mode & 32:
+        return C, err
     assert err.item() == 0
     ref = A.double() @ B.double()
     return C.double().cpu(), ref
@@ -62,3 +68,48 @@ def test_tf32(mode, N, K):
 def test_3xtf32(mode, N, K):
     C, ref = _run(mode, N, K)
     assert (C - ref).abs().max() / ref.abs().max() < 1e-5
+
+
+# tf32 with MN-major operands (B given as [K][N], A as [K][M]) and 3xTF32 on them:
+# the layouts the fold of the memory-update chain uses.
+@pytest.mark.parametrize("mode", [3, 7, 10, 14, 11, 15])
+@pytest.mark.parametrize("N,K", [(128, 64), (64, 128), (16, 8), (128, 32)])
+def test_tf32_mn_major(mode, N, K):
+    C, ref = _run(mode, N, K)
+    tol = 1e-5 if mode & 4 else 5e-3
+    assert (C - ref).abs().max() / ref.abs().max() < tol
+
+
+# A read from tensor memory (row m in lane m), B from shared memory: the SRE
+# product of the memory-update chain keeps H^T resident in tensor memory.
+@pytest.mark.parametrize("mode", [18, 22, 19, 23])
+@pytest.mark.parametrize("N,K", [(64, 128), (128, 64), (16, 16), (256, 128)])
+def test_tf32_a_in_tmem(mode, N, K):
+    C, ref = _run(mode, N, K)
+    tol = 1e-5 if mode & 4 else 5e-3
+    assert (C - ref).abs().max() / ref.abs().max() < tol
+
+
+def test_bounded_wait_gives_up_and_reports():
+    C, err = _run(2 | 32, 64, 64)
+    assert err.item() == 1
+    assert torch.isnan(C).all()
+
+
+def test_timeout_surfaces_through_the_state_sync_point():
+    """The state's error word set by a kernel whose bounded wait gave up makes
+    lola_state_check (the sync point) return LOLA_ERR_TIMEOUT; a reset clears it."""
+    import synth
+    from tests import parity as P
+    w = P.small_workload(2, B=1, Hkv=1, Hq=2, T=128, eta=64, lam=32, chunk=64)
+    dev = P.to_device(w, synth.full_arrays(w))
+    layer = P.make_layer(w, dev["W"])
+    layer.prefill(dev["q"][:, :w.T].contiguous(), dev["k"][:, :w.T].contiguous(), dev["v"][:, :w.T].contiguous())
+    layer.check()                                  # a healthy call reports nothing
+    word = layer.export()["err_word"]
+    _run(2 | 32, 64, 64, err=word)                 # a wait that gives up, writing the state's word
+    with pytest.raises(lola.LolaError, match="TIMEOUT"):
+        layer.check()
+    layer.reset()
+    layer.check()
+    layer.close()

@@ -87,3 +87,19 @@ def test_null_arguments_rejected(L):
     assert L.lola_sre_map(None, None, None, 64, None, None, None) == -1
     n = ctypes.c_size_t()
     assert L.lola_state_bytes(ctypes.byref(_cfg()), ctypes.byref(n)) == 0 and n.value > 0
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="passes fake pointers; only meaningful where no GPU can run the call")
+def test_noalloc_size_check_without_a_gpu(L):
+    """The one-shot entry point's size check runs before any CUDA call: the 8B-shaped
+    4096-token prefill with B = 1 passes it (and then fails only for want of a device),
+    the same shape with B = 2 is refused with LOLA_ERR_BUF_TOO_SMALL."""
+    import ctypes
+    buf = ctypes.create_string_buffer(64)
+    p = ctypes.c_void_p(ctypes.addressof(buf))
+    rc = L.lola_prefill_once_noalloc(ctypes.byref(_cfg()), p, p, p, p, 4096, p, None)
+    assert rc == -3, L.lola_last_error_string().decode()        # LOLA_ERR_CUDA: no device here
+    rc = L.lola_prefill_once_noalloc(ctypes.byref(_cfg(B=2)), p, p, p, p, 4096, p, None)
+    assert rc == -2
+    assert "built-in array" in L.lola_last_error_string().decode()
