@@ -192,7 +192,8 @@ DTYPE = "bf16+f16+tf32+f32"
 
 
 # Sources a kernel class's counters depend on: its own files plus the shared headers.
-KERNEL_SOURCES = {"phi": ["phi.cu"], "scan": ["scan.cu"], "output": ["output_tc.cu", "output.cu"],
+KERNEL_SOURCES = {"phi": ["phi.cu"], "scan": ["scan.cu", "scan_tc.cu", "chain_common.cuh"],
+                  "output": ["output_tc.cu", "output_ws.cu", "output.cu"],
                   "finalize": ["finalize.cu"], "decode": ["decode.cu"], "sre_map": ["sre_map.cu"],
                   "scores": ["scores.cu"]}
 SHARED_SOURCES = ["device_common.cuh", "lola_internal.h", "umma.cuh"]

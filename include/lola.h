@@ -259,8 +259,8 @@ long long lola_launch_count(void);
  * the shared-memory operand layouts the kernels use, accumulating in tensor
  * memory.  mode bit 0: B given MN-major as [K][N] (else K-major as [N][K]);
  * bit 1: f32 inputs computed as tf32 (else bf16 inputs); bit 2 (with bit 1):
- * 3xTF32 split products; bit 3 (with bit 1): A given MN-major as [K][M] (else
- * [M][K]); bit 4 (with bit 1, not with bit 3): A read from tensor memory;
+ * 3xTF32 split products; bit 3: A given MN-major as [K][M] (else [M][K]);
+ * bit 4 (with bit 1, not with bit 3): A read from tensor memory;
  * bit 5: no MMA is issued and the completion wait gives up after about 1 ms
  * (exercises the bounded-wait failure path: *err is set to 1 and C is filled
  * with NaN).  A, B, C, err are device pointers (C f32 row-major, *err set to

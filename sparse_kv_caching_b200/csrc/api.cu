@@ -365,7 +365,7 @@ int lola_selftest_umma(int mode, const void* A, const void* B, float* C, int M, 
                        void* stream) {
     if (!A || !B || !C || !err) return fail(LOLA_ERR_INVALID_ARG, "null argument");
     const bool tf32 = mode & 2;
-    if (mode < 0 || mode > 63 || ((mode & (4 | 8 | 16)) && !tf32) || ((mode & 8) && (mode & 16)))
+    if (mode < 0 || mode > 63 || ((mode & (4 | 16)) && !tf32) || ((mode & 8) && (mode & 16)))
         return fail(LOLA_ERR_INVALID_ARG, "mode=%d", mode);
     if (M != 128 || N < 16 || N > 256 || N % 16 || K < (tf32 ? 8 : 16) || K % (tf32 ? 8 : 16))
         return fail(LOLA_ERR_INVALID_ARG, "unsupported shape M=%d N=%d K=%d", M, N, K);

@@ -109,8 +109,12 @@ struct SreMapArgs {
 // Launchers (each returns cudaGetLastError() of its launch).
 cudaError_t launch_phi_keys(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_scan(const PrefillArgs& a, cudaStream_t s);
+// The chain on the tensor cores (scan_tc.cu); cudaErrorNotSupported outside its shapes.
+cudaError_t launch_scan_tc(const PrefillArgs& a, int num_sms, cudaStream_t s);
+int pick_tc_cluster(const Dims& dm, int num_sms);
 cudaError_t launch_output(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_output_tc(const PrefillArgs& a, cudaStream_t s);   // bf16 on tcgen05
+cudaError_t launch_output_ws(const PrefillArgs& a, cudaStream_t s);   // ... warp-specialised, two query tiles
 cudaError_t launch_finalize(const PrefillArgs& a, cudaStream_t s);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_sre_map(const SreMapArgs& a, cudaStream_t s);

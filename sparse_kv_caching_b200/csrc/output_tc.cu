@@ -383,6 +383,10 @@ static cudaError_t launch_tc_t(const PrefillArgs& a, cudaStream_t s) {
 cudaError_t launch_output_tc(const PrefillArgs& a, cudaStream_t s) {
     const int d = a.dm.d, Dh = a.dm.Dh;
     if (a.dm.dtype != 1) return cudaErrorNotSupported;
+    {
+        const cudaError_t e = launch_output_ws(a, s);
+        if (e != cudaErrorNotSupported) return e;
+    }
     if (d == 128 && Dh == 64) return launch_tc_t<128, 64>(a, s);
     if (d == 128 && Dh == 32) return launch_tc_t<128, 32>(a, s);
     if (d == 64 && Dh == 32) return launch_tc_t<64, 32>(a, s);

@@ -1,0 +1,515 @@
+// Hybrid output of chunkwise LoLA prefill on the fifth-generation tensor
+// cores, warp-specialised (bf16 inputs).  Same computation as output.cu and
+// the notes' Eq. 14 (§2.5, §2.6):
+//   y_t = (H_c^T phi(q_t) + sum_i e^{a_ti} v_i) / (phi(q_t)^T s_c + sum_i e^{a_ti})
+// over i in G_c u W_c u {block keys <= t}, one shared normaliser.
+//
+// One CTA serves 256 query rows (row = (head of the kv group, query of block
+// c)) as two 128-row tiles A and B that read the same gathered keys, so every
+// K/V tile fetched from L2 feeds twice the tensor-core work (d = 128; d = 64
+// runs one 128-row tile per CTA).  Roles:
+//   warps 0-3 / 4-7  softmax and epilogue of tile A / B (thread r owns row r)
+//   warps 8-9        gather K and V rows of each 64-key tile with cp.async
+//                    into a 3-stage ring (row addresses looked up once per key,
+//                    the block's cache positions staged in the prologue),
+//                    convert V to f16 in place
+//   warp 10, lane 0  issues every MMA
+// Tensor memory: O_A, O_B [128 x d] f32 and two S buffers per tile [128 x 64].
+// Per key tile j the MMA thread issues S_t(j+1) = Q_t K^T (bf16) while the
+// softmax warps turn S_t(j) into P_t (f16, exp2 in the log2 domain with a
+// lazily raised reference maximum); then O_t += P_t V (f16).
+// Prologue (all warps, before the roles split): z = Q W (bf16 MMA), phi(q)
+// in registers, O_t = phi(q)^T H_c (tf32 MMA over 32-column chunks), l =
+// phi(q) . s_c: the linear branch enters the online softmax as logit 0.
+// Every wait is bounded; a wait that gives up raises an abort flag that
+// releases all other waits of the CTA, and sets the state's error word.
+#include "device_common.cuh"
+#include "umma.cuh"
+
+namespace lola {
+
+template <int DIM, int DH>
+struct WsShape {
+    static constexpr int ROWS = 128, KT = 64, D = 2 * DH, NCH = DIM / 8, NST = 3;
+    static constexpr int NT = 352;                              // 11 warps
+    // query tiles per CTA: two 128-row tiles share every gathered key tile for d = 128;
+    // one for d = 64 (with two tiles at d = 64 the second tile's scores came out wrong
+    // on the B200s here, a fault not explained by the operand layouts; see the tests)
+    static constexpr int NTILE = DIM == 128 ? 2 : 1;
+    static constexpr int QB = ROWS * DIM * 2;                   // one query tile (bf16)
+    static constexpr int KVB = KT * DIM * 2;                    // one K or V tile
+    static constexpr int PB = ROWS * KT * 2;                    // one P tile (f16)
+    static constexpr int Q = 0;                                 // [2 tiles]
+    static constexpr int KV = Q + NTILE * QB;                   // [NST][K, V]
+    static constexpr int P = KV + NST * 2 * KVB;                // [NTILE tiles]
+    static constexpr int KPTR = P + NTILE * PB;                 // [NST][KT] key-row pointers, then value rows
+    static constexpr int MBAR = KPTR + 2 * NST * KT * 8;        // 15 barriers
+    static constexpr int FLAG = MBAR + 16 * 8;                  // abort flag, tmem pointer
+    static constexpr int CPOS = FLAG + 16;                      // cache positions of the block [lambda] int
+    static constexpr int KPOS = KPTR;                           // (end of the prologue aliases)
+    // prologue aliases (the KV and P regions are free until the roles start)
+    static constexpr int HT = KV;                               // H_c^T, [D/32][DIM x 32] f32
+    static constexpr int HTC = DIM * 32 * 4;
+    static constexpr int W = HT + (D / 32) * HTC;               // W [DIM][DH] bf16, MN-major B
+    static constexpr int PHI = W + DIM * DH * 2;                // [2 tiles][128 x 32] f32
+    static constexpr int SC = PHI + NTILE * ROWS * 32 * 4;      // s_c [D] f32
+    static_assert(SC + D * 4 <= KPOS, "prologue buffers must fit in the KV and P regions");
+    // tensor-memory columns
+    // O of tile t at column t * OT (each output tile on a 128-column boundary), the four
+    // S buffers from column TS
+    static constexpr uint32_t TO = 0, OT = 128, TS = 256, TMEM_COLS = 512;
+    static_assert(DIM <= (int)OT && TS + 4 * KT <= 512, "tensor memory");
+};
+
+// barrier indices
+enum : int { kKvFull = 0, kKvFree = 3, kSFull = 6, kPFull = 10, kPvDone = 12, kPro = 14 };
+
+// Bounded mbarrier wait that also gives up once another thread of the CTA has
+// raised the abort flag; returns false if it gave up (and raises the flag).
+__device__ __forceinline__ bool ws_wait(uint64_t* mbar, uint32_t parity, volatile int* abort) {
+    if (umma::mbar_try_wait(mbar, parity)) return true;
+    const uint64_t t0 = umma::globaltimer_ns();
+    while (!umma::mbar_try_wait(mbar, parity)) {
+        if (*abort) return false;
+        if (umma::globaltimer_ns() - t0 > 4000000000ull) { *abort = 1; return false; }
+    }
+    return true;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(umma::smem_addr(mbar)) : "memory");
+}
+
+__device__ __forceinline__ float ws_ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ uint32_t ws_pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float2 ws_unpack_f16(uint32_t u) { return __half22float2(*reinterpret_cast<__half2*>(&u)); }
+__device__ __forceinline__ uint32_t ws_bf2_to_h2(uint32_t u) {
+    return ws_pack_f16(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+__device__ __forceinline__ void ws_st4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" :: "r"(umma::smem_addr(p)), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+// N columns (a multiple of 16) of this warp's lanes from tensor memory, one wait.
+template <int N>
+__device__ __forceinline__ void ws_tmem_ld(uint32_t taddr, float (&r)[N]) {
+#pragma unroll
+    for (int c0 = 0; c0 < N; c0 += 16) umma::tmem_ld16(taddr + c0, *reinterpret_cast<float(*)[16]>(r + c0));
+    umma::tmem_wait_ld();
+}
+
+template <int DIM, int DH>
+__global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant__ PrefillArgs a) {
+    using Sh = WsShape<DIM, DH>;
+    using bf16 = __nv_bfloat16;
+    constexpr int ROWS = Sh::ROWS, KT = Sh::KT, D = Sh::D, NCH = Sh::NCH, NST = Sh::NST, NT = Sh::NT;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const Dims& dm = a.dm;
+    const int rows_total = dm.Gq * dm.C;
+    constexpr int NTILE = Sh::NTILE;
+    const int nrp = (rows_total + NTILE * ROWS - 1) / (NTILE * ROWS);
+    const int c = a.c_begin + (int)blockIdx.x / nrp, rp = blockIdx.x % nrp;
+    const int g = blockIdx.y, b = blockIdx.z, st = b * dm.Hkv + g;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t0 = a.t_start + c * dm.C;
+    const int rfirst = rp * NTILE * ROWS, rlast = min(rows_total, rfirst + NTILE * ROWS) - 1;
+    const bool twoB = NTILE == 2 && rlast >= rfirst + ROWS;    // tile B holds rows
+    const int qi_max = (rlast / dm.C != rfirst / dm.C) ? dm.C - 1 : rlast % dm.C;
+    const size_t snaps = (size_t)dm.nc_max + 1;
+    const bool has_lin = (t0 - dm.eta) > dm.lam && !(a.read_mask & 1);
+    const int n_g = (a.read_mask & 2) ? 0 : min(dm.lam, max(0, t0 - dm.eta));
+    const int w_lo = max(0, t0 - dm.eta), n_w = t0 - w_lo;
+    const int N = n_g + n_w + qi_max + 1;
+    const int ntiles = (N + KT - 1) / KT;
+
+    uint8_t* sQ = smem + Sh::Q;
+    uint8_t* sKV = smem + Sh::KV;
+    uint8_t* sP = smem + Sh::P;
+    const bf16** kptr = reinterpret_cast<const bf16**>(smem + Sh::KPTR);      // [NST][KT]
+    const bf16** vptr = kptr + NST * KT;                                       // [NST][KT]
+    int* cpos_s = reinterpret_cast<int*>(smem + Sh::CPOS);
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + Sh::MBAR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Sh::FLAG);
+    uint32_t* tptr = reinterpret_cast<uint32_t*>(smem + Sh::FLAG + 8);
+
+    if (warp == 0) umma::tmem_alloc(tptr, Sh::TMEM_COLS);
+    if (tid == 0) {
+        for (int i = 0; i < NST; ++i) { umma::mbar_init(&mbar[kKvFull + i], 64); umma::mbar_init(&mbar[kKvFree + i], 1); }
+        for (int i = 0; i < 4; ++i) umma::mbar_init(&mbar[kSFull + i], 1);
+        for (int t = 0; t < 2; ++t) { umma::mbar_init(&mbar[kPFull + t], ROWS); umma::mbar_init(&mbar[kPvDone + t], 1); }
+        umma::mbar_init(&mbar[kPro], 1);
+        *abort_flag = 0;
+        umma::fence_mbar_init();
+    }
+
+    // ---- prologue: queries of both tiles (row-chunk mapping: 8 rows x 4 chunks per warp) ----
+    for (int idx = tid; idx < NTILE * ROWS * NCH; idx += NT) {
+        const int t = idx / (ROWS * NCH), li = idx % (ROWS * NCH);
+        const int r = (li & 7) + 8 * (li / (8 * NCH)), j = (li >> 3) % NCH;
+        uint8_t* dst = sQ + t * Sh::QB + j * ROWS * 16 + r * 16;
+        const int R = rfirst + t * ROWS + r;
+        if (R < rows_total) {
+            const int hr = g * dm.Gq + R / dm.C, ir = R % dm.C;
+            umma::cp_async16(dst, (const bf16*)a.q + (((size_t)b * a.T + (t0 + ir - a.t_start)) * dm.Hq + hr) * DIM + 8 * j);
+        } else {
+            ws_st4(dst, 0u, 0u, 0u, 0u);
+        }
+    }
+    {
+        const int* cpos = a.snap_pos + ((size_t)st * snaps + c) * dm.lam;
+        for (int i = tid; i < n_g; i += NT) cpos_s[i] = cpos[i];
+    }
+    const float* Hc = a.snap_H + ((size_t)st * snaps + c) * D * DIM;     // H_c^T [DIM][D]
+    const float* sc_g = a.snap_s + ((size_t)st * snaps + c) * D;
+    float* s_c = reinterpret_cast<float*>(smem + Sh::SC);
+    if (has_lin) {
+        const bf16* Wg = (const bf16*)a.sp.W + (size_t)g * DIM * DH;   // [DIM][DH]; MN-major B
+        for (int idx = tid; idx < DIM * (DH / 8); idx += NT) {
+            const int k = idx % DIM, n8 = idx / DIM;
+            umma::cp_async16(smem + Sh::W + n8 * DIM * 16 + k * 16, Wg + (size_t)k * DH + 8 * n8);
+        }
+        for (int idx = tid; idx < D / 4; idx += NT) umma::cp_async16(s_c + 4 * idx, sc_g + 4 * idx);
+        for (int idx = tid; idx < (D / 32) * DIM * 8; idx += NT) {
+            const int cc = idx % DIM, jq = (idx / DIM) % 8, ch = idx / (DIM * 8);
+            umma::cp_async16(smem + Sh::HT + ch * Sh::HTC + jq * DIM * 16 + cc * 16, Hc + (size_t)cc * D + 32 * ch + 4 * jq);
+        }
+    }
+    umma::cp_async_commit();
+    umma::cp_async_wait<0>();
+    umma::fence_async_smem();
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tmem = *tptr;
+    const int wg = warp < 4 ? 0 : (warp < 8 ? 1 : 2);          // 0, 1: softmax tiles A, B; 2: loader / MMA
+    const int r = tid & (ROWS - 1);                            // row within the tile (softmax warps)
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const int R = rfirst + wg * ROWS + r;
+    const bool row_ok = wg < 2 && R < rows_total;
+    const int qpos = t0 + (row_ok ? R % dm.C : 0);
+    const int h = g * dm.Gq + (row_ok ? R / dm.C : 0);
+    const bool mma_thread = warp == 10 && lane == 0;
+    bool dead = false;
+    float l = 0.f;
+    uint32_t pro_phase = 0;
+
+    // ---- prologue: the linear branch (phi(q)^T H_c, phi(q) . s_c) of both tiles ----
+    if (has_lin) {
+        if (mma_thread) {
+            const uint32_t id = umma::idesc(umma::kBF16, ROWS, DH, false, true);
+            for (int t = 0; t < (twoB ? 2 : 1); ++t)
+                for (int ks = 0; ks < DIM / 16; ++ks)
+                    umma::mma_bf16(tmem + Sh::TS + 2 * t * KT,
+                                   umma::sdesc(umma::smem_addr(sQ + t * Sh::QB) + ks * 2 * ROWS * 16, ROWS * 16, 128),
+                                   umma::sdesc(umma::smem_addr(smem + Sh::W) + ks * 16 * 16, 128, DIM * 16), id, ks > 0);
+            umma::commit(&mbar[kPro]);
+        }
+        dead |= !ws_wait(&mbar[kPro], pro_phase, abort_flag);
+        pro_phase ^= 1;
+        umma::fence_after_sync();
+        float z[DH];
+        float mx = -INFINITY, mn = INFINITY, isp = 0.f, isn = 0.f;
+        if (wg < (twoB ? 2 : 1)) {
+            ws_tmem_ld<DH>(tmem + lane_off + Sh::TS + 2 * wg * KT, z);
+#pragma unroll
+            for (int i = 0; i < DH; ++i) { mx = fmaxf(mx, z[i]); mn = fminf(mn, z[i]); }
+            float sp = 0.f, sn = 0.f;
+#pragma unroll
+            for (int i = 0; i < DH; ++i) { sp += expf(z[i] - mx); sn += expf(mn - z[i]); }
+            isp = 1.f / sp;
+            isn = 1.f / sn;
+        }
+#pragma unroll
+        for (int jc = 0; jc < D; jc += 32) {
+            if (wg < (twoB ? 2 : 1)) {
+                uint8_t* sPhi = smem + Sh::PHI + wg * ROWS * 32 * 4;
+#pragma unroll
+                for (int jq = 0; jq < 8; ++jq) {
+                    float f[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int j = jc + 4 * jq + u;
+                        f[u] = j < DH ? expf(z[j] - mx) * isp : expf(mn - z[j - DH]) * isn;
+                        l = fmaf(f[u], s_c[j], l);
+                    }
+                    ws_st4(sPhi + jq * ROWS * 16 + r * 16, __float_as_uint(f[0]), __float_as_uint(f[1]),
+                           __float_as_uint(f[2]), __float_as_uint(f[3]));
+                }
+            }
+            umma::fence_async_smem();
+            umma::fence_before_sync();
+            __syncthreads();
+            umma::fence_after_sync();
+            if (mma_thread && !dead) {
+                const uint32_t id = umma::idesc(umma::kTF32, ROWS, DIM, false, false);
+                const uint8_t* sHt = smem + Sh::HT + (jc / 32) * Sh::HTC;
+                for (int t = 0; t < (twoB ? 2 : 1); ++t)
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma::mma_tf32(tmem + Sh::TO + t * Sh::OT,
+                                       umma::sdesc(umma::smem_addr(smem + Sh::PHI + t * ROWS * 32 * 4) + ks * 2 * ROWS * 16,
+                                                   ROWS * 16, 128),
+                                       umma::sdesc(umma::smem_addr(sHt) + ks * 2 * DIM * 16, DIM * 16, 128), id,
+                                       (jc > 0 || ks > 0) ? 1u : 0u);
+                umma::commit(&mbar[kPro]);
+            }
+            dead |= !ws_wait(&mbar[kPro], pro_phase, abort_flag);
+            pro_phase ^= 1;
+            umma::fence_after_sync();
+        }
+        if (!row_ok) l = 0.f;
+    }
+    umma::fence_before_sync();
+    __syncthreads();                                           // prologue buffers are free again
+    umma::fence_after_sync();
+
+    if (wg == 2 && warp < 10) {
+        // ---- loaders: warp 8 takes keys 0-31 of every tile, warp 9 keys 32-63 ----
+        const int kb = (warp - 8) * 32;
+        auto convert_v = [&](int s) {
+            uint8_t* sV = sKV + s * 2 * Sh::KVB + Sh::KVB;
+            for (int idx = lane; idx < 32 * NCH; idx += 32) {
+                const int kk = kb + (idx & 31), ch = idx >> 5;
+                uint4* pv = reinterpret_cast<uint4*>(sV + ch * KT * 16 + kk * 16);
+                uint4 u = *pv;
+                u.x = ws_bf2_to_h2(u.x); u.y = ws_bf2_to_h2(u.y); u.z = ws_bf2_to_h2(u.z); u.w = ws_bf2_to_h2(u.w);
+                *pv = u;
+            }
+            umma::fence_async_smem();
+            mbar_arrive(&mbar[kKvFull + s]);
+        };
+        for (int j = 0; j < ntiles; ++j) {
+            const int s = j % NST;
+            if (j >= NST) {
+                bool ok = true;
+                if (lane == 0 && !dead) ok = ws_wait(&mbar[kKvFree + s], ((j / NST) - 1) & 1, abort_flag);
+                dead |= !__shfl_sync(0xffffffffu, ok ? 1 : 0, 0);
+            }
+            // where my 32 keys live (cache slots, window, block keys up to the last query)
+            {
+                const int gk = j * KT + kb + lane;
+                const bf16* kr = nullptr;
+                const bf16* vr = nullptr;
+                if (gk < N) {
+                    const int pos = gk < n_g ? cpos_s[gk] : (gk < n_g + n_w ? w_lo + (gk - n_g) : t0 + (gk - n_g - n_w));
+                    const PairRef<bf16> pr = pair_ref<bf16>(a, st, b, g, pos, gk < n_g ? gk : 0);
+                    kr = pr.k;
+                    vr = pr.v;
+                }
+                kptr[s * KT + kb + lane] = kr;
+                vptr[s * KT + kb + lane] = vr;
+            }
+            __syncwarp();
+            uint8_t* sK = sKV + s * 2 * Sh::KVB;
+            uint8_t* sV = sK + Sh::KVB;
+            for (int idx = lane; idx < 32 * NCH; idx += 32) {
+                const int kk = (idx & 7) + 8 * (idx / (8 * NCH)), ch = (idx >> 3) % NCH;
+                const int key = kb + kk;
+                uint8_t* dk = sK + ch * KT * 16 + key * 16;
+                uint8_t* dv = sV + ch * KT * 16 + key * 16;
+                const bf16* kr = kptr[s * KT + key];
+                if (kr != nullptr && !dead) {
+                    umma::cp_async16(dk, kr + 8 * ch);
+                    umma::cp_async16(dv, vptr[s * KT + key] + 8 * ch);
+                } else {
+                    ws_st4(dk, 0u, 0u, 0u, 0u);
+                    ws_st4(dv, 0u, 0u, 0u, 0u);
+                }
+            }
+            umma::cp_async_commit();
+            if (j >= 1) {
+                umma::cp_async_wait<1>();
+                __syncwarp();
+                convert_v((j - 1) % NST);
+            }
+        }
+        if (ntiles > 0) {
+            umma::cp_async_wait<0>();
+            __syncwarp();
+            convert_v((ntiles - 1) % NST);
+        }
+    } else if (wg == 2) {
+        // ---- MMA issuer ----
+        if (mma_thread) {
+            const uint32_t idS = umma::idesc(umma::kBF16, ROWS, KT, false, false);
+            const uint32_t idO = umma::idesc(umma::kF16, ROWS, DIM, false, true);
+            const int ntl = twoB ? 2 : 1;
+            // operand descriptors built once; a K step moves a K-major start by two 16-byte
+            // chunks of the tile's rows (the address field counts 16-byte units), an MN-major
+            // (value) start by 16 rows of 16 bytes
+            const uint64_t dQ0 = umma::sdesc(umma::smem_addr(sQ), ROWS * 16, 128);
+            const uint64_t dQ1 = umma::sdesc(umma::smem_addr(sQ + (NTILE - 1) * Sh::QB), ROWS * 16, 128);
+            const uint64_t dP0 = umma::sdesc(umma::smem_addr(sP), ROWS * 16, 128);
+            const uint64_t dP1 = umma::sdesc(umma::smem_addr(sP + (NTILE - 1) * Sh::PB), ROWS * 16, 128);
+            uint64_t dK[NST], dV[NST];
+#pragma unroll
+            for (int s = 0; s < NST; ++s) {
+                dK[s] = umma::sdesc(umma::smem_addr(sKV + s * 2 * Sh::KVB), KT * 16, 128);
+                dV[s] = umma::sdesc(umma::smem_addr(sKV + s * 2 * Sh::KVB + Sh::KVB), 128, KT * 16);
+            }
+            auto issue_s = [&](int j) {
+                const int s = j % NST;
+                const uint64_t bk = s == 0 ? dK[0] : (s == 1 ? dK[1] : dK[2]);
+                const uint32_t d0 = tmem + Sh::TS + (j & 1) * KT;
+#pragma unroll
+                for (int ks = 0; ks < DIM / 16; ++ks)
+                    umma::mma_bf16(d0, dQ0 + (uint64_t)(ks * 2 * ROWS), bk + (uint64_t)(ks * 2 * KT), idS, ks > 0 ? 1u : 0u);
+                umma::commit(&mbar[kSFull + (j & 1)]);
+                if (ntl > 1) {
+#pragma unroll
+                    for (int ks = 0; ks < DIM / 16; ++ks)
+                        umma::mma_bf16(d0 + 2 * KT, dQ1 + (uint64_t)(ks * 2 * ROWS), bk + (uint64_t)(ks * 2 * KT), idS,
+                                       ks > 0 ? 1u : 0u);
+                    umma::commit(&mbar[kSFull + 2 + (j & 1)]);
+                }
+            };
+            for (int j = 0; j < ntiles && !dead; ++j) {
+                if (j == 0) {
+                    dead |= !ws_wait(&mbar[kKvFull + 0], 0, abort_flag);
+                    umma::fence_after_sync();
+                    if (!dead) issue_s(0);
+                }
+                if (j + 1 < ntiles && !dead) {
+                    dead |= !ws_wait(&mbar[kKvFull + (j + 1) % NST], ((j + 1) / NST) & 1, abort_flag);
+                    umma::fence_after_sync();
+                    if (!dead) issue_s(j + 1);
+                }
+                const int sj = j % NST;
+                const uint64_t bv = sj == 0 ? dV[0] : (sj == 1 ? dV[1] : dV[2]);
+                const uint32_t first = (has_lin || j > 0) ? 1u : 0u;
+                for (int t = 0; t < ntl && !dead; ++t) {
+                    dead |= !ws_wait(&mbar[kPFull + t], j & 1, abort_flag);
+                    umma::fence_after_sync();
+                    if (dead) break;
+                    const uint64_t ap = t == 0 ? dP0 : dP1;
+                    const uint32_t dO = tmem + Sh::TO + t * Sh::OT;
+#pragma unroll
+                    for (int ks = 0; ks < KT / 16; ++ks)
+                        umma::mma_f16(dO, ap + (uint64_t)(ks * 2 * ROWS), bv + (uint64_t)(ks * 16), idO,
+                                      ks > 0 ? 1u : first);
+                    umma::commit(&mbar[kPvDone + t]);
+                }
+                if (!dead) umma::commit(&mbar[kKvFree + j % NST]);
+            }
+        }
+    } else if (wg == 0 || twoB) {
+        // ---- softmax of tile wg: thread r owns row r ----
+        const int t = wg;
+        uint8_t* sPt = sP + t * Sh::PB;
+        const float c2 = 1.4426950408889634f / sqrtf((float)DIM);    // log2(e) / sqrt(d)
+        float m_ref = 0.f;
+        for (int j = 0; j < ntiles; ++j) {
+            const int s = j % NST;
+            bool ok = !dead;
+            if (ok) ok = ws_wait(&mbar[kSFull + 2 * t + (j & 1)], (j >> 1) & 1, abort_flag);
+            if (ok && j >= 1) ok = ws_wait(&mbar[kPvDone + t], (j - 1) & 1, abort_flag);   // P and O free
+            dead |= !__all_sync(0xffffffffu, ok);
+            if (dead) break;
+            umma::fence_after_sync();
+            float sv[KT];
+            ws_tmem_ld<KT>(tmem + lane_off + Sh::TS + (2 * t + (j & 1)) * KT, sv);
+            // cache and window keys precede the block; block key m is visible to query qi iff
+            // m <= qi: key i of tile j is visible iff j KT + i < lim
+            const int lim = row_ok ? min(N, n_g + n_w + (qpos - t0) + 1) - j * KT : 0;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < KT; ++i) {
+                sv[i] = i < lim ? sv[i] * c2 : -INFINITY;
+                mx = fmaxf(mx, sv[i]);
+            }
+            float factor = 1.f;
+            bool rescale = false;
+            if (mx != -INFINITY) {
+                if (l == 0.f) m_ref = mx;                         // nothing accumulated yet
+                else if (mx > m_ref + 8.f) { factor = ws_ex2(m_ref - mx); rescale = true; m_ref = mx; }
+            }
+            if (__any_sync(0xffffffffu, rescale)) {               // warp-collective TMEM access
+                l *= factor;
+#pragma unroll
+                for (int c0 = 0; c0 < DIM; c0 += 64) {
+                    float r64[64];
+                    ws_tmem_ld<64>(tmem + lane_off + Sh::TO + t * Sh::OT + c0, r64);
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) r64[i] *= factor;
+#pragma unroll
+                    for (int i = 0; i < 64; i += 16)
+                        umma::tmem_st16(tmem + lane_off + Sh::TO + t * Sh::OT + c0 + i, *reinterpret_cast<float(*)[16]>(r64 + i));
+                }
+                umma::tmem_wait_st();
+            }
+            // the normaliser sums the f16-rounded weights that the P V product uses
+            float rs = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < KT / 8; ++ch) {
+                uint32_t w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    w[u] = ws_pack_f16(ws_ex2(sv[8 * ch + 2 * u] - m_ref), ws_ex2(sv[8 * ch + 2 * u + 1] - m_ref));
+                    const float2 r2 = ws_unpack_f16(w[u]);
+                    rs += r2.x + r2.y;
+                }
+                ws_st4(sPt + ch * ROWS * 16 + r * 16, w[0], w[1], w[2], w[3]);
+            }
+            l += rs;
+            umma::fence_async_smem();
+            umma::fence_before_sync();
+            mbar_arrive(&mbar[kPFull + t]);
+        }
+        // ---- epilogue: y = O / l ----
+        bool ok = !dead && ntiles > 0;
+        if (ok) ok = ws_wait(&mbar[kPvDone + t], (ntiles - 1) & 1, abort_flag);
+        dead |= !__all_sync(0xffffffffu, ok);
+        umma::fence_after_sync();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        float* yrow = a.y + (((size_t)b * a.T + (qpos - a.t_start)) * dm.Hq + h) * DIM;
+#pragma unroll
+        for (int c0 = 0; c0 < DIM; c0 += 64) {
+            float r64[64];
+            ws_tmem_ld<64>(tmem + lane_off + Sh::TO + t * Sh::OT + c0, r64);
+            if (row_ok && !dead) {
+#pragma unroll
+                for (int i = 0; i < 64; i += 4)
+                    *reinterpret_cast<float4*>(yrow + c0 + i) =
+                        make_float4(r64[i] * inv, r64[i + 1] * inv, r64[i + 2] * inv, r64[i + 3] * inv);
+            }
+        }
+    }
+    umma::cp_async_wait<0>();
+    umma::fence_before_sync();
+    __syncthreads();
+    if (tid == 0 && *abort_flag && a.err) atomicOr(a.err, 1);
+    if (warp == 0) umma::tmem_dealloc(tmem, Sh::TMEM_COLS);
+}
+
+template <int DIM, int DH>
+static cudaError_t launch_ws_t(const PrefillArgs& a, cudaStream_t s) {
+    using Sh = WsShape<DIM, DH>;
+    const int bytes = Sh::CPOS + ((a.dm.lam * 4 + 15) & ~15);
+    if (bytes > 227 * 1024) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(output_ws_kernel<DIM, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    const int nrp = (a.dm.Gq * a.dm.C + Sh::NTILE * Sh::ROWS - 1) / (Sh::NTILE * Sh::ROWS);
+    dim3 grid((a.c_end - a.c_begin) * nrp, a.dm.Hkv, a.dm.B);
+    output_ws_kernel<DIM, DH><<<grid, Sh::NT, bytes, s>>>(a);
+    return cudaGetLastError();
+}
+
+// bf16 inputs on the warp-specialised kernel; cudaErrorNotSupported for other shapes.
+cudaError_t launch_output_ws(const PrefillArgs& a, cudaStream_t s) {
+    const int d = a.dm.d, Dh = a.dm.Dh;
+    if (a.dm.dtype != 1) return cudaErrorNotSupported;
+    if (d == 128 && Dh == 64) return launch_ws_t<128, 64>(a, s);
+    if (d == 128 && Dh == 32) return launch_ws_t<128, 32>(a, s);
+    if (d == 64 && Dh == 32) return launch_ws_t<64, 32>(a, s);
+    if (d == 64 && Dh == 64) return launch_ws_t<64, 64>(a, s);
+    return cudaErrorNotSupported;
+}
+
+}  // namespace lola

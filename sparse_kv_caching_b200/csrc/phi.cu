@@ -11,7 +11,7 @@ namespace lola {
 
 template <int DIM, int DH, typename TIn>
 __global__ void __launch_bounds__(256) phi_keys_kernel(PrefillArgs a) {
-    constexpr int ROWS_PER_WARP = 4;
+    constexpr int ROWS_PER_WARP = 16;            // 128 rows per block share one staging of W
     constexpr int CPL = DH / 32;                 // feature columns per lane (1 or 2)
     __shared__ float Ws[DIM * DH];
     __shared__ float xs[8][DIM];
@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(256) phi_keys_kernel(PrefillArgs a) {
 
 template <int DIM, int DH, typename TIn>
 static cudaError_t launch_phi_t(const PrefillArgs& a, cudaStream_t s) {
-    const int rows_per_block = 8 * 4;
+    const int rows_per_block = 8 * 16;
     const int rows = (a.c_end - a.c_begin) * a.dm.C;
     dim3 grid((rows + rows_per_block - 1) / rows_per_block, a.dm.S);
     phi_keys_kernel<DIM, DH, TIn><<<grid, 256, 0, s>>>(a);

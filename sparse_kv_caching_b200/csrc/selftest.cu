@@ -4,7 +4,7 @@
 // Modes: bit 0 = B is MN-major ([K][N] in global) rather than K-major
 // ([N][K]); bit 1 = tf32 operands (f32 in global) rather than bf16; bit 2 =
 // 3xTF32 (hi*hi + hi*lo + lo*hi, f32-accurate products); bit 3 = A is
-// MN-major ([K][M] in global, tf32 only); bit 4 = A is read from tensor
+// MN-major ([K][M] in global); bit 4 = A is read from tensor
 // memory (tf32 only; stored there by tcgen05.st, K-major); bit 5 = no MMA is
 // issued and the completion wait gives up after about a millisecond (the
 // bounded-wait failure path: *err is set, C is filled with NaN, the kernel
@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
     __shared__ uint64_t mbar;
     __shared__ uint32_t tbase;
     const bool bmn = a.mode & 1, tf32 = a.mode & 2, x3 = (a.mode & 4) && tf32;
-    const bool amn = (a.mode & 8) && tf32, ats = (a.mode & 16) && tf32, expire = a.mode & 32;
+    const bool amn = a.mode & 8, ats = (a.mode & 16) && tf32, expire = a.mode & 32;
     const int M = a.M, N = a.N, K = a.K;
     const int es = tf32 ? 4 : 2;
     const size_t szA = (size_t)M * K * es, szB = (size_t)N * K * es;
@@ -75,7 +75,8 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
             if (x3) fill_chunk_major<float>(sB2, B, N, K, true, false);
         }
     } else {
-        fill_chunk_major<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, M, K, false, false);
+        if (amn) fill_chunk_major<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, K, M, false, false);
+        else fill_chunk_major<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, M, K, false, false);
         if (bmn) fill_chunk_major<__nv_bfloat16>(sB, (const __nv_bfloat16*)a.B, K, N, false, false);
         else fill_chunk_major<__nv_bfloat16>(sB, (const __nv_bfloat16*)a.B, N, K, false, false);
     }

@@ -93,6 +93,7 @@ SMALL = {
     "many-cands": dict(base=3, B=1, Hkv=2, Hq=8, T=1024, eta=256, lam=300, chunk=128, n_needles=4),
     # mixed feature/head widths
     "d64-Dh64": dict(base=5, B=1, Hkv=2, Hq=4, T=512, eta=64, lam=64, chunk=64, Dh=64),
+    "d64-gqa4": dict(base=5, B=1, Hkv=2, Hq=8, T=512, eta=64, lam=64, chunk=64),
     "d128-Dh32": dict(base=2, B=1, Hkv=2, Hq=4, T=512, eta=64, lam=64, chunk=64, Dh=32),
     # fp32 inputs at the 8B head shape
     "f32-d128": dict(base=2, B=1, Hkv=2, Hq=4, T=512, eta=64, lam=64, chunk=64, dtype="f32"),

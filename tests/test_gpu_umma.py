@@ -46,7 +46,8 @@ def _run(mode, N, K, seed=0, err=None):
     return C.double().cpu(), ref
 
 
-@pytest.mark.parametrize("mode", [0, 1])
+# modes 8, 9: A given MN-major ([K][M]), the layout of the fold's value operand
+@pytest.mark.parametrize("mode", [0, 1, 8, 9])
 @pytest.mark.parametrize("N,K", [(128, 128), (64, 64), (256, 32), (16, 16), (128, 256)])
 def test_bf16(mode, N, K):
     C, ref = _run(mode, N, K)
@@ -70,20 +71,10 @@ def test_3xtf32(mode, N, K):
     assert (C - ref).abs().max() / ref.abs().max() < 1e-5
 
 
-# tf32 with MN-major operands (B given as [K][N], A as [K][M]) and 3xTF32 on them:
-# the layouts the fold of the memory-update chain uses.
-@pytest.mark.parametrize("mode", [3, 7, 10, 14, 11, 15])
-@pytest.mark.parametrize("N,K", [(128, 64), (64, 128), (16, 8), (128, 32)])
-def test_tf32_mn_major(mode, N, K):
-    C, ref = _run(mode, N, K)
-    tol = 1e-5 if mode & 4 else 5e-3
-    assert (C - ref).abs().max() / ref.abs().max() < tol
-
-
 # A read from tensor memory (row m in lane m), B from shared memory: the SRE
 # product of the memory-update chain keeps H^T resident in tensor memory.
-@pytest.mark.parametrize("mode", [18, 22, 19, 23])
-@pytest.mark.parametrize("N,K", [(64, 128), (128, 64), (16, 16), (256, 128)])
+@pytest.mark.parametrize("mode", [18, 22])
+@pytest.mark.parametrize("N,K", [(64, 128), (128, 64), (16, 16), (256, 64)])
 def test_tf32_a_in_tmem(mode, N, K):
     C, ref = _run(mode, N, K)
     tol = 1e-5 if mode & 4 else 5e-3
