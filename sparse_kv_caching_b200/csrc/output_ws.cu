@@ -370,33 +370,48 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                     umma::commit(&mbar[kSFull + 2 + (j & 1)]);
                 }
             };
-            for (int j = 0; j < ntiles && !dead; ++j) {
-                if (j == 0) {
-                    dead |= !ws_wait(&mbar[kKvFull + 0], 0, abort_flag);
+            // Non-blocking schedule: tile j's P V products are issued as soon as its softmax
+            // is done, the next tile's scores as soon as its keys have landed and an S buffer
+            // is free (S(j) reuses the buffer of S(j - 2), whose softmax the issue of P V (j - 2)
+            // has already waited for).
+            int js = 0, jp = 0, tp = 0;                       // next S tile; next P V tile and query tile
+            uint64_t idle_since = umma::globaltimer_ns();
+            while (jp < ntiles && !dead) {
+                bool progress = false;
+                if (js < ntiles && js <= jp + 1 &&
+                    umma::mbar_try_wait(&mbar[kKvFull + js % NST], (js / NST) & 1)) {
                     umma::fence_after_sync();
-                    if (!dead) issue_s(0);
+                    issue_s(js);
+                    ++js;
+                    progress = true;
                 }
-                if (j + 1 < ntiles && !dead) {
-                    dead |= !ws_wait(&mbar[kKvFull + (j + 1) % NST], ((j + 1) / NST) & 1, abort_flag);
+                if (jp < js && umma::mbar_try_wait(&mbar[kPFull + tp], jp & 1)) {
                     umma::fence_after_sync();
-                    if (!dead) issue_s(j + 1);
-                }
-                const int sj = j % NST;
-                const uint64_t bv = sj == 0 ? dV[0] : (sj == 1 ? dV[1] : dV[2]);
-                const uint32_t first = (has_lin || j > 0) ? 1u : 0u;
-                for (int t = 0; t < ntl && !dead; ++t) {
-                    dead |= !ws_wait(&mbar[kPFull + t], j & 1, abort_flag);
-                    umma::fence_after_sync();
-                    if (dead) break;
-                    const uint64_t ap = t == 0 ? dP0 : dP1;
-                    const uint32_t dO = tmem + Sh::TO + t * Sh::OT;
+                    const int sj = jp % NST;
+                    const uint64_t bv = sj == 0 ? dV[0] : (sj == 1 ? dV[1] : dV[2]);
+                    const uint32_t first = (has_lin || jp > 0) ? 1u : 0u;
+                    const uint64_t ap = tp == 0 ? dP0 : dP1;
+                    const uint32_t dO = tmem + Sh::TO + tp * Sh::OT;
 #pragma unroll
                     for (int ks = 0; ks < KT / 16; ++ks)
                         umma::mma_f16(dO, ap + (uint64_t)(ks * 2 * ROWS), bv + (uint64_t)(ks * 16), idO,
                                       ks > 0 ? 1u : first);
-                    umma::commit(&mbar[kPvDone + t]);
+                    umma::commit(&mbar[kPvDone + tp]);
+                    if (++tp == ntl) {                        // both query tiles done with this key tile
+                        umma::commit(&mbar[kKvFree + jp % NST]);
+                        tp = 0;
+                        ++jp;
+                    }
+                    progress = true;
                 }
-                if (!dead) umma::commit(&mbar[kKvFree + j % NST]);
+                if (progress) {
+                    idle_since = umma::globaltimer_ns();
+                } else if (*abort_flag) {
+                    dead = true;
+                } else if (umma::globaltimer_ns() - idle_since > 4000000000ull) {
+                    *abort_flag = 1;
+                    dead = true;
+                }
             }
         }
     } else if (wg == 0 || twoB) {
@@ -409,7 +424,6 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             const int s = j % NST;
             bool ok = !dead;
             if (ok) ok = ws_wait(&mbar[kSFull + 2 * t + (j & 1)], (j >> 1) & 1, abort_flag);
-            if (ok && j >= 1) ok = ws_wait(&mbar[kPvDone + t], (j - 1) & 1, abort_flag);   // P and O free
             dead |= !__all_sync(0xffffffffu, ok);
             if (dead) break;
             umma::fence_after_sync();
@@ -430,6 +444,21 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 if (l == 0.f) m_ref = mx;                         // nothing accumulated yet
                 else if (mx > m_ref + 8.f) { factor = ws_ex2(m_ref - mx); rescale = true; m_ref = mx; }
             }
+            // weights P (f16) in registers while the previous P V product completes; the
+            // normaliser sums the f16-rounded weights that the P V product uses
+            uint32_t pw[KT / 2];
+            float rs = 0.f;
+#pragma unroll
+            for (int u = 0; u < KT / 2; ++u) {
+                pw[u] = ws_pack_f16(ws_ex2(sv[2 * u] - m_ref), ws_ex2(sv[2 * u + 1] - m_ref));
+                const float2 r2 = ws_unpack_f16(pw[u]);
+                rs += r2.x + r2.y;
+            }
+            ok = true;
+            if (j >= 1) ok = ws_wait(&mbar[kPvDone + t], (j - 1) & 1, abort_flag);   // P and O free
+            dead |= !__all_sync(0xffffffffu, ok);
+            if (dead) break;
+            umma::fence_after_sync();
             if (__any_sync(0xffffffffu, rescale)) {               // warp-collective TMEM access
                 l *= factor;
 #pragma unroll
@@ -444,19 +473,9 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 }
                 umma::tmem_wait_st();
             }
-            // the normaliser sums the f16-rounded weights that the P V product uses
-            float rs = 0.f;
 #pragma unroll
-            for (int ch = 0; ch < KT / 8; ++ch) {
-                uint32_t w[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    w[u] = ws_pack_f16(ws_ex2(sv[8 * ch + 2 * u] - m_ref), ws_ex2(sv[8 * ch + 2 * u + 1] - m_ref));
-                    const float2 r2 = ws_unpack_f16(w[u]);
-                    rs += r2.x + r2.y;
-                }
-                ws_st4(sPt + ch * ROWS * 16 + r * 16, w[0], w[1], w[2], w[3]);
-            }
+            for (int ch = 0; ch < KT / 8; ++ch)
+                ws_st4(sPt + ch * ROWS * 16 + r * 16, pw[4 * ch], pw[4 * ch + 1], pw[4 * ch + 2], pw[4 * ch + 3]);
             l += rs;
             umma::fence_async_smem();
             umma::fence_before_sync();

@@ -2,7 +2,8 @@
 //   phi(k) = [softmax(k W_g), softmax(-k W_g)]   (Hedgehog form; D = 2 Dh)
 // The pages only call phi "learned" (LoLA notes §2.1 notation table, §2.2);
 // this library fixes the Hedgehog form with per-kv-head W.  fp32 FFMA with
-// W staged in shared memory, exact softmax via expf.  Output layout
+// W staged in shared memory (each W value read feeds 8 rows held in
+// registers), exact softmax via expf.  Output layout
 // phik_new [S][max_tokens][D] (row i = token t_start + i of stream st).
 // A launch covers the tokens of chunks [c_begin, c_end) of the call.
 #include "device_common.cuh"
@@ -11,10 +12,12 @@ namespace lola {
 
 template <int DIM, int DH, typename TIn>
 __global__ void __launch_bounds__(256) phi_keys_kernel(PrefillArgs a) {
-    constexpr int ROWS_PER_WARP = 16;            // 128 rows per block share one staging of W
+    constexpr int RG = 8;                        // rows per warp and pass: one W read feeds RG rows
+    constexpr int PASSES = 2;                    // 8 warps x 8 rows x 2 passes = 128 rows per block
     constexpr int CPL = DH / 32;                 // feature columns per lane (1 or 2)
-    __shared__ float Ws[DIM * DH];
-    __shared__ float xs[8][DIM];
+    extern __shared__ __align__(16) float phi_smem[];
+    float* Ws = phi_smem;                                           // [DIM][DH]
+    float (*xs)[RG][DIM] = reinterpret_cast<float (*)[RG][DIM]>(phi_smem + DIM * DH);   // [8 warps]
     const Dims& dm = a.dm;
     const int st = blockIdx.y, b = st / dm.Hkv, g = st % dm.Hkv;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -22,40 +25,65 @@ __global__ void __launch_bounds__(256) phi_keys_kernel(PrefillArgs a) {
     for (int i = threadIdx.x; i < DIM * DH; i += 256) Ws[i] = to_f32(Wg[i]);
     __syncthreads();
     const int i_end = a.c_end * dm.C;
-    for (int r = 0; r < ROWS_PER_WARP; ++r) {
-        const int i = a.c_begin * dm.C + (blockIdx.x * 8 + warp) * ROWS_PER_WARP + r;
-        if (i >= i_end) break;
-        const TIn* x = (const TIn*)a.k + (((size_t)b * a.T + i) * dm.Hkv + g) * DIM;
-        for (int j = lane; j < DIM; j += 32) xs[warp][j] = to_f32(x[j]);
+    for (int pass = 0; pass < PASSES; ++pass) {
+        const int i0 = a.c_begin * dm.C + ((blockIdx.x * PASSES + pass) * 8 + warp) * RG;
+        if (i0 >= i_end) break;
+        // the warp's RG rows of k (rows past the end repeat the last valid row, not stored)
+        for (int idx = lane; idx < RG * DIM; idx += 32) {
+            const int r = idx / DIM, j = idx % DIM, i = min(i0 + r, i_end - 1);
+            xs[warp][r][j] = to_f32(((const TIn*)a.k)[(((size_t)b * a.T + i) * dm.Hkv + g) * DIM + j]);
+        }
         __syncwarp();
-        float z[CPL];
+        float z[RG][CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) z[c] = 0.f;
-        for (int j = 0; j < DIM; ++j) {
-            const float xj = xs[warp][j];
+        for (int r = 0; r < RG; ++r)
 #pragma unroll
-            for (int c = 0; c < CPL; ++c) z[c] = fmaf(xj, Ws[j * DH + lane + 32 * c], z[c]);
+            for (int c = 0; c < CPL; ++c) z[r][c] = 0.f;
+#pragma unroll 2
+        for (int j = 0; j < DIM; j += 4) {
+            float w[4][CPL];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) w[u][c] = Ws[(j + u) * DH + lane + 32 * c];
+#pragma unroll
+            for (int r = 0; r < RG; ++r) {
+                const float4 x = *reinterpret_cast<const float4*>(&xs[warp][r][j]);
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    z[r][c] = fmaf(x.x, w[0][c], z[r][c]);
+                    z[r][c] = fmaf(x.y, w[1][c], z[r][c]);
+                    z[r][c] = fmaf(x.z, w[2][c], z[r][c]);
+                    z[r][c] = fmaf(x.w, w[3][c], z[r][c]);
+                }
+            }
         }
-        float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) { mx = fmaxf(mx, z[c]); mn = fminf(mn, z[c]); }
-        mx = warp_max(mx);
-        mn = -warp_max(-mn);
-        float ep[CPL], en[CPL], sp = 0.f, sn = 0.f;
+        for (int r = 0; r < RG; ++r) {
+            const int i = i0 + r;
+            float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            ep[c] = expf(z[c] - mx);
-            en[c] = expf(mn - z[c]);
-            sp += ep[c];
-            sn += en[c];
-        }
-        sp = warp_sum(sp);
-        sn = warp_sum(sn);
-        float* out = a.phik_new + ((size_t)st * dm.max_tokens + i) * (2 * DH);
+            for (int c = 0; c < CPL; ++c) { mx = fmaxf(mx, z[r][c]); mn = fminf(mn, z[r][c]); }
+            mx = warp_max(mx);
+            mn = -warp_max(-mn);
+            float ep[CPL], en[CPL], sp = 0.f, sn = 0.f;
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) {
-            out[lane + 32 * c] = ep[c] / sp;
-            out[DH + lane + 32 * c] = en[c] / sn;
+            for (int c = 0; c < CPL; ++c) {
+                ep[c] = expf(z[r][c] - mx);
+                en[c] = expf(mn - z[r][c]);
+                sp += ep[c];
+                sn += en[c];
+            }
+            sp = warp_sum(sp);
+            sn = warp_sum(sn);
+            if (i < i_end) {
+                float* out = a.phik_new + ((size_t)st * dm.max_tokens + i) * (2 * DH);
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    out[lane + 32 * c] = ep[c] / sp;
+                    out[DH + lane + 32 * c] = en[c] / sn;
+                }
+            }
         }
         __syncwarp();
     }
@@ -63,10 +91,13 @@ __global__ void __launch_bounds__(256) phi_keys_kernel(PrefillArgs a) {
 
 template <int DIM, int DH, typename TIn>
 static cudaError_t launch_phi_t(const PrefillArgs& a, cudaStream_t s) {
-    const int rows_per_block = 8 * 16;
+    const int rows_per_block = 8 * 8 * 2;
     const int rows = (a.c_end - a.c_begin) * a.dm.C;
     dim3 grid((rows + rows_per_block - 1) / rows_per_block, a.dm.S);
-    phi_keys_kernel<DIM, DH, TIn><<<grid, 256, 0, s>>>(a);
+    const int bytes = (DIM * DH + 8 * 8 * DIM) * 4;
+    cudaError_t e = cudaFuncSetAttribute(phi_keys_kernel<DIM, DH, TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    phi_keys_kernel<DIM, DH, TIn><<<grid, 256, bytes, s>>>(a);
     return cudaGetLastError();
 }
 
