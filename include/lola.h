@@ -263,7 +263,9 @@ long long lola_launch_count(void);
  * bit 4 (with bit 1, not with bit 3): A read from tensor memory;
  * bit 5: no MMA is issued and the completion wait gives up after about 1 ms
  * (exercises the bounded-wait failure path: *err is set to 1 and C is filled
- * with NaN).  A, B, C, err are device pointers (C f32 row-major, *err set to
+ * with NaN); bit 6 (bf16 only): both operands in the 128-byte swizzled
+ * layout (64-element rows in 1024-byte atoms of 8 rows, K % 64 == 0 and, with
+ * bit 0, N % 64 == 0).  A, B, C, err are device pointers (C f32 row-major, *err set to
  * 1 if the MMA completion wait gave up).  Requires M = 128, 16 <= N <= 256
  * with N % 16 == 0, K a multiple of 16 (bf16, or A in tensor memory) or 8
  * (tf32), operands that fit in shared memory and at most 512 tensor-memory

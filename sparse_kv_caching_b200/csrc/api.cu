@@ -365,8 +365,11 @@ int lola_selftest_umma(int mode, const void* A, const void* B, float* C, int M, 
                        void* stream) {
     if (!A || !B || !C || !err) return fail(LOLA_ERR_INVALID_ARG, "null argument");
     const bool tf32 = mode & 2;
-    if (mode < 0 || mode > 63 || ((mode & (4 | 16)) && !tf32) || ((mode & 8) && (mode & 16)))
+    if (mode < 0 || mode > 127 || ((mode & (4 | 16)) && !tf32) || ((mode & 8) && (mode & 16)) ||
+        ((mode & 64) && tf32))
         return fail(LOLA_ERR_INVALID_ARG, "mode=%d", mode);
+    if ((mode & 64) && (K % 64 || ((mode & 1) && N % 64)))
+        return fail(LOLA_ERR_INVALID_ARG, "swizzled operands need K %% 64 == 0 (and N %% 64 == 0 for MN-major B)");
     if (M != 128 || N < 16 || N > 256 || N % 16 || K < (tf32 ? 8 : 16) || K % (tf32 ? 8 : 16))
         return fail(LOLA_ERR_INVALID_ARG, "unsupported shape M=%d N=%d K=%d", M, N, K);
     if ((mode & 16) && K % 16) return fail(LOLA_ERR_INVALID_ARG, "A in tensor memory needs K %% 16 == 0");

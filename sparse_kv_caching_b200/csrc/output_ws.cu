@@ -10,9 +10,14 @@
 // runs one 128-row tile per CTA).  Roles:
 //   warps 0-3 / 4-7  softmax and epilogue of tile A / B (thread r owns row r)
 //   warps 8-9        gather K and V rows of each 64-key tile with cp.async
-//                    into a 3-stage ring (row addresses looked up once per key,
-//                    the block's cache positions staged in the prologue),
-//                    convert V to f16 in place
+//                    into a 3-stage ring (row addresses looked up once per key
+//                    and shared by shuffles, the block's cache positions staged
+//                    in the prologue), convert V to f16 in place
+// K and V tiles sit in the 128-byte swizzled layout: each 128-byte half of a
+// key row is one contiguous shared-memory row (its 16-byte chunks permuted), so
+// the eight lanes that copy it touch one global line and one shared row, and
+// the same bytes serve as the K-major B operand of Q K^T and the MN-major B
+// operand of P V.
 //   warp 10, lane 0  issues every MMA
 // Tensor memory: O_A, O_B [128 x d] f32 and two S buffers per tile [128 x 64].
 // Per key tile j the MMA thread issues S_t(j+1) = Q_t K^T (bf16) while the
@@ -42,11 +47,10 @@ struct WsShape {
     static constexpr int Q = 0;                                 // [2 tiles]
     static constexpr int KV = Q + NTILE * QB;                   // [NST][K, V]
     static constexpr int P = KV + NST * 2 * KVB;                // [NTILE tiles]
-    static constexpr int KPTR = P + NTILE * PB;                 // [NST][KT] key-row pointers, then value rows
-    static constexpr int MBAR = KPTR + 2 * NST * KT * 8;        // 15 barriers
+    static constexpr int MBAR = P + NTILE * PB;                 // 15 barriers
     static constexpr int FLAG = MBAR + 16 * 8;                  // abort flag, tmem pointer
     static constexpr int CPOS = FLAG + 16;                      // cache positions of the block [lambda] int
-    static constexpr int KPOS = KPTR;                           // (end of the prologue aliases)
+    static constexpr int KPOS = MBAR;                           // (end of the prologue aliases)
     // prologue aliases (the KV and P regions are free until the roles start)
     static constexpr int HT = KV;                               // H_c^T, [D/32][DIM x 32] f32
     static constexpr int HTC = DIM * 32 * 4;
@@ -111,7 +115,9 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
     using Sh = WsShape<DIM, DH>;
     using bf16 = __nv_bfloat16;
     constexpr int ROWS = Sh::ROWS, KT = Sh::KT, D = Sh::D, NCH = Sh::NCH, NST = Sh::NST, NT = Sh::NT;
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // swizzle atoms want 1024-byte aligned tiles (the launch adds the slack)
+    uint8_t* smem = smem_raw + ((1024u - (umma::smem_addr(smem_raw) & 1023u)) & 1023u);
     const Dims& dm = a.dm;
     const int rows_total = dm.Gq * dm.C;
     constexpr int NTILE = Sh::NTILE;
@@ -133,8 +139,6 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
     uint8_t* sQ = smem + Sh::Q;
     uint8_t* sKV = smem + Sh::KV;
     uint8_t* sP = smem + Sh::P;
-    const bf16** kptr = reinterpret_cast<const bf16**>(smem + Sh::KPTR);      // [NST][KT]
-    const bf16** vptr = kptr + NST * KT;                                       // [NST][KT]
     int* cpos_s = reinterpret_cast<int*>(smem + Sh::CPOS);
     uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + Sh::MBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Sh::FLAG);
@@ -272,15 +276,26 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
 
     if (wg == 2 && warp < 10) {
         // ---- loaders: warp 8 takes keys 0-31 of every tile, warp 9 keys 32-63 ----
+        constexpr int NH = DIM / 64;                           // 128-byte halves of a key row
+        constexpr int HB = KT * 128;                           // one half of a K or V tile
         const int kb = (warp - 8) * 32;
+        // V (bf16) to f16 in place: this warp's 32 rows are NH contiguous 4 KB runs
         auto convert_v = [&](int s) {
-            uint8_t* sV = sKV + s * 2 * Sh::KVB + Sh::KVB;
-            for (int idx = lane; idx < 32 * NCH; idx += 32) {
-                const int kk = kb + (idx & 31), ch = idx >> 5;
-                uint4* pv = reinterpret_cast<uint4*>(sV + ch * KT * 16 + kk * 16);
-                uint4 u = *pv;
-                u.x = ws_bf2_to_h2(u.x); u.y = ws_bf2_to_h2(u.y); u.z = ws_bf2_to_h2(u.z); u.w = ws_bf2_to_h2(u.w);
-                *pv = u;
+            uint8_t* sV = sKV + s * 2 * Sh::KVB + Sh::KVB + kb * 128;
+#pragma unroll
+            for (int u0 = 0; u0 < NH * 8; u0 += 4) {
+                uint4 x[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int idx = (u0 + u) * 32 + lane;
+                    x[u] = *reinterpret_cast<const uint4*>(sV + (idx >> 8) * HB + (idx & 255) * 16);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int idx = (u0 + u) * 32 + lane;
+                    ws_st4(sV + (idx >> 8) * HB + (idx & 255) * 16, ws_bf2_to_h2(x[u].x), ws_bf2_to_h2(x[u].y),
+                           ws_bf2_to_h2(x[u].z), ws_bf2_to_h2(x[u].w));
+                }
             }
             umma::fence_async_smem();
             mbar_arrive(&mbar[kKvFull + s]);
@@ -292,35 +307,33 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 if (lane == 0 && !dead) ok = ws_wait(&mbar[kKvFree + s], ((j / NST) - 1) & 1, abort_flag);
                 dead |= !__shfl_sync(0xffffffffu, ok ? 1 : 0, 0);
             }
-            // where my 32 keys live (cache slots, window, block keys up to the last query)
+            // where my key lives (cache slot, window, or block key up to the last query)
+            unsigned long long kr = 0, vr = 0;
             {
                 const int gk = j * KT + kb + lane;
-                const bf16* kr = nullptr;
-                const bf16* vr = nullptr;
-                if (gk < N) {
+                if (gk < N && !dead) {
                     const int pos = gk < n_g ? cpos_s[gk] : (gk < n_g + n_w ? w_lo + (gk - n_g) : t0 + (gk - n_g - n_w));
                     const PairRef<bf16> pr = pair_ref<bf16>(a, st, b, g, pos, gk < n_g ? gk : 0);
-                    kr = pr.k;
-                    vr = pr.v;
+                    kr = reinterpret_cast<unsigned long long>(pr.k);
+                    vr = reinterpret_cast<unsigned long long>(pr.v);
                 }
-                kptr[s * KT + kb + lane] = kr;
-                vptr[s * KT + kb + lane] = vr;
             }
-            __syncwarp();
             uint8_t* sK = sKV + s * 2 * Sh::KVB;
             uint8_t* sV = sK + Sh::KVB;
-            for (int idx = lane; idx < 32 * NCH; idx += 32) {
-                const int kk = (idx & 7) + 8 * (idx / (8 * NCH)), ch = (idx >> 3) % NCH;
-                const int key = kb + kk;
-                uint8_t* dk = sK + ch * KT * 16 + key * 16;
-                uint8_t* dv = sV + ch * KT * 16 + key * 16;
-                const bf16* kr = kptr[s * KT + key];
-                if (kr != nullptr && !dead) {
-                    umma::cp_async16(dk, kr + 8 * ch);
-                    umma::cp_async16(dv, vptr[s * KT + key] + 8 * ch);
+            // one 16-byte chunk per lane: eight lanes per half row, four half rows per pass
+#pragma unroll
+            for (int it = 0; it < NH * 8; ++it) {
+                const int q = it * 32 + lane, c = q & 7, kh = q >> 3;
+                const int kl = NH == 2 ? kh >> 1 : kh, hf = NH == 2 ? (kh & 1) : 0;
+                const unsigned long long kq = __shfl_sync(0xffffffffu, kr, kl);
+                const unsigned long long vq = __shfl_sync(0xffffffffu, vr, kl);
+                const uint32_t off = hf * HB + umma::sw128_off(kb + kl, c);
+                if (kq != 0ull) {
+                    umma::cp_async16(sK + off, reinterpret_cast<const bf16*>(kq) + 64 * hf + 8 * c);
+                    umma::cp_async16(sV + off, reinterpret_cast<const bf16*>(vq) + 64 * hf + 8 * c);
                 } else {
-                    ws_st4(dk, 0u, 0u, 0u, 0u);
-                    ws_st4(dv, 0u, 0u, 0u, 0u);
+                    ws_st4(sK + off, 0u, 0u, 0u, 0u);
+                    ws_st4(sV + off, 0u, 0u, 0u, 0u);
                 }
             }
             umma::cp_async_commit();
@@ -341,9 +354,10 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             const uint32_t idS = umma::idesc(umma::kBF16, ROWS, KT, false, false);
             const uint32_t idO = umma::idesc(umma::kF16, ROWS, DIM, false, true);
             const int ntl = twoB ? 2 : 1;
-            // operand descriptors built once; a K step moves a K-major start by two 16-byte
-            // chunks of the tile's rows (the address field counts 16-byte units), an MN-major
-            // (value) start by 16 rows of 16 bytes
+            // operand descriptors built once (the address field counts 16-byte units).  Q and P
+            // (chunk-major, K-major): a K step moves the start by two 16-byte chunks of the
+            // tile's rows.  K (swizzled, K-major): 32 bytes inside a 128-byte half row, the next
+            // half KT rows further.  V (swizzled, MN-major): 16 key rows of 128 bytes.
             const uint64_t dQ0 = umma::sdesc(umma::smem_addr(sQ), ROWS * 16, 128);
             const uint64_t dQ1 = umma::sdesc(umma::smem_addr(sQ + (NTILE - 1) * Sh::QB), ROWS * 16, 128);
             const uint64_t dP0 = umma::sdesc(umma::smem_addr(sP), ROWS * 16, 128);
@@ -351,8 +365,8 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             uint64_t dK[NST], dV[NST];
 #pragma unroll
             for (int s = 0; s < NST; ++s) {
-                dK[s] = umma::sdesc(umma::smem_addr(sKV + s * 2 * Sh::KVB), KT * 16, 128);
-                dV[s] = umma::sdesc(umma::smem_addr(sKV + s * 2 * Sh::KVB + Sh::KVB), 128, KT * 16);
+                dK[s] = umma::sdesc_sw128(umma::smem_addr(sKV + s * 2 * Sh::KVB), 16, 1024);
+                dV[s] = umma::sdesc_sw128(umma::smem_addr(sKV + s * 2 * Sh::KVB + Sh::KVB), KT * 128, 1024);
             }
             auto issue_s = [&](int j) {
                 const int s = j % NST;
@@ -360,13 +374,14 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 const uint32_t d0 = tmem + Sh::TS + (j & 1) * KT;
 #pragma unroll
                 for (int ks = 0; ks < DIM / 16; ++ks)
-                    umma::mma_bf16(d0, dQ0 + (uint64_t)(ks * 2 * ROWS), bk + (uint64_t)(ks * 2 * KT), idS, ks > 0 ? 1u : 0u);
+                    umma::mma_bf16(d0, dQ0 + (uint64_t)(ks * 2 * ROWS), bk + (uint64_t)((ks >> 2) * KT * 8 + (ks & 3) * 2),
+                                   idS, ks > 0 ? 1u : 0u);
                 umma::commit(&mbar[kSFull + (j & 1)]);
                 if (ntl > 1) {
 #pragma unroll
                     for (int ks = 0; ks < DIM / 16; ++ks)
-                        umma::mma_bf16(d0 + 2 * KT, dQ1 + (uint64_t)(ks * 2 * ROWS), bk + (uint64_t)(ks * 2 * KT), idS,
-                                       ks > 0 ? 1u : 0u);
+                        umma::mma_bf16(d0 + 2 * KT, dQ1 + (uint64_t)(ks * 2 * ROWS),
+                                       bk + (uint64_t)((ks >> 2) * KT * 8 + (ks & 3) * 2), idS, ks > 0 ? 1u : 0u);
                     umma::commit(&mbar[kSFull + 2 + (j & 1)]);
                 }
             };
@@ -394,7 +409,7 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                     const uint32_t dO = tmem + Sh::TO + tp * Sh::OT;
 #pragma unroll
                     for (int ks = 0; ks < KT / 16; ++ks)
-                        umma::mma_f16(dO, ap + (uint64_t)(ks * 2 * ROWS), bv + (uint64_t)(ks * 16), idO,
+                        umma::mma_f16(dO, ap + (uint64_t)(ks * 2 * ROWS), bv + (uint64_t)(ks * 128), idO,
                                       ks > 0 ? 1u : first);
                     umma::commit(&mbar[kPvDone + tp]);
                     if (++tp == ntl) {                        // both query tiles done with this key tile
@@ -421,7 +436,6 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
         const float c2 = 1.4426950408889634f / sqrtf((float)DIM);    // log2(e) / sqrt(d)
         float m_ref = 0.f;
         for (int j = 0; j < ntiles; ++j) {
-            const int s = j % NST;
             bool ok = !dead;
             if (ok) ok = ws_wait(&mbar[kSFull + 2 * t + (j & 1)], (j >> 1) & 1, abort_flag);
             dead |= !__all_sync(0xffffffffu, ok);
@@ -510,7 +524,7 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
 template <int DIM, int DH>
 static cudaError_t launch_ws_t(const PrefillArgs& a, cudaStream_t s) {
     using Sh = WsShape<DIM, DH>;
-    const int bytes = Sh::CPOS + ((a.dm.lam * 4 + 15) & ~15);
+    const int bytes = Sh::CPOS + ((a.dm.lam * 4 + 15) & ~15) + 1024;   // + alignment slack
     if (bytes > 227 * 1024) return cudaErrorNotSupported;
     cudaError_t e = cudaFuncSetAttribute(output_ws_kernel<DIM, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;

@@ -8,7 +8,8 @@
 // memory (tf32 only; stored there by tcgen05.st, K-major); bit 5 = no MMA is
 // issued and the completion wait gives up after about a millisecond (the
 // bounded-wait failure path: *err is set, C is filled with NaN, the kernel
-// frees its tensor memory and returns).
+// frees its tensor memory and returns); bit 6 = bf16 operands in the 128-byte
+// swizzled layout (rows of 64 elements, 8-row atoms) instead of chunk-major.
 #include "device_common.cuh"
 #include "umma.cuh"
 
@@ -43,16 +44,29 @@ __device__ void fill_chunk_major(uint8_t* dst, const T* src, int R, int Kc, bool
     }
 }
 
+// Copy a row-major [R][Kc] bf16 matrix into 128-byte swizzled blocks: block
+// kb holds elements [64 kb, 64 kb + 64) of every row, R rows of 128 bytes.
+__device__ void fill_sw128(uint8_t* dst, const __nv_bfloat16* src, int R, int Kc) {
+    const int nchunks = R * (Kc / 8);
+    for (int idx = threadIdx.x; idx < nchunks; idx += blockDim.x) {
+        const int c = idx % 8, r = (idx / 8) % R, kb = idx / (8 * R);
+        const uint4 v = *reinterpret_cast<const uint4*>(src + (size_t)r * Kc + 64 * kb + 8 * c);
+        *reinterpret_cast<uint4*>(dst + (size_t)kb * R * 128 + umma::sw128_off(r, c)) = v;
+    }
+}
+
 __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint64_t mbar;
     __shared__ uint32_t tbase;
     const bool bmn = a.mode & 1, tf32 = a.mode & 2, x3 = (a.mode & 4) && tf32;
     const bool amn = a.mode & 8, ats = (a.mode & 16) && tf32, expire = a.mode & 32;
+    const bool sw = (a.mode & 64) && !tf32;
     const int M = a.M, N = a.N, K = a.K;
     const int es = tf32 ? 4 : 2;
     const size_t szA = (size_t)M * K * es, szB = (size_t)N * K * es;
-    uint8_t* sA = smem;
+    // swizzle atoms want a 1024-byte aligned base (the launch adds the slack)
+    uint8_t* sA = smem + ((1024u - (umma::smem_addr(smem) & 1023u)) & 1023u);
     uint8_t* sB = smem + szA;
     uint8_t* sA2 = sB + szB;                       // lo parts (3xTF32)
     uint8_t* sB2 = sA2 + szA;
@@ -74,6 +88,11 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
             fill_chunk_major<float>(sB, B, N, K, false, x3);
             if (x3) fill_chunk_major<float>(sB2, B, N, K, true, false);
         }
+    } else if (sw) {
+        if (amn) fill_sw128(sA, (const __nv_bfloat16*)a.A, K, M);
+        else fill_sw128(sA, (const __nv_bfloat16*)a.A, M, K);
+        if (bmn) fill_sw128(sB, (const __nv_bfloat16*)a.B, K, N);
+        else fill_sw128(sB, (const __nv_bfloat16*)a.B, N, K);
     } else {
         if (amn) fill_chunk_major<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, K, M, false, false);
         else fill_chunk_major<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, M, K, false, false);
@@ -127,6 +146,17 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
             for (int ks = 0; ks < K / kstep; ++ks) {
                 const uint32_t aoff = amn ? ks * kstep * 16 : ks * 2 * M * 16;
                 const uint32_t boff = bmn ? ks * kstep * 16 : ks * 2 * N * 16;
+                if (sw) {
+                    // K-major: 16-element steps of 32 bytes inside a 64-element block,
+                    // blocks R x 128 bytes apart; MN-major: 16 K rows = two 1024-byte groups
+                    const uint32_t ka = amn ? ks * 2048u : (ks / 4) * M * 128u + (ks % 4) * 32u;
+                    const uint32_t kb = bmn ? ks * 2048u : (ks / 4) * N * 128u + (ks % 4) * 32u;
+                    const uint64_t da = umma::sdesc_sw128(a0 + ka, amn ? K * 128u : 16u, 1024u);
+                    const uint64_t dbs = umma::sdesc_sw128(b0 + kb, bmn ? K * 128u : 16u, 1024u);
+                    umma::mma_bf16(tmem, da, dbs, id, acc);
+                    acc = 1;
+                    continue;
+                }
                 const uint64_t db = umma::sdesc(bbase + boff, lboB, sboB);
                 if (ats) {
                     const uint32_t ta = tmem + N + (p == 2 ? K : 0) + ks * kstep;
@@ -161,7 +191,7 @@ size_t selftest_smem(int mode, int M, int N, int K) {
     const bool tf32 = mode & 2, x3 = (mode & 4) && tf32;
     const size_t es = tf32 ? 4 : 2;
     size_t b = (size_t)M * K * es + (size_t)N * K * es;
-    return x3 ? 2 * b : b;
+    return (x3 ? 2 * b : b) + 1024;   // + alignment slack of the operand base
 }
 
 int selftest_tmem_cols(int mode, int N, int K) {

@@ -36,6 +36,22 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, ui
     return d;                                     // base offset 0, swizzle none
 }
 
+// The same descriptor for a 128-byte swizzled layout: 8-row atoms of 128-byte
+// rows, 1024-byte aligned, in which the 16-byte chunk c of row r sits at chunk
+// c ^ (r % 8).  K-major: sbo = stride between 8-row groups, lbo unused (the
+// K extent of one MMA stays inside a row); a K step inside the row moves the
+// start address by its byte offset.  MN-major: lbo = stride between 64-element
+// (128-byte) blocks along M or N, sbo = stride between groups of 8 K rows.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return sdesc(saddr, lbo_bytes, sbo_bytes) | ((uint64_t)2 << 61);
+}
+
+// Byte offset of the 16-byte chunk c of row r inside a 128-byte swizzled tile
+// whose rows are 128 bytes apart.
+__host__ __device__ constexpr uint32_t sw128_off(uint32_t r, uint32_t c) {
+    return r * 128u + (((c ^ r) & 7u) << 4);
+}
+
 enum Fmt : uint32_t { kF16 = 0, kBF16 = 1, kTF32 = 2 };
 
 // Instruction descriptor: f32 accumulate, dense, no negation.

@@ -55,6 +55,16 @@ def test_bf16(mode, N, K):
     assert (C - ref).abs().max() / ref.abs().max() < 1e-5
 
 
+# modes 64 + (0, 1, 8, 9): the 128-byte swizzled layout, in which the output
+# kernel holds its key tiles (K-major for Q K^T, MN-major for P V)
+@pytest.mark.parametrize("mode", [64, 65, 72, 73])
+@pytest.mark.parametrize("N,K", [(128, 128), (64, 64), (256, 64), (128, 256)])
+def test_bf16_swizzled(mode, N, K):
+    C, ref = _run(mode, N, K)
+    assert torch.isfinite(C).all()
+    assert (C - ref).abs().max() / ref.abs().max() < 1e-5
+
+
 # tf32 operands are used K-major only (the MN-major tf32 form is not used by
 # the library and is not tested).
 @pytest.mark.parametrize("mode", [2])
