@@ -184,9 +184,9 @@ def load_peaks():
 # What each part of the path computes in (bf16 inputs).
 PRECISIONS = {"inputs": "bf16 q, k, v, W", "phi": "f32",
               "sre": "3xTF32 tensor-core products (f32-accurate), f32 accumulation",
-              "fold": "tf32 tensor-core products with split operands (f32-accurate), f32 state",
+              "fold": "bf16 tensor-core products of 3-part bf16 splits (products to 2^-24 relative), f32 state",
               "select": "exact radix select over f32 score bits",
-              "attention": "bf16 QK^T, f16 PV, tf32 phi(q)^T H on the tensor cores, f32 softmax and accumulation",
+              "attention": "bf16 QK^T, f16 PV (P in tensor memory), tf32 phi(q)^T H on the tensor cores, f32 softmax and accumulation",
               "output": "f32 y", "decode": "f32 on the CUDA cores"}
 DTYPE = "bf16+f16+tf32+f32"
 

@@ -260,12 +260,13 @@ long long lola_launch_count(void);
  * memory.  mode bit 0: B given MN-major as [K][N] (else K-major as [N][K]);
  * bit 1: f32 inputs computed as tf32 (else bf16 inputs); bit 2 (with bit 1):
  * 3xTF32 split products; bit 3: A given MN-major as [K][M] (else [M][K]);
- * bit 4 (with bit 1, not with bit 3): A read from tensor memory;
+ * bit 4 (not with bit 3): A read from tensor memory (K % 32 == 0 for bf16);
  * bit 5: no MMA is issued and the completion wait gives up after about 1 ms
  * (exercises the bounded-wait failure path: *err is set to 1 and C is filled
- * with NaN); bit 6 (bf16 only): both operands in the 128-byte swizzled
- * layout (64-element rows in 1024-byte atoms of 8 rows, K % 64 == 0 and, with
- * bit 0, N % 64 == 0).  A, B, C, err are device pointers (C f32 row-major, *err set to
+ * with NaN); bit 6: operands in the 128-byte swizzled layout (128-byte rows
+ * in 1024-byte atoms of 8 rows; K % 64 == 0 for bf16, K % 32 == 0 for tf32;
+ * with bit 0, N % 64 == 0; tf32 takes it for K-major operands only, not with
+ * bits 0 or 3).  A, B, C, err are device pointers (C f32 row-major, *err set to
  * 1 if the MMA completion wait gave up).  Requires M = 128, 16 <= N <= 256
  * with N % 16 == 0, K a multiple of 16 (bf16, or A in tensor memory) or 8
  * (tf32), operands that fit in shared memory and at most 512 tensor-memory

@@ -365,14 +365,14 @@ int lola_selftest_umma(int mode, const void* A, const void* B, float* C, int M, 
                        void* stream) {
     if (!A || !B || !C || !err) return fail(LOLA_ERR_INVALID_ARG, "null argument");
     const bool tf32 = mode & 2;
-    if (mode < 0 || mode > 127 || ((mode & (4 | 16)) && !tf32) || ((mode & 8) && (mode & 16)) ||
-        ((mode & 64) && tf32))
+    if (mode < 0 || mode > 127 || ((mode & 4) && !tf32) || ((mode & 8) && (mode & 16)) ||
+        ((mode & 64) && tf32 && (mode & (1 | 8))))
         return fail(LOLA_ERR_INVALID_ARG, "mode=%d", mode);
-    if ((mode & 64) && (K % 64 || ((mode & 1) && N % 64)))
-        return fail(LOLA_ERR_INVALID_ARG, "swizzled operands need K %% 64 == 0 (and N %% 64 == 0 for MN-major B)");
+    if ((mode & 64) && (K % (tf32 ? 32 : 64) || ((mode & 1) && N % 64)))
+        return fail(LOLA_ERR_INVALID_ARG, "swizzled operands need 128-byte rows along K (and N %% 64 == 0 for MN-major B)");
     if (M != 128 || N < 16 || N > 256 || N % 16 || K < (tf32 ? 8 : 16) || K % (tf32 ? 8 : 16))
         return fail(LOLA_ERR_INVALID_ARG, "unsupported shape M=%d N=%d K=%d", M, N, K);
-    if ((mode & 16) && K % 16) return fail(LOLA_ERR_INVALID_ARG, "A in tensor memory needs K %% 16 == 0");
+    if ((mode & 16) && K % (tf32 ? 16 : 32)) return fail(LOLA_ERR_INVALID_ARG, "A in tensor memory needs K %% 16 == 0 (tf32) or K %% 32 == 0 (bf16)");
     if (lola::selftest_tmem_cols(mode, N, K) > 512)
         return fail(LOLA_ERR_UNSUPPORTED, "accumulator and A need more than 512 tensor-memory columns");
     if (lola::selftest_smem(mode, M, N, K) > (size_t)kMaxSmem)

@@ -22,7 +22,9 @@
 // Tensor memory: O_A, O_B [128 x d] f32 and two S buffers per tile [128 x 64].
 // Per key tile j the MMA thread issues S_t(j+1) = Q_t K^T (bf16) while the
 // softmax warps turn S_t(j) into P_t (f16, exp2 in the log2 domain with a
-// lazily raised reference maximum); then O_t += P_t V (f16).
+// lazily raised reference maximum) and store it over S_t(j) in tensor memory
+// (two f16 per column); then O_t += P_t V (f16, A = P_t read from tensor
+// memory, B = V from shared memory).
 // Prologue (all warps, before the roles split): z = Q W (bf16 MMA), phi(q)
 // in registers, O_t = phi(q)^T H_c (tf32 MMA over 32-column chunks), l =
 // phi(q) . s_c: the linear branch enters the online softmax as logit 0.
@@ -35,7 +37,7 @@ namespace lola {
 
 template <int DIM, int DH>
 struct WsShape {
-    static constexpr int ROWS = 128, KT = 64, D = 2 * DH, NCH = DIM / 8, NST = 3;
+    static constexpr int ROWS = 128, KT = 64, D = 2 * DH, NCH = DIM / 8, NST = 4;
     static constexpr int NT = 352;                              // 11 warps
     // query tiles per CTA: two 128-row tiles share every gathered key tile for d = 128;
     // one for d = 64 (with two tiles at d = 64 the second tile's scores came out wrong
@@ -43,12 +45,10 @@ struct WsShape {
     static constexpr int NTILE = DIM == 128 ? 2 : 1;
     static constexpr int QB = ROWS * DIM * 2;                   // one query tile (bf16)
     static constexpr int KVB = KT * DIM * 2;                    // one K or V tile
-    static constexpr int PB = ROWS * KT * 2;                    // one P tile (f16)
     static constexpr int Q = 0;                                 // [2 tiles]
     static constexpr int KV = Q + NTILE * QB;                   // [NST][K, V]
-    static constexpr int P = KV + NST * 2 * KVB;                // [NTILE tiles]
-    static constexpr int MBAR = P + NTILE * PB;                 // 15 barriers
-    static constexpr int FLAG = MBAR + 16 * 8;                  // abort flag, tmem pointer
+    static constexpr int MBAR = KV + NST * 2 * KVB;             // 17 barriers
+    static constexpr int FLAG = MBAR + 24 * 8;                  // abort flag, tmem pointer
     static constexpr int CPOS = FLAG + 16;                      // cache positions of the block [lambda] int
     static constexpr int KPOS = MBAR;                           // (end of the prologue aliases)
     // prologue aliases (the KV and P regions are free until the roles start)
@@ -65,8 +65,8 @@ struct WsShape {
     static_assert(DIM <= (int)OT && TS + 4 * KT <= 512, "tensor memory");
 };
 
-// barrier indices
-enum : int { kKvFull = 0, kKvFree = 3, kSFull = 6, kPFull = 10, kPvDone = 12, kPro = 14 };
+// barrier indices (four ring stages)
+enum : int { kKvFull = 0, kKvFree = 4, kSFull = 8, kPFull = 12, kPvDone = 14, kPro = 16 };
 
 // Bounded mbarrier wait that also gives up once another thread of the CTA has
 // raised the abort flag; returns false if it gave up (and raises the flag).
@@ -138,7 +138,7 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
 
     uint8_t* sQ = smem + Sh::Q;
     uint8_t* sKV = smem + Sh::KV;
-    uint8_t* sP = smem + Sh::P;
+    static_assert(NST == 4, "barrier indices assume four stages");
     int* cpos_s = reinterpret_cast<int*>(smem + Sh::CPOS);
     uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + Sh::MBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Sh::FLAG);
@@ -352,25 +352,21 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
         // ---- MMA issuer ----
         if (mma_thread) {
             const uint32_t idS = umma::idesc(umma::kBF16, ROWS, KT, false, false);
-            const uint32_t idO = umma::idesc(umma::kF16, ROWS, DIM, false, true);
+            const uint32_t idO = umma::idesc(umma::kF16, ROWS, DIM, false, true);   // A = P in tensor memory
             const int ntl = twoB ? 2 : 1;
-            // operand descriptors built once (the address field counts 16-byte units).  Q and P
+            // operand descriptors built once (the address field counts 16-byte units).  Q
             // (chunk-major, K-major): a K step moves the start by two 16-byte chunks of the
             // tile's rows.  K (swizzled, K-major): 32 bytes inside a 128-byte half row, the next
-            // half KT rows further.  V (swizzled, MN-major): 16 key rows of 128 bytes.
+            // half KT rows further.  V (swizzled, MN-major): 16 key rows of 128 bytes.  P (tensor
+            // memory, two f16 per column): 8 columns.
             const uint64_t dQ0 = umma::sdesc(umma::smem_addr(sQ), ROWS * 16, 128);
             const uint64_t dQ1 = umma::sdesc(umma::smem_addr(sQ + (NTILE - 1) * Sh::QB), ROWS * 16, 128);
-            const uint64_t dP0 = umma::sdesc(umma::smem_addr(sP), ROWS * 16, 128);
-            const uint64_t dP1 = umma::sdesc(umma::smem_addr(sP + (NTILE - 1) * Sh::PB), ROWS * 16, 128);
-            uint64_t dK[NST], dV[NST];
-#pragma unroll
-            for (int s = 0; s < NST; ++s) {
-                dK[s] = umma::sdesc_sw128(umma::smem_addr(sKV + s * 2 * Sh::KVB), 16, 1024);
-                dV[s] = umma::sdesc_sw128(umma::smem_addr(sKV + s * 2 * Sh::KVB + Sh::KVB), KT * 128, 1024);
-            }
+            // stage s sits 2 KVB bytes after stage s - 1
+            const uint64_t dK0 = umma::sdesc_sw128(umma::smem_addr(sKV), 16, 1024);
+            const uint64_t dV0 = umma::sdesc_sw128(umma::smem_addr(sKV + Sh::KVB), KT * 128, 1024);
             auto issue_s = [&](int j) {
                 const int s = j % NST;
-                const uint64_t bk = s == 0 ? dK[0] : (s == 1 ? dK[1] : dK[2]);
+                const uint64_t bk = dK0 + (uint64_t)(s * (2 * Sh::KVB / 16));
                 const uint32_t d0 = tmem + Sh::TS + (j & 1) * KT;
 #pragma unroll
                 for (int ks = 0; ks < DIM / 16; ++ks)
@@ -387,30 +383,31 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             };
             // Non-blocking schedule: tile j's P V products are issued as soon as its softmax
             // is done, the next tile's scores as soon as its keys have landed and an S buffer
-            // is free (S(j) reuses the buffer of S(j - 2), whose softmax the issue of P V (j - 2)
-            // has already waited for).
+            // is free (S(j) reuses the buffer of S(j - 2) and P(j - 2): the issue of P V (j - 2)
+            // has waited for that softmax, and the tensor cores run P V (j - 2) before S(j)).
             int js = 0, jp = 0, tp = 0;                       // next S tile; next P V tile and query tile
             uint64_t idle_since = umma::globaltimer_ns();
             while (jp < ntiles && !dead) {
                 bool progress = false;
+                // test_wait, not try_wait: a try_wait on a barrier that is not ready may
+                // suspend this thread while the other one completes
                 if (js < ntiles && js <= jp + 1 &&
-                    umma::mbar_try_wait(&mbar[kKvFull + js % NST], (js / NST) & 1)) {
+                    umma::mbar_test_wait(&mbar[kKvFull + js % NST], (js / NST) & 1)) {
                     umma::fence_after_sync();
                     issue_s(js);
                     ++js;
                     progress = true;
                 }
-                if (jp < js && umma::mbar_try_wait(&mbar[kPFull + tp], jp & 1)) {
+                if (jp < js && umma::mbar_test_wait(&mbar[kPFull + tp], jp & 1)) {
                     umma::fence_after_sync();
                     const int sj = jp % NST;
-                    const uint64_t bv = sj == 0 ? dV[0] : (sj == 1 ? dV[1] : dV[2]);
+                    const uint64_t bv = dV0 + (uint64_t)(sj * (2 * Sh::KVB / 16));
                     const uint32_t first = (has_lin || jp > 0) ? 1u : 0u;
-                    const uint64_t ap = tp == 0 ? dP0 : dP1;
+                    const uint32_t aP = tmem + Sh::TS + (2 * tp + (jp & 1)) * KT;
                     const uint32_t dO = tmem + Sh::TO + tp * Sh::OT;
 #pragma unroll
                     for (int ks = 0; ks < KT / 16; ++ks)
-                        umma::mma_f16(dO, ap + (uint64_t)(ks * 2 * ROWS), bv + (uint64_t)(ks * 128), idO,
-                                      ks > 0 ? 1u : first);
+                        umma::mma_f16_ts(dO, aP + 8 * ks, bv + (uint64_t)(ks * 128), idO, ks > 0 ? 1u : first);
                     umma::commit(&mbar[kPvDone + tp]);
                     if (++tp == ntl) {                        // both query tiles done with this key tile
                         umma::commit(&mbar[kKvFree + jp % NST]);
@@ -432,7 +429,6 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
     } else if (wg == 0 || twoB) {
         // ---- softmax of tile wg: thread r owns row r ----
         const int t = wg;
-        uint8_t* sPt = sP + t * Sh::PB;
         const float c2 = 1.4426950408889634f / sqrtf((float)DIM);    // log2(e) / sqrt(d)
         float m_ref = 0.f;
         for (int j = 0; j < ntiles; ++j) {
@@ -458,8 +454,8 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 if (l == 0.f) m_ref = mx;                         // nothing accumulated yet
                 else if (mx > m_ref + 8.f) { factor = ws_ex2(m_ref - mx); rescale = true; m_ref = mx; }
             }
-            // weights P (f16) in registers while the previous P V product completes; the
-            // normaliser sums the f16-rounded weights that the P V product uses
+            // weights P (f16); the normaliser sums the f16-rounded weights that the P V
+            // product uses
             uint32_t pw[KT / 2];
             float rs = 0.f;
 #pragma unroll
@@ -468,8 +464,18 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 const float2 r2 = ws_unpack_f16(pw[u]);
                 rs += r2.x + r2.y;
             }
+            // P(j) over S(j): the tensor cores finished P V (j - 2), which read this buffer,
+            // before S(j), whose scores were just read
+            {
+                const uint32_t pcol = tmem + lane_off + Sh::TS + (2 * t + (j & 1)) * KT;
+#pragma unroll
+                for (int c0 = 0; c0 < KT / 2; c0 += 16)
+                    umma::tmem_st16(pcol + c0, *reinterpret_cast<const float(*)[16]>(pw + c0));
+            }
+            // P V (j - 1) complete: O may be rescaled, and the MMA thread has taken the previous
+            // phase of this tile's P barrier (arriving again before that would alias its parity)
             ok = true;
-            if (j >= 1) ok = ws_wait(&mbar[kPvDone + t], (j - 1) & 1, abort_flag);   // P and O free
+            if (j >= 1) ok = ws_wait(&mbar[kPvDone + t], (j - 1) & 1, abort_flag);
             dead |= !__all_sync(0xffffffffu, ok);
             if (dead) break;
             umma::fence_after_sync();
@@ -487,11 +493,8 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 }
                 umma::tmem_wait_st();
             }
-#pragma unroll
-            for (int ch = 0; ch < KT / 8; ++ch)
-                ws_st4(sPt + ch * ROWS * 16 + r * 16, pw[4 * ch], pw[4 * ch + 1], pw[4 * ch + 2], pw[4 * ch + 3]);
+            umma::tmem_wait_st();
             l += rs;
-            umma::fence_async_smem();
             umma::fence_before_sync();
             mbar_arrive(&mbar[kPFull + t]);
         }

@@ -16,7 +16,9 @@
 //     the launch keeps H_hi = H rounded down to tf32 and H_lo = H - H_hi.
 //   * SRE: for a tile of 64 candidates, P^T = H^T Phi^T is three tf32 MMAs
 //     with A = H_hi / H_lo read from tensor memory and B = Phi_hi / Phi_lo
-//     (the candidates' phi rows, split the same way) in shared memory:
+//     (the candidates' phi rows, split the same way) in shared memory, in the
+//     128-byte swizzled layout (each 128-byte piece of a phi row is one
+//     shared-memory row, so a warp's copies touch few lines and rows):
 //     P = H_hi Phi_hi + H_lo Phi_hi + H_hi Phi_lo, f32-accurate products
 //     (the dropped H_lo Phi_lo term is 2^-22 relative) with f32 accumulation.
 //     The epilogue reads P^T back (lane c, column e), divides by den_e =
@@ -58,8 +60,8 @@ __host__ __device__ inline TcOffsets tc_offsets(int D, int DV, int esize, int la
     TcOffsets o;
     int p = 0;
     auto take = [&](int n, int al) { p = (p + al - 1) / al * al; const int r = p; p += n; return r; };
-    o.raw = take(3 * TN * D * 4, 128);
-    o.lo = take(2 * TN * D * 4, 128);
+    o.raw = take(3 * TN * D * 4, 1024);        // 128-byte swizzled tiles: 1024-byte aligned
+    o.lo = take(2 * TN * D * 4, 1024);
     const int ring = p;
     // fold: A = value parts [3][128 / 8 chunks][FK rows][16 B], B = phi parts [3][D / 8][FK][16 B],
     // then the folded rows as loaded (phi [FK][D] f32, values [FK][DV])
@@ -121,7 +123,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     constexpr uint32_t cH = 0, cHhi = D, cHlo = 2 * D, cP = 3 * D;
     static_assert(3 * D + 2 * TN <= (int)TCOLS, "tensor memory");
     static_assert(DV % 32 == 0 && DV <= M && D % 16 == 0, "shape");
-    extern __shared__ __align__(1024) uint8_t smem[];
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // swizzle atoms want 1024-byte aligned tiles (the launch adds the slack)
+    uint8_t* smem = smem_raw + ((1024u - (umma::smem_addr(smem_raw) & 1023u)) & 1023u);
     const Dims& dm = a.dm;
     const int lam = dm.lam, C = dm.C, eta = dm.eta;
     int rank = 0;
@@ -232,9 +236,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     };
 
     // ---- SRE of the candidates of one block -------------------------------------
-    // Ring of three raw phi tiles (the tile's rows, K-major B operand: chunk j/4 of row r
-    // at (j/4)(TN 16) + 16 r), two tf32-low tiles, and per tile the partial and final
-    // 1/den and the value-row pointers (four slots).  Loads run two tiles ahead.
+    // Ring of three raw phi tiles (the tile's rows, K-major B operand, 128-byte swizzled:
+    // the 16-byte chunk jc of row r, jc = 8 kb + c, at kb (TN 128) + 128 r + 16 (c ^ r % 8)),
+    // two tf32-low tiles in the same layout, and per tile the partial and final 1/den and
+    // the value-row pointers (four slots).  Loads run two tiles ahead.
     float* dpart = reinterpret_cast<float*>(smem + o.dpart);
     float* invd = reinterpret_cast<float*>(smem + o.inv);
     const TIn** vptr = reinterpret_cast<const TIn**>(smem + o.vptr);
@@ -242,21 +247,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     auto lo_tile = [&](int lb) { return smem + o.lo + lb * (TN * D * 4); };
     // cp.async the phi rows of tile t (slot i of this CTA's tiles) into raw[i % 3]; rows
     // past n are zero; the value-row pointers go to vptr[i % 4].  Always commits a group.
+    static_assert(NT == 4 * TN, "four threads per candidate row");
     auto issue_loads = [&](int t, int i, int n) {
         if (t >= 0) {
-            // thread (r, q): row r of the tile, chunks q, q + 4, ... of it (one row lookup)
+            // thread 4 r + q looks up row r of the tile (warp w: rows 8 w .. 8 w + 7); the warp
+            // then copies its eight rows with eight lanes per 128-byte piece (one global line,
+            // one shared row), the row's address taken from the lane that looked it up
             uint8_t* base = raw_tile(i % 3);
-            const int r = tid / (NT / TN), q = tid % (NT / TN), e = t * TN + r;
-            uint8_t* dst = base + r * 16;
+            const int r = tid / 4, e = t * TN + r;
+            unsigned long long src = 0ull;
+            const TIn* vrow = nullptr;
             if (e < n) {
                 const PairRef<TIn> pr = pair_ref<TIn>(a, st, b, g, cand_pos[e], e);
+                src = reinterpret_cast<unsigned long long>(pr.phik);
+                vrow = pr.v;
+            }
+            if ((tid & 3) == 0) vptr[(i % 4) * TN + r] = vrow;
+            const int c = lane & 7;
 #pragma unroll
-                for (int jc = q; jc < D / 4; jc += NT / TN) umma::cp_async16(dst + jc * (TN * 16), pr.phik + 4 * jc);
-                if (q == 0) vptr[(i % 4) * TN + r] = pr.v;
-            } else {
-#pragma unroll
-                for (int jc = q; jc < D / 4; jc += NT / TN) st_shared_zero16(dst + jc * (TN * 16));
-                if (q == 0) vptr[(i % 4) * TN + r] = nullptr;
+            for (int u = 0; u < D / 16; ++u) {                // D / 4 chunks x 8 rows / 32 lanes
+                const int rr = 4 * (u & 1) + (lane >> 3), kb = u >> 1, row = 8 * warp + rr;
+                const unsigned long long p = __shfl_sync(0xffffffffu, src, 4 * rr);
+                uint8_t* dst = base + kb * (TN * 128) + umma::sw128_off(row, c);
+                if (p != 0ull) umma::cp_async16(dst, reinterpret_cast<const float*>(p) + 32 * kb + 4 * c);
+                else st_shared_zero16(dst);
             }
         }
         umma::cp_async_commit();
@@ -270,14 +284,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
         const int r = tid % TN, q = tid / TN;
         float d0 = 0.f, d1 = 0.f;
         for (int jc = q; jc < D / 4; jc += NT / TN) {
-            float4* p = reinterpret_cast<float4*>(phi + jc * TN * 4 + r * 4);
+            const int off = ((jc >> 3) * (TN * 128) + (int)umma::sw128_off(r, jc & 7)) / 4;
+            float4* p = reinterpret_cast<float4*>(phi + off);
             const float4 x = *p;
             const float4 s4 = *reinterpret_cast<const float4*>(ss + 4 * jc);
             d0 = fmaf(x.x, s4.x, d0); d1 = fmaf(x.y, s4.y, d1);
             d0 = fmaf(x.z, s4.z, d0); d1 = fmaf(x.w, s4.w, d1);
             const float4 h = make_float4(umma::tf32_hi(x.x), umma::tf32_hi(x.y), umma::tf32_hi(x.z), umma::tf32_hi(x.w));
             *p = h;
-            *reinterpret_cast<float4*>(plo + jc * TN * 4 + r * 4) = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
+            *reinterpret_cast<float4*>(plo + off) = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
         }
         dp[q * TN + r] = d0 + d1;
     };
@@ -293,14 +308,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
         if (tid != 0 || failed) return;
         const int pb = i & 1;
         const uint32_t id = umma::idesc(umma::kTF32, M, TN, false, false);
-        const uint64_t bh0 = umma::sdesc(umma::smem_addr(raw_tile(i % 3)), TN * 16, 128);
-        const uint64_t bl0 = umma::sdesc(umma::smem_addr(lo_tile(i & 1)), TN * 16, 128);
+        const uint64_t bh0 = umma::sdesc_sw128(umma::smem_addr(raw_tile(i % 3)), 16, 1024);
+        const uint64_t bl0 = umma::sdesc_sw128(umma::smem_addr(lo_tile(i & 1)), 16, 1024);
         const uint32_t dP = tmem + cP + pb * TN;
-        // a K step of 8 moves the operand start by 2 chunks of TN rows (the descriptor's
-        // address field counts 16-byte units)
+        // a K step of 8 moves the operand start by 32 bytes inside a 128-byte row piece, the
+        // next piece TN rows further (the descriptor's address field counts 16-byte units)
 #pragma unroll
         for (int ks = 0; ks < D / 8; ++ks) {
-            const uint64_t step = (uint64_t)(ks * 2 * TN);
+            const uint64_t step = (uint64_t)((ks >> 2) * (TN * 8) + (ks & 3) * 2);
             umma::mma_tf32_ts(dP, tmem + cHhi + ks * 8, bh0 + step, id, ks > 0 ? 1u : 0u);
             umma::mma_tf32_ts(dP, tmem + cHlo + ks * 8, bh0 + step, id, 1u);
             umma::mma_tf32_ts(dP, tmem + cHhi + ks * 8, bl0 + step, id, 1u);
@@ -593,7 +608,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
 }
 
 size_t scan_tc_smem_bytes(const Dims& dm, int ncl) {
-    const size_t b = (size_t)tc_offsets(dm.D, dm.d, dm.esize, dm.lam, dm.C, ncl).total;
+    const size_t b = (size_t)tc_offsets(dm.D, dm.d, dm.esize, dm.lam, dm.C, ncl).total + 1024;   // + alignment slack
     return b < (size_t)kTcMinSmem ? (size_t)kTcMinSmem : b;
 }
 

@@ -5,11 +5,13 @@
 // ([N][K]); bit 1 = tf32 operands (f32 in global) rather than bf16; bit 2 =
 // 3xTF32 (hi*hi + hi*lo + lo*hi, f32-accurate products); bit 3 = A is
 // MN-major ([K][M] in global); bit 4 = A is read from tensor
-// memory (tf32 only; stored there by tcgen05.st, K-major); bit 5 = no MMA is
+// memory (stored there by tcgen05.st, K-major: one f32 per column for tf32,
+// two bf16 per column otherwise); bit 5 = no MMA is
 // issued and the completion wait gives up after about a millisecond (the
 // bounded-wait failure path: *err is set, C is filled with NaN, the kernel
-// frees its tensor memory and returns); bit 6 = bf16 operands in the 128-byte
-// swizzled layout (rows of 64 elements, 8-row atoms) instead of chunk-major.
+// frees its tensor memory and returns); bit 6 = operands in the 128-byte
+// swizzled layout (128-byte rows, 8-row atoms) instead of chunk-major (tf32:
+// K-major operands only).
 #include "device_common.cuh"
 #include "umma.cuh"
 
@@ -44,14 +46,26 @@ __device__ void fill_chunk_major(uint8_t* dst, const T* src, int R, int Kc, bool
     }
 }
 
-// Copy a row-major [R][Kc] bf16 matrix into 128-byte swizzled blocks: block
-// kb holds elements [64 kb, 64 kb + 64) of every row, R rows of 128 bytes.
-__device__ void fill_sw128(uint8_t* dst, const __nv_bfloat16* src, int R, int Kc) {
-    const int nchunks = R * (Kc / 8);
+// Copy a row-major [R][Kc] matrix into 128-byte swizzled blocks: block kb
+// holds the kb-th 128 bytes of every row (64 bf16 or 32 f32), R rows of 128
+// bytes; f32 may be split as for fill_chunk_major.
+template <typename T>
+__device__ void fill_sw128(uint8_t* dst, const T* src, int R, int Kc, bool split_lo = false, bool split_hi = false) {
+    constexpr int TPC = 16 / sizeof(T), TPB = 128 / sizeof(T);
+    const int nchunks = R * (Kc / TPC);
     for (int idx = threadIdx.x; idx < nchunks; idx += blockDim.x) {
         const int c = idx % 8, r = (idx / 8) % R, kb = idx / (8 * R);
-        const uint4 v = *reinterpret_cast<const uint4*>(src + (size_t)r * Kc + 64 * kb + 8 * c);
-        *reinterpret_cast<uint4*>(dst + (size_t)kb * R * 128 + umma::sw128_off(r, c)) = v;
+        const T* s = src + (size_t)r * Kc + TPB * kb + TPC * c;
+        T* d = reinterpret_cast<T*>(dst + (size_t)kb * R * 128 + umma::sw128_off(r, c));
+#pragma unroll
+        for (int i = 0; i < TPC; ++i) {
+            T x = s[i];
+            if constexpr (sizeof(T) == 4) {
+                if (split_hi) x = umma::tf32_hi(x);
+                else if (split_lo) x = x - umma::tf32_hi(x);
+            }
+            d[i] = x;
+        }
     }
 }
 
@@ -60,8 +74,8 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
     __shared__ uint64_t mbar;
     __shared__ uint32_t tbase;
     const bool bmn = a.mode & 1, tf32 = a.mode & 2, x3 = (a.mode & 4) && tf32;
-    const bool amn = a.mode & 8, ats = (a.mode & 16) && tf32, expire = a.mode & 32;
-    const bool sw = (a.mode & 64) && !tf32;
+    const bool amn = a.mode & 8, ats = a.mode & 16, expire = a.mode & 32;
+    const bool sw = a.mode & 64;
     const int M = a.M, N = a.N, K = a.K;
     const int es = tf32 ? 4 : 2;
     const size_t szA = (size_t)M * K * es, szB = (size_t)N * K * es;
@@ -74,14 +88,22 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
     if (tf32) {
         const float* A = (const float*)a.A;
         const float* B = (const float*)a.B;
-        if (amn) {   // A given as [K][M]: rows = K, chunks along M
+        if (sw) {    // K-major operands only
+            if (!ats) {
+                fill_sw128<float>(sA, A, M, K, false, x3);
+                if (x3) fill_sw128<float>(sA2, A, M, K, true, false);
+            }
+            fill_sw128<float>(sB, B, N, K, false, x3);
+            if (x3) fill_sw128<float>(sB2, B, N, K, true, false);
+        } else if (amn) {   // A given as [K][M]: rows = K, chunks along M
             fill_chunk_major<float>(sA, A, K, M, false, x3);
             if (x3) fill_chunk_major<float>(sA2, A, K, M, true, false);
         } else if (!ats) {
             fill_chunk_major<float>(sA, A, M, K, false, x3);
             if (x3) fill_chunk_major<float>(sA2, A, M, K, true, false);
         }
-        if (bmn) {   // rows = K, chunks along N
+        if (sw) {
+        } else if (bmn) {   // rows = K, chunks along N
             fill_chunk_major<float>(sB, B, K, N, false, x3);
             if (x3) fill_chunk_major<float>(sB2, B, K, N, true, false);
         } else {
@@ -89,10 +111,10 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
             if (x3) fill_chunk_major<float>(sB2, B, N, K, true, false);
         }
     } else if (sw) {
-        if (amn) fill_sw128(sA, (const __nv_bfloat16*)a.A, K, M);
-        else fill_sw128(sA, (const __nv_bfloat16*)a.A, M, K);
-        if (bmn) fill_sw128(sB, (const __nv_bfloat16*)a.B, K, N);
-        else fill_sw128(sB, (const __nv_bfloat16*)a.B, N, K);
+        if (amn) fill_sw128<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, K, M);
+        else fill_sw128<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, M, K);
+        if (bmn) fill_sw128<__nv_bfloat16>(sB, (const __nv_bfloat16*)a.B, K, N);
+        else fill_sw128<__nv_bfloat16>(sB, (const __nv_bfloat16*)a.B, N, K);
     } else {
         if (amn) fill_chunk_major<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, K, M, false, false);
         else fill_chunk_major<__nv_bfloat16>(sA, (const __nv_bfloat16*)a.A, M, K, false, false);
@@ -101,7 +123,7 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
     }
     umma::fence_async_smem();
     // accumulator columns [0, N); with A in tensor memory, A (hi) at column N and A_lo after it
-    const int need_cols = N + (ats ? K * (x3 ? 2 : 1) : 0);
+    const int need_cols = N + (ats ? (tf32 ? K * (x3 ? 2 : 1) : K / 2) : 0);
     const uint32_t ncols = need_cols <= 32 ? 32 : need_cols <= 64 ? 64 : need_cols <= 128 ? 128
                          : need_cols <= 256 ? 256 : 512;
     if (warp == 0) umma::tmem_alloc(&tbase, ncols);
@@ -110,7 +132,26 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = tbase;
-    if (ats) {
+    if (ats && !tf32) {
+        // thread r of the 128 stores row r of A into lane r, two bf16 per column
+        const uint16_t* A = (const uint16_t*)a.A;
+        const int r = threadIdx.x;
+        const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+        for (int k0 = 0; k0 < K; k0 += 32) {
+            float w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint32_t lo = r < M ? A[(size_t)r * K + k0 + 2 * i] : 0u;
+                const uint32_t hi = r < M ? A[(size_t)r * K + k0 + 2 * i + 1] : 0u;
+                w[i] = __uint_as_float(lo | (hi << 16));
+            }
+            umma::tmem_st16(tmem + lane_off + N + k0 / 2, w);
+        }
+        umma::tmem_wait_st();
+        umma::fence_before_sync();
+        __syncthreads();
+        umma::fence_after_sync();
+    } else if (ats) {
         // thread r of the 128 stores row r of A (and of A_lo) into lane r, one f32 per column
         const float* A = (const float*)a.A;
         const int r = threadIdx.x;
@@ -147,18 +188,23 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
                 const uint32_t aoff = amn ? ks * kstep * 16 : ks * 2 * M * 16;
                 const uint32_t boff = bmn ? ks * kstep * 16 : ks * 2 * N * 16;
                 if (sw) {
-                    // K-major: 16-element steps of 32 bytes inside a 64-element block,
-                    // blocks R x 128 bytes apart; MN-major: 16 K rows = two 1024-byte groups
+                    // K-major: K steps of 32 bytes (16 bf16, 8 f32) inside a 128-byte block,
+                    // blocks R x 128 bytes apart; MN-major (bf16): 16 K rows = two 1024-byte groups
                     const uint32_t ka = amn ? ks * 2048u : (ks / 4) * M * 128u + (ks % 4) * 32u;
                     const uint32_t kb = bmn ? ks * 2048u : (ks / 4) * N * 128u + (ks % 4) * 32u;
-                    const uint64_t da = umma::sdesc_sw128(a0 + ka, amn ? K * 128u : 16u, 1024u);
-                    const uint64_t dbs = umma::sdesc_sw128(b0 + kb, bmn ? K * 128u : 16u, 1024u);
-                    umma::mma_bf16(tmem, da, dbs, id, acc);
+                    const uint64_t da = umma::sdesc_sw128(abase + ka, amn ? K * 128u : 16u, 1024u);
+                    const uint64_t dbs = umma::sdesc_sw128(bbase + kb, bmn ? K * 128u : 16u, 1024u);
+                    if (ats && tf32) umma::mma_tf32_ts(tmem, tmem + N + (p == 2 ? K : 0) + ks * kstep, dbs, id, acc);
+                    else if (ats) umma::mma_f16_ts(tmem, tmem + N + ks * 8, dbs, id, acc);
+                    else if (tf32) umma::mma_tf32(tmem, da, dbs, id, acc);
+                    else umma::mma_bf16(tmem, da, dbs, id, acc);
                     acc = 1;
                     continue;
                 }
                 const uint64_t db = umma::sdesc(bbase + boff, lboB, sboB);
-                if (ats) {
+                if (ats && !tf32) {
+                    umma::mma_f16_ts(tmem, tmem + N + ks * 8, db, id, acc);   // 16 bf16 = 8 columns
+                } else if (ats) {
                     const uint32_t ta = tmem + N + (p == 2 ? K : 0) + ks * kstep;
                     umma::mma_tf32_ts(tmem, ta, db, id, acc);
                 } else {
@@ -195,8 +241,8 @@ size_t selftest_smem(int mode, int M, int N, int K) {
 }
 
 int selftest_tmem_cols(int mode, int N, int K) {
-    const bool tf32 = mode & 2, x3 = (mode & 4) && tf32, ats = (mode & 16) && tf32;
-    return N + (ats ? K * (x3 ? 2 : 1) : 0);
+    const bool tf32 = mode & 2, x3 = (mode & 4) && tf32, ats = mode & 16;
+    return N + (ats ? (tf32 ? K * (x3 ? 2 : 1) : K / 2) : 0);
 }
 
 cudaError_t launch_selftest(int mode, const void* A, const void* B, float* C, int M, int N, int K, int* err,

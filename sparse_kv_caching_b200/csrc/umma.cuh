@@ -92,6 +92,17 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
         :: "r"(d_tmem), "r"(a_tmem), "l"(b), "r"(id), "r"(acc));
 }
 
+// D[tmem] (+)= A[tmem] * B[smem] with 16-bit operands (kind::f16: f16 or bf16 as
+// the instruction descriptor says); A K-major in tensor memory: row m of A in lane
+// m, two elements per 32-bit column (element 2 i in the low half of column i).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t id, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+        :: "r"(d_tmem), "r"(a_tmem), "l"(b), "r"(id), "r"(acc));
+}
+
 // Arrive on an mbarrier once all previously issued MMAs of this thread complete.
 __device__ __forceinline__ void commit(uint64_t* mbar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -151,6 +162,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* mbar, uint32_t phase) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok) : "r"(smem_addr(mbar)), "r"(phase) : "memory");
+    return ok != 0;
+}
+// Non-blocking test of the same condition: never suspends the thread, for a
+// thread that polls several barriers in turn.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* mbar, uint32_t phase) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok) : "r"(smem_addr(mbar)), "r"(phase) : "memory");
     return ok != 0;

@@ -259,6 +259,28 @@ def test_pipelined_host_prefill_matches_device(T, Tpad):
         assert torch.equal(e1[key], e2[key]), key
 
 
+@pytest.mark.slow
+def test_repeated_full_batch_prefill_is_deterministic():
+    """The 16K workload's shapes (B 4, lambda 1024, eta 512, C 128) on a 4096-token
+    prefix, prefilled eight times from a reset state: every pass must finish
+    without a device-side wait giving up (the kernels' barrier phases must not
+    alias under any interleaving of their roles) and give the same bits."""
+    w = synth.workload(3, T=4096)
+    full = synth.full_arrays(w)
+    dev = P.to_device(w, full)
+    q, k, v = (dev[x][:, :w.T].contiguous() for x in ("q", "k", "v"))
+    layer = P.make_layer(w, dev["W"], max_tokens=w.T)
+    y0 = None
+    for _ in range(8):
+        layer.reset()
+        y = layer.prefill(q, k, v)
+        layer.check()
+        if y0 is None:
+            y0 = y.clone()
+        else:
+            assert torch.equal(y, y0)
+
+
 def test_invalid_arguments_are_errors():
     import sparse_kv_caching_b200 as lola
     w = P.small_workload(2, B=1, Hkv=2, Hq=8, T=256, eta=64, lam=64, chunk=64)

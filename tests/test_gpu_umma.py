@@ -65,6 +65,27 @@ def test_bf16_swizzled(mode, N, K):
     assert (C - ref).abs().max() / ref.abs().max() < 1e-5
 
 
+# bf16 with A in tensor memory (two elements per column), the form of the
+# output kernel's P V product (A = P; B = V MN-major, chunk-major or swizzled)
+@pytest.mark.parametrize("mode", [16, 17, 80, 81])
+@pytest.mark.parametrize("N,K", [(128, 64), (64, 128), (256, 64), (128, 128)])
+def test_bf16_a_in_tmem(mode, N, K):
+    C, ref = _run(mode, N, K)
+    assert torch.isfinite(C).all()
+    assert (C - ref).abs().max() / ref.abs().max() < 1e-5
+
+
+# tf32 in the swizzled layout, K-major: plain, 3xTF32, and with A in tensor
+# memory (the chain's SRE form: A = H^T parts in tensor memory, B = phi rows)
+@pytest.mark.parametrize("mode", [66, 70, 82, 86])
+@pytest.mark.parametrize("N,K", [(64, 128), (128, 64), (64, 32), (256, 64)])
+def test_tf32_swizzled(mode, N, K):
+    C, ref = _run(mode, N, K)
+    tol = 1e-5 if mode & 4 else 5e-3
+    assert torch.isfinite(C).all()
+    assert (C - ref).abs().max() / ref.abs().max() < tol
+
+
 # tf32 operands are used K-major only (the MN-major tf32 form is not used by
 # the library and is not tested).
 @pytest.mark.parametrize("mode", [2])
