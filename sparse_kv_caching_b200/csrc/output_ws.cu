@@ -80,9 +80,6 @@ __device__ __forceinline__ bool ws_wait(uint64_t* mbar, uint32_t parity, volatil
     return true;
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* mbar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(umma::smem_addr(mbar)) : "memory");
-}
 
 __device__ __forceinline__ float ws_ex2(float x) {
     float y;
@@ -298,7 +295,7 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 }
             }
             umma::fence_async_smem();
-            mbar_arrive(&mbar[kKvFull + s]);
+            umma::mbar_arrive(&mbar[kKvFull + s]);
         };
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % NST;
@@ -496,7 +493,7 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             umma::tmem_wait_st();
             l += rs;
             umma::fence_before_sync();
-            mbar_arrive(&mbar[kPFull + t]);
+            umma::mbar_arrive(&mbar[kPFull + t]);
         }
         // ---- epilogue: y = O / l ----
         bool ok = !dead && ntiles > 0;

@@ -14,7 +14,11 @@
 //   * H^T lives in tensor memory for the whole launch: lane c holds column c
 //     of H (rows c >= d are zero), one f32 per TMEM column j < D.  Beside it
 //     the launch keeps H_hi = H rounded down to tf32 and H_lo = H - H_hi.
-//   * SRE: for a tile of 64 candidates, P^T = H^T Phi^T is three tf32 MMAs
+//   * SRE, warp-specialised: the compute warps copy a tile's phi rows, split
+//     them and hand the tile to a ninth warp that issues its products, then
+//     take the scores of the previous tile while those run (named barriers
+//     among the compute warps, mbarriers between them and the issuing warp).
+//     For a tile of 64 candidates, P^T = H^T Phi^T is three tf32 MMAs
 //     with A = H_hi / H_lo read from tensor memory and B = Phi_hi / Phi_lo
 //     (the candidates' phi rows, split the same way) in shared memory, in the
 //     128-byte swizzled layout (each 128-byte piece of a phi row is one
@@ -42,7 +46,10 @@
 
 namespace lola {
 
-constexpr int kTcThreads = 256;
+constexpr int kTcCompute = 256;  // warps 0-7: loads, tf32 split, epilogue, selection, fold
+constexpr int kTcMmaWarp = 8;    // warp 8: issues the SRE products
+constexpr int kTcThreads = kTcCompute + 32;
+constexpr uint32_t kTcComputeBar = 1;   // named barrier of the compute warps
 constexpr int kTcTN = 64;        // candidates per SRE tile (N of the SRE product)
 constexpr int kTcFK = 64;        // folded pairs per fold product (K)
 constexpr int kTcMinSmem = 170 * 1024;   // one chain CTA per SM: its tensor memory is not shared
@@ -89,7 +96,7 @@ __host__ __device__ inline TcOffsets tc_offsets(int D, int DV, int esize, int la
     o.tmp = take(32 * 4, 16);
     o.part = take(4 * TN * 4, 16);
     o.ss = take(D * 4, 16);
-    o.mbar = take(4 * 8, 8);
+    o.mbar = take(8 * 8, 8);
     o.tptr = take(16, 16);
     o.total = p;
     return o;
@@ -151,12 +158,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     int* tmp = reinterpret_cast<int*>(smem + o.tmp);
     float* part = reinterpret_cast<float*>(smem + o.part);
     float* ss = reinterpret_cast<float*>(smem + o.ss);
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + o.mbar);   // [0], [1]: SRE tiles; [2]: fold
+    // [0], [1]: SRE products of tiles i % 2 done; [2]: fold products done; [3], [4]: tile i % 2
+    // split and ready for its products
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + o.mbar);
     uint32_t* tptr = reinterpret_cast<uint32_t*>(smem + o.tptr);
 
     if (warp == 0) umma::tmem_alloc(tptr, TCOLS);
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) umma::mbar_init(&mbar[i], 1);
+        for (int i = 0; i < 5; ++i) umma::mbar_init(&mbar[i], 1);
         umma::fence_mbar_init();
     }
     const size_t snaps = (size_t)dm.nc_max + 1;
@@ -170,12 +179,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = *tptr;
-    uint32_t phases = 0u;                                     // bit i: parity of mbar[i]
+    uint32_t phases = 0u;                                     // bit i: parity of mbar[i] (barriers this thread waits on)
     bool failed = false;                                      // uniform across the CTA
+    const bool compute = warp < kTcCompute / 32;
 
     // H^T entering the launch into tensor memory (and its tf32 split); warp half
     // h covers columns j in [h D/2, (h+1) D/2)
-    {
+    if (compute) {
         const float* Hrow = a.sp.H + (size_t)st * D * DV;                              // [D][DV]
         const float* Hsnap = a.snap_H + ((size_t)st * snaps + a.c_begin) * D * DV;      // [DV][D]
         for (int j0 = half * (D / 2); j0 < (half + 1) * (D / 2); j0 += 16) {
@@ -202,7 +212,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     auto publish = [&](int c) {
         float* sH = a.snap_H + ((size_t)st * snaps + c) * D * DV;
         const bool mine = crow < DV && (NCL == 1 || crow / (DV / NCL) == rank);
-        {
+        if (compute) {
             float x[D / 2];
 #pragma unroll
             for (int j0 = 0; j0 < D / 2; j0 += 16)
@@ -235,6 +245,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
         }
     };
 
+    // the same among the compute warps only (during the SRE, while the issuing warp runs its loop)
+    auto wait_mma_c = [&](int i) {
+        bool ok = true;
+        if (!failed) ok = umma::mbar_wait(&mbar[i], (phases >> i) & 1u);
+        phases ^= 1u << i;
+        umma::fence_after_sync();
+        if (umma::named_sync_or(kTcComputeBar, kTcCompute, !ok)) {
+            if (!failed && a.err && tid == 0) atomicOr(a.err, 1);
+            failed = true;
+        }
+    };
+
     // ---- SRE of the candidates of one block -------------------------------------
     // Ring of three raw phi tiles (the tile's rows, K-major B operand, 128-byte swizzled:
     // the 16-byte chunk jc of row r, jc = 8 kb + c, at kb (TN 128) + 128 r + 16 (c ^ r % 8)),
@@ -247,7 +269,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     auto lo_tile = [&](int lb) { return smem + o.lo + lb * (TN * D * 4); };
     // cp.async the phi rows of tile t (slot i of this CTA's tiles) into raw[i % 3]; rows
     // past n are zero; the value-row pointers go to vptr[i % 4].  Always commits a group.
-    static_assert(NT == 4 * TN, "four threads per candidate row");
+    static_assert(kTcCompute == 4 * TN, "four compute threads per candidate row");
     auto issue_loads = [&](int t, int i, int n) {
         if (t >= 0) {
             // thread 4 r + q looks up row r of the tile (warp w: rows 8 w .. 8 w + 7); the warp
@@ -283,7 +305,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
         float* dp = dpart + (i % 3) * 4 * TN;
         const int r = tid % TN, q = tid / TN;
         float d0 = 0.f, d1 = 0.f;
-        for (int jc = q; jc < D / 4; jc += NT / TN) {
+        for (int jc = q; jc < D / 4; jc += kTcCompute / TN) {
             const int off = ((jc >> 3) * (TN * 128) + (int)umma::sw128_off(r, jc & 7)) / 4;
             float4* p = reinterpret_cast<float4*>(phi + off);
             const float4 x = *p;
@@ -304,8 +326,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
             invd[(i % 3) * TN + tid] = dn > 0.f ? 1.f / dn : 0.f;
         }
     };
-    auto issue_sre_mma = [&](int i) {
-        if (tid != 0 || failed) return;
+    auto issue_sre_mma = [&](int i) {                        // lane 0 of the issuing warp
         const int pb = i & 1;
         const uint32_t id = umma::idesc(umma::kTF32, M, TN, false, false);
         const uint64_t bh0 = umma::sdesc_sw128(umma::smem_addr(raw_tile(i % 3)), 16, 1024);
@@ -352,7 +373,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
             }
             part[quarter * TN + 32 * half + lane] = x[0];
         }
-        __syncthreads();
+        umma::named_sync(kTcComputeBar, kTcCompute);
         if (tid < TN) {
             const int e = t * TN + tid;
             if (e < n) {
@@ -369,18 +390,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
         const int mt = nt > rank ? (nt - rank + NCL - 1) / NCL : 0;    // tiles rank, rank + NCL, ...
         float* out = NCL > 1 ? xsc + xb * NM : score;
         auto tile_of = [&](int i) { return i < mt ? rank + i * NCL : -1; };
-        if (mt > 0) {
+        if (mt > 0 && compute) {
             issue_loads(tile_of(0), 0, n);
             issue_loads(tile_of(1), 1, n);
             issue_loads(tile_of(2), 2, n);
             umma::cp_async_wait<2>();
-            __syncthreads();
-            prep(0);
-            umma::fence_async_smem();
-            umma::fence_before_sync();
-            __syncthreads();
-            umma::fence_after_sync();
-            issue_sre_mma(0);
+            umma::named_sync(kTcComputeBar, kTcCompute);
+            // split tile i and hand it to the issuing warp (mbar[3 + i % 2])
+            auto prep_and_pass = [&](int i) {
+                prep(i);
+                umma::fence_async_smem();
+                umma::fence_before_sync();
+                umma::named_sync(kTcComputeBar, kTcCompute);
+                if (tid == 0) umma::mbar_arrive(&mbar[3 + (i & 1)]);
+            };
+            prep_and_pass(0);
             den_final(0);
             // this thread's values (column crow of its 32 candidates) of a tile, loaded one
             // tile ahead of the epilogue that needs them
@@ -399,24 +423,39 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
                 const int t = tile_of(i);
                 if (i + 1 < mt) {
                     umma::cp_async_wait<1>();                 // tile i + 1 has landed (i + 2 may be in flight)
-                    __syncthreads();
-                    prep(i + 1);
-                    umma::fence_async_smem();
-                    umma::fence_before_sync();
-                    __syncthreads();
-                    umma::fence_after_sync();
-                    issue_sre_mma(i + 1);
+                    umma::named_sync(kTcComputeBar, kTcCompute);
+                    // lo[(i + 1) % 2] was last read by the products of tile i - 1, waited for
+                    prep_and_pass(i + 1);
                     den_final(i + 1);
                     load_values(i + 1, vnext);
                 }
-                wait_mma(i & 1);                              // tile i's products; raw[i % 3] is free
+                wait_mma_c(i & 1);                            // tile i's products; raw[i % 3] is free
                 issue_loads(tile_of(i + 3), i + 3, n);
                 epilogue(t, i, n, out, vcur);
                 umma::fence_before_sync();
 #pragma unroll
                 for (int k = 0; k < 32; ++k) vcur[k] = vnext[k];
             }
-            __syncthreads();
+            umma::named_sync(kTcComputeBar, kTcCompute);
+        } else if (mt > 0 && warp == kTcMmaWarp) {
+            // the issuing warp: tile i's products once the compute warps have split it; the
+            // ready barriers alternate, so a compute warp signalling tile i + 2 has already
+            // waited for the products of tile i, issued after this warp saw tile i ready
+            for (int i = 0; i < mt; ++i) {
+                const int rb = 3 + (i & 1);
+                bool ok = true;
+                if (lane == 0 && !failed) ok = umma::mbar_wait(&mbar[rb], (phases >> rb) & 1u);
+                phases ^= 1u << rb;
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) failed = true;                       // made uniform after the block
+                umma::fence_after_sync();
+                if (lane == 0 && !failed) issue_sre_mma(i);
+                __syncwarp();
+            }
+        }
+        if (__syncthreads_or(failed ? 1 : 0)) {
+            if (!failed && a.err && tid == 0) atomicOr(a.err, 1);
+            failed = true;
         }
         if constexpr (NCL > 1) {
             cg::cluster_group cluster = cg::this_cluster();
@@ -545,7 +584,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
             wait_mma(2);                                      // the operands may be overwritten now
         }
         // refresh the tf32 split of H^T
-        for (int j0 = half * (D / 2); j0 < (half + 1) * (D / 2); j0 += 16) {
+        for (int j0 = half * (D / 2); compute && j0 < (half + 1) * (D / 2); j0 += 16) {
             float x[16], hi[16], lo[16];
             umma::tmem_ld16(tmem + lane_off + cH + j0, x);
             umma::tmem_wait_ld();
@@ -589,7 +628,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     {
         float* Ho = a.sp.H + (size_t)st * D * DV;
         const bool mine = crow < DV && (NCL == 1 || crow / (DV / NCL) == rank);
-        for (int j0 = half * (D / 2); j0 < (half + 1) * (D / 2); j0 += 16) {
+        for (int j0 = half * (D / 2); compute && j0 < (half + 1) * (D / 2); j0 += 16) {
             float x[16];
             umma::tmem_ld16(tmem + lane_off + cH + j0, x);
             umma::tmem_wait_ld();

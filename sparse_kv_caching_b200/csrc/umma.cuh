@@ -166,6 +166,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* mbar, uint32_t phase) {
         : "=r"(ok) : "r"(smem_addr(mbar)), "r"(phase) : "memory");
     return ok != 0;
 }
+__device__ __forceinline__ void mbar_arrive(uint64_t* mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(smem_addr(mbar)) : "memory");
+}
+
+// Named barrier `id` over the first `nthreads` threads of the CTA (a warp-multiple),
+// and its OR-reduction form.
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ bool named_sync_or(uint32_t id, uint32_t nthreads, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred q, o;\n\t"
+        "setp.ne.b32 q, %3, 0;\n\t"
+        "bar.red.or.pred o, %1, %2, q;\n\t"
+        "selp.u32 %0, 1, 0, o;\n\t}\n"
+        : "=r"(r) : "r"(id), "r"(nthreads), "r"(pred ? 1u : 0u) : "memory");
+    return r != 0;
+}
+
 // Non-blocking test of the same condition: never suspends the thread, for a
 // thread that polls several barriers in turn.
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* mbar, uint32_t phase) {
