@@ -10,9 +10,10 @@
 // runs one 128-row tile per CTA).  Roles:
 //   warps 0-3 / 4-7  softmax and epilogue of tile A / B (thread r owns row r)
 //   warps 8-9        gather K and V rows of each 64-key tile with cp.async
-//                    into a 3-stage ring (row addresses looked up once per key
+//                    into a 4-stage ring (row addresses looked up once per key
 //                    and shared by shuffles, the block's cache positions staged
-//                    in the prologue), convert V to f16 in place
+//                    in the prologue); tile A's softmax warps turn V into f16
+//                    in place once their weights are stored
 // K and V tiles sit in the 128-byte swizzled layout: each 128-byte half of a
 // key row is one contiguous shared-memory row (its 16-byte chunks permuted), so
 // the eight lanes that copy it touch one global line and one shared row, and
@@ -65,7 +66,8 @@ struct WsShape {
     static_assert(DIM <= (int)OT && TS + 4 * KT <= 512, "tensor memory");
 };
 
-// barrier indices (four ring stages)
+// barrier indices (four ring stages): K and V landed, stage free; S ready (two buffers
+// per query tile), P ready (for tile A: V in f16 too), P V done (per query tile); prologue
 enum : int { kKvFull = 0, kKvFree = 4, kSFull = 8, kPFull = 12, kPvDone = 14, kPro = 16 };
 
 // Bounded mbarrier wait that also gives up once another thread of the CTA has
@@ -90,7 +92,6 @@ __device__ __forceinline__ uint32_t ws_pack_f16(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
-__device__ __forceinline__ float2 ws_unpack_f16(uint32_t u) { return __half22float2(*reinterpret_cast<__half2*>(&u)); }
 __device__ __forceinline__ uint32_t ws_bf2_to_h2(uint32_t u) {
     return ws_pack_f16(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
@@ -143,7 +144,10 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
 
     if (warp == 0) umma::tmem_alloc(tptr, Sh::TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i < NST; ++i) { umma::mbar_init(&mbar[kKvFull + i], 64); umma::mbar_init(&mbar[kKvFree + i], 1); }
+        for (int i = 0; i < NST; ++i) {
+            umma::mbar_init(&mbar[kKvFull + i], 64);
+            umma::mbar_init(&mbar[kKvFree + i], 1);
+        }
         for (int i = 0; i < 4; ++i) umma::mbar_init(&mbar[kSFull + i], 1);
         for (int t = 0; t < 2; ++t) { umma::mbar_init(&mbar[kPFull + t], ROWS); umma::mbar_init(&mbar[kPvDone + t], 1); }
         umma::mbar_init(&mbar[kPro], 1);
@@ -276,24 +280,7 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
         constexpr int NH = DIM / 64;                           // 128-byte halves of a key row
         constexpr int HB = KT * 128;                           // one half of a K or V tile
         const int kb = (warp - 8) * 32;
-        // V (bf16) to f16 in place: this warp's 32 rows are NH contiguous 4 KB runs
-        auto convert_v = [&](int s) {
-            uint8_t* sV = sKV + s * 2 * Sh::KVB + Sh::KVB + kb * 128;
-#pragma unroll
-            for (int u0 = 0; u0 < NH * 8; u0 += 4) {
-                uint4 x[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int idx = (u0 + u) * 32 + lane;
-                    x[u] = *reinterpret_cast<const uint4*>(sV + (idx >> 8) * HB + (idx & 255) * 16);
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int idx = (u0 + u) * 32 + lane;
-                    ws_st4(sV + (idx >> 8) * HB + (idx & 255) * 16, ws_bf2_to_h2(x[u].x), ws_bf2_to_h2(x[u].y),
-                           ws_bf2_to_h2(x[u].z), ws_bf2_to_h2(x[u].w));
-                }
-            }
+        auto landed = [&](int s) {                             // this warp's copies of stage s are in
             umma::fence_async_smem();
             umma::mbar_arrive(&mbar[kKvFull + s]);
         };
@@ -304,46 +291,47 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 if (lane == 0 && !dead) ok = ws_wait(&mbar[kKvFree + s], ((j / NST) - 1) & 1, abort_flag);
                 dead |= !__shfl_sync(0xffffffffu, ok ? 1 : 0, 0);
             }
-            // where my key lives (cache slot, window, or block key up to the last query)
-            unsigned long long kr = 0, vr = 0;
+            // where my key lives (cache slot, window, or block key up to the last query); keys
+            // past the last one are zero-filled (their source address is only a placeholder)
+            unsigned long long kr = reinterpret_cast<unsigned long long>(a.k), dv = 0;
+            bool valid = false;
             {
                 const int gk = j * KT + kb + lane;
                 if (gk < N && !dead) {
                     const int pos = gk < n_g ? cpos_s[gk] : (gk < n_g + n_w ? w_lo + (gk - n_g) : t0 + (gk - n_g - n_w));
                     const PairRef<bf16> pr = pair_ref<bf16>(a, st, b, g, pos, gk < n_g ? gk : 0);
                     kr = reinterpret_cast<unsigned long long>(pr.k);
-                    vr = reinterpret_cast<unsigned long long>(pr.v);
+                    dv = reinterpret_cast<unsigned long long>(pr.v) - kr;
+                    valid = true;
                 }
             }
             uint8_t* sK = sKV + s * 2 * Sh::KVB;
             uint8_t* sV = sK + Sh::KVB;
-            // one 16-byte chunk per lane: eight lanes per half row, four half rows per pass
+            // one 16-byte chunk of K and of V per lane and pass: eight lanes per half row,
+            // four half rows per pass
 #pragma unroll
             for (int it = 0; it < NH * 8; ++it) {
                 const int q = it * 32 + lane, c = q & 7, kh = q >> 3;
                 const int kl = NH == 2 ? kh >> 1 : kh, hf = NH == 2 ? (kh & 1) : 0;
                 const unsigned long long kq = __shfl_sync(0xffffffffu, kr, kl);
-                const unsigned long long vq = __shfl_sync(0xffffffffu, vr, kl);
+                const unsigned long long dq = __shfl_sync(0xffffffffu, dv, kl);
+                const bool vq = __shfl_sync(0xffffffffu, valid ? 1 : 0, kl) != 0;
                 const uint32_t off = hf * HB + umma::sw128_off(kb + kl, c);
-                if (kq != 0ull) {
-                    umma::cp_async16(sK + off, reinterpret_cast<const bf16*>(kq) + 64 * hf + 8 * c);
-                    umma::cp_async16(sV + off, reinterpret_cast<const bf16*>(vq) + 64 * hf + 8 * c);
-                } else {
-                    ws_st4(sK + off, 0u, 0u, 0u, 0u);
-                    ws_st4(sV + off, 0u, 0u, 0u, 0u);
-                }
+                const bf16* ks = reinterpret_cast<const bf16*>(kq) + 64 * hf + 8 * c;
+                umma::cp_async16_zfill(sK + off, ks, vq);
+                umma::cp_async16_zfill(sV + off, vq ? reinterpret_cast<const bf16*>(kq + dq) + 64 * hf + 8 * c : ks, vq);
             }
             umma::cp_async_commit();
             if (j >= 1) {
                 umma::cp_async_wait<1>();
                 __syncwarp();
-                convert_v((j - 1) % NST);
+                landed((j - 1) % NST);
             }
         }
         if (ntiles > 0) {
             umma::cp_async_wait<0>();
             __syncwarp();
-            convert_v((ntiles - 1) % NST);
+            landed((ntiles - 1) % NST);
         }
     } else if (wg == 2) {
         // ---- MMA issuer ----
@@ -395,6 +383,7 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                     ++js;
                     progress = true;
                 }
+                // (tile B's P V follows tile A's, whose P barrier also covers V in f16)
                 if (jp < js && umma::mbar_test_wait(&mbar[kPFull + tp], jp & 1)) {
                     umma::fence_after_sync();
                     const int sj = jp % NST;
@@ -440,26 +429,31 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             // m <= qi: key i of tile j is visible iff j KT + i < lim
             const int lim = row_ok ? min(N, n_g + n_w + (qpos - t0) + 1) - j * KT : 0;
             float mx = -INFINITY;
+            if (lim >= KT) {
 #pragma unroll
-            for (int i = 0; i < KT; ++i) {
-                sv[i] = i < lim ? sv[i] * c2 : -INFINITY;
-                mx = fmaxf(mx, sv[i]);
+                for (int i = 0; i < KT; ++i) mx = fmaxf(mx, sv[i]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < KT; ++i) {
+                    sv[i] = i < lim ? sv[i] : -INFINITY;
+                    mx = fmaxf(mx, sv[i]);
+                }
             }
+            mx *= c2;                                             // scores in the log2 domain (c2 > 0)
             float factor = 1.f;
             bool rescale = false;
             if (mx != -INFINITY) {
                 if (l == 0.f) m_ref = mx;                         // nothing accumulated yet
                 else if (mx > m_ref + 8.f) { factor = ws_ex2(m_ref - mx); rescale = true; m_ref = mx; }
             }
-            // weights P (f16); the normaliser sums the f16-rounded weights that the P V
-            // product uses
+            // weights P (f16) for the product; the normaliser sums them before rounding
             uint32_t pw[KT / 2];
             float rs = 0.f;
 #pragma unroll
             for (int u = 0; u < KT / 2; ++u) {
-                pw[u] = ws_pack_f16(ws_ex2(sv[2 * u] - m_ref), ws_ex2(sv[2 * u + 1] - m_ref));
-                const float2 r2 = ws_unpack_f16(pw[u]);
-                rs += r2.x + r2.y;
+                const float e0 = ws_ex2(fmaf(sv[2 * u], c2, -m_ref)), e1 = ws_ex2(fmaf(sv[2 * u + 1], c2, -m_ref));
+                pw[u] = ws_pack_f16(e0, e1);
+                rs += e0 + e1;
             }
             // P(j) over S(j): the tensor cores finished P V (j - 2), which read this buffer,
             // before S(j), whose scores were just read
@@ -489,6 +483,23 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                         umma::tmem_st16(tmem + lane_off + Sh::TO + t * Sh::OT + c0 + i, *reinterpret_cast<float(*)[16]>(r64 + i));
                 }
                 umma::tmem_wait_st();
+            }
+            if (t == 0) {
+                // V of this stage (bf16; landed before S(j) was issued, the wait only makes that
+                // visible to these threads) to f16 in place, 16-byte chunks spread over the
+                // tile's threads; P V (j) waits for this barrier
+                ok = ws_wait(&mbar[kKvFull + j % NST], (j / NST) & 1, abort_flag);
+                dead |= !__all_sync(0xffffffffu, ok);
+                if (dead) break;
+                constexpr int NCV = KT * DIM / 8;                 // 16-byte chunks of the V tile
+                uint8_t* sV = sKV + (j % NST) * 2 * Sh::KVB + Sh::KVB;
+#pragma unroll
+                for (int u = 0; u < NCV / ROWS; ++u) {
+                    uint4* pv = reinterpret_cast<uint4*>(sV + (u * ROWS + r) * 16);
+                    const uint4 x = *pv;
+                    *pv = make_uint4(ws_bf2_to_h2(x.x), ws_bf2_to_h2(x.y), ws_bf2_to_h2(x.z), ws_bf2_to_h2(x.w));
+                }
+                umma::fence_async_smem();
             }
             umma::tmem_wait_st();
             l += rs;

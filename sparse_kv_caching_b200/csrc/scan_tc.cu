@@ -51,12 +51,13 @@ constexpr int kTcMmaWarp = 8;    // warp 8: issues the SRE products
 constexpr int kTcThreads = kTcCompute + 32;
 constexpr uint32_t kTcComputeBar = 1;   // named barrier of the compute warps
 constexpr int kTcTN = 64;        // candidates per SRE tile (N of the SRE product)
-constexpr int kTcFK = 64;        // folded pairs per fold product (K)
+constexpr int kTcFK = 64;        // folded pairs per fold product (K), f32 inputs
+constexpr int kTcFKB = 128;      // the same for bf16 inputs (one product per block at C <= 128)
 constexpr int kTcMinSmem = 170 * 1024;   // one chain CTA per SM: its tensor memory is not shared
 
 struct TcOffsets {               // byte offsets in dynamic shared memory
     int raw, lo, dpart, inv, vptr;   // SRE ring: raw[3] phi tiles, lo[2], den partials[3], 1/den[3], value rows[4]
-    int fa, fb, fphi, fv;            // fold operands and staged rows (alias the SRE ring)
+    int fa, fb, fphi, fv, fpsum;     // fold operands, staged rows, column partial sums (alias the SRE ring)
     int score, xsc, cand_pos, keep, eq_list, fold_e, flags, ranks, slot_pos, free_slots, hist, tmp, part, ss, mbar,
         tptr;
     int total;
@@ -70,13 +71,23 @@ __host__ __device__ inline TcOffsets tc_offsets(int D, int DV, int esize, int la
     o.raw = take(3 * TN * D * 4, 1024);        // 128-byte swizzled tiles: 1024-byte aligned
     o.lo = take(2 * TN * D * 4, 1024);
     const int ring = p;
-    // fold: A = value parts [3][128 / 8 chunks][FK rows][16 B], B = phi parts [3][D / 8][FK][16 B],
-    // then the folded rows as loaded (phi [FK][D] f32, values [FK][DV])
+    // fold: A = value parts [AP][128 / 8 chunks][FK rows][16 B], B = phi parts [3][D / 8][FK][16 B];
+    // f32 inputs stage the folded rows as loaded (phi [FK][D] f32, values [FK][DV]); bf16 inputs
+    // copy the values straight into A and split phi from global memory, keeping per row range
+    // column sums of phi [256 / (D / 8)][D] f32
     p = 0;
-    o.fa = take(3 * FK * 128 * 2, 128);
-    o.fb = take(3 * FK * D * 2, 128);
-    o.fphi = take(FK * D * 4, 128);
-    o.fv = take(FK * DV * esize, 128);
+    if (esize == 4) {
+        o.fa = take(3 * FK * 128 * 2, 128);
+        o.fb = take(3 * FK * D * 2, 128);
+        o.fphi = take(FK * D * 4, 128);
+        o.fv = take(FK * DV * esize, 128);
+        o.fpsum = 0;
+    } else {
+        o.fa = take(kTcFKB * 128 * 2, 128);
+        o.fb = take(3 * kTcFKB * D * 2, 128);
+        o.fphi = o.fv = 0;
+        o.fpsum = take(8 * 256 * 4, 16);
+    }
     p = ring > p ? ring : p;
     o.dpart = take(3 * 4 * TN * 4, 16);
     o.inv = take(3 * TN * 4, 16);
@@ -278,13 +289,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
             uint8_t* base = raw_tile(i % 3);
             const int r = tid / 4, e = t * TN + r;
             unsigned long long src = 0ull;
-            const TIn* vrow = nullptr;
-            if (e < n) {
-                const PairRef<TIn> pr = pair_ref<TIn>(a, st, b, g, cand_pos[e], e);
-                src = reinterpret_cast<unsigned long long>(pr.phik);
-                vrow = pr.v;
-            }
-            if ((tid & 3) == 0) vptr[(i % 4) * TN + r] = vrow;
+            // rows past n: zero phi, and the value row of candidate 0 (a valid address, so
+            // that the value loads need no test; those scores are never stored)
+            const PairRef<TIn> pr = pair_ref<TIn>(a, st, b, g, cand_pos[e < n ? e : 0], e < n ? e : 0);
+            if (e < n) src = reinterpret_cast<unsigned long long>(pr.phik);
+            if ((tid & 3) == 0) vptr[(i % 4) * TN + r] = pr.v;
             const int c = lane & 7;
 #pragma unroll
             for (int u = 0; u < D / 16; ++u) {                // D / 4 chunks x 8 rows / 32 lanes
@@ -410,11 +419,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
             // tile ahead of the epilogue that needs them
             auto load_values = [&](int i, TIn (&v)[32]) {
                 const TIn* const* vp = vptr + (i % 4) * TN + 32 * half;
-                const TIn zero = TIn(0.f);
+                if (32 * quarter < DV) {                      // warp-uniform
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const TIn* row = vp[k];
-                    v[k] = (row != nullptr && crow < DV) ? row[crow] : zero;
+                    for (int k = 0; k < 32; ++k) v[k] = vp[k][crow];
                 }
             };
             TIn vcur[32], vnext[32];
@@ -474,7 +481,98 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     // The folded rows are staged with cp.async (phi [FK][D] f32, values [FK][DV]), then
     // split into MN-major bf16 operand parts: A part p = value row k, columns c, at
     // (c/8)(FK 16) + 16 k; B part p = phi row k, columns j, at (j/8)(FK 16) + 16 k.
-    auto fold = [&](int nf) {
+    // bf16 inputs: up to kTcFKB folded pairs per product.  The value rows go straight into
+    // the A operand (bf16 is exact: one part); thread (j8, rr) of the compute warps reads
+    // columns 8 j8 .. 8 j8 + 7 of rows rr RPT .. rr RPT + RPT - 1 of phi from global memory,
+    // splits them into the three B parts and keeps the column sums of its rows; s then adds
+    // the row ranges' sums in range order.
+    auto fold_b16 = [&](int nf) {
+        constexpr int FKB = kTcFKB, J8 = D / 8, RR = kTcCompute / J8, RPT = FKB / RR;
+        static_assert(RR * J8 == kTcCompute && RPT * RR == FKB, "fold tiling");
+        uint8_t* fa = smem + o.fa;
+        uint8_t* fb = smem + o.fb;
+        float* psum = reinterpret_cast<float*>(smem + o.fpsum);
+        for (int f0 = 0; f0 < nf; f0 += FKB) {
+            const int nff = min(FKB, nf - f0), nk = (nff + 15) & ~15;
+            for (int idx = tid; idx < nk * (M / 8); idx += NT) {
+                const int k = idx / (M / 8), c8 = idx % (M / 8);
+                uint8_t* dst = fa + c8 * (FKB * 16) + k * 16;
+                if (k < nff && 8 * c8 < DV) {
+                    const int e = fold_e[f0 + k];
+                    umma::cp_async16(dst, pair_ref<TIn>(a, st, b, g, cand_pos[e], e).v + 8 * c8);
+                } else {
+                    st_shared_zero16(dst);
+                }
+            }
+            umma::cp_async_commit();
+            if (compute) {
+                const int j8 = tid % J8, rr = tid / J8;
+                float cs[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) cs[i] = 0.f;
+#pragma unroll 2
+                for (int u = 0; u < RPT; ++u) {
+                    const int k = rr * RPT + u;
+                    if (k >= nk) break;
+                    uint32_t w0[4] = {0u, 0u, 0u, 0u}, w1[4] = {0u, 0u, 0u, 0u}, w2[4] = {0u, 0u, 0u, 0u};
+                    if (k < nff) {
+                        const int e = fold_e[f0 + k];
+                        const float* src = pair_ref<TIn>(a, st, b, g, cand_pos[e], e).phik + 8 * j8;
+                        const float4 xa = *reinterpret_cast<const float4*>(src);
+                        const float4 xb4 = *reinterpret_cast<const float4*>(src + 4);
+                        const float xs[8] = {xa.x, xa.y, xa.z, xa.w, xb4.x, xb4.y, xb4.z, xb4.w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) cs[i] += xs[i];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint16_t p0, p1, p2, q0, q1, q2;
+                            split3_bf16(xs[2 * q], p0, p1, p2);
+                            split3_bf16(xs[2 * q + 1], q0, q1, q2);
+                            w0[q] = (uint32_t)p0 | ((uint32_t)q0 << 16);
+                            w1[q] = (uint32_t)p1 | ((uint32_t)q1 << 16);
+                            w2[q] = (uint32_t)p2 | ((uint32_t)q2 << 16);
+                        }
+                    }
+                    const int off = j8 * (FKB * 16) + k * 16;
+                    *reinterpret_cast<uint4*>(fb + off) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+                    *reinterpret_cast<uint4*>(fb + FKB * D * 2 + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+                    *reinterpret_cast<uint4*>(fb + 2 * FKB * D * 2 + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) psum[rr * D + 8 * j8 + i] = cs[i];
+            }
+            umma::cp_async_wait<0>();
+            __syncthreads();
+            for (int j = tid; j < D; j += NT) {
+                float acc = 0.f;
+                for (int q = 0; q < RR; ++q) acc += psum[q * D + j];
+                ss[j] += acc;
+            }
+            umma::fence_async_smem();
+            umma::fence_before_sync();
+            __syncthreads();
+            umma::fence_after_sync();
+            if (tid == 0 && !failed) {
+                const uint32_t id = umma::idesc(umma::kBF16, M, D, true, true);
+                const uint32_t A0 = umma::smem_addr(fa), B0 = umma::smem_addr(fb);
+                constexpr uint32_t PB = FKB * D * 2;                      // bytes between phi parts
+                const uint64_t a0 = umma::sdesc(A0, 128, FKB * 16), b0 = umma::sdesc(B0, 128, FKB * 16);
+#pragma unroll
+                for (int ks = 0; ks < FKB / 16; ++ks) {
+                    if (ks * 16 >= nk) break;
+                    // a K step of 16 moves the start by 256 bytes; the phi parts are PB bytes apart
+                    const uint64_t da = a0 + (uint64_t)((ks * 256) >> 4);
+                    umma::mma_bf16(tmem + cH, da, b0 + (uint64_t)((ks * 256) >> 4), id, 1u);
+                    umma::mma_bf16(tmem + cH, da, b0 + (uint64_t)((PB + ks * 256) >> 4), id, 1u);
+                    umma::mma_bf16(tmem + cH, da, b0 + (uint64_t)((2 * PB + ks * 256) >> 4), id, 1u);
+                }
+                umma::commit(&mbar[2]);
+            }
+            wait_mma(2);                                      // the operands may be overwritten now
+        }
+    };
+
+    auto fold_f32 = [&](int nf) {
         uint8_t* fa = smem + o.fa;
         uint8_t* fb = smem + o.fb;
         const float* fphi = reinterpret_cast<const float*>(smem + o.fphi);
@@ -582,6 +680,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
                 umma::commit(&mbar[2]);
             }
             wait_mma(2);                                      // the operands may be overwritten now
+        }
+    };
+
+    auto fold = [&](int nf) {
+        if constexpr (!F32IN) {
+            fold_b16(nf);
+        } else {
+            fold_f32(nf);
         }
         // refresh the tf32 split of H^T
         for (int j0 = half * (D / 2); compute && j0 < (half + 1) * (D / 2); j0 += 16) {
