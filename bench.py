@@ -23,6 +23,7 @@ collective), timing is the max over ranks, value = all ranks' tokens / time.
 from __future__ import annotations
 
 import argparse
+from dataclasses import replace
 import hashlib
 import json
 import os
@@ -698,6 +699,10 @@ def main():
     ap.add_argument("--impl", default="lola", choices=["lola", "reference"])
     ap.add_argument("--workload", type=int, default=3)
     ap.add_argument("--extra", default="2,5", help="further prefill workloads reported under 'workloads'")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the headline workload's batch (reduced cases for profiler captures)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override the headline workload's prefill length (a multiple of its chunk)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-next", action="store_true", help="skip the SRE-map, scoring-rule and read-mask legs")
     ap.add_argument("--cpu-streams", type=int, default=None,
@@ -713,7 +718,10 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    w = synth.workload(args.workload)
+    over = {k: v for k, v in (("B", args.batch), ("T", args.tokens)) if v is not None}
+    w = synth.workload(args.workload, **over)
+    if over:
+        w = replace(w, name=w.name + "-reduced-" + "-".join(f"{k}{v}" for k, v in over.items()))
     if args.impl == "reference":
         return run_reference(args, w, rank)
 
