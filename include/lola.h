@@ -266,7 +266,9 @@ long long lola_launch_count(void);
  * with NaN); bit 6: operands in the 128-byte swizzled layout (128-byte rows
  * in 1024-byte atoms of 8 rows; K % 64 == 0 for bf16, K % 32 == 0 for tf32;
  * with bit 0, N % 64 == 0; tf32 takes it for K-major operands only, not with
- * bits 0 or 3).  A, B, C, err are device pointers (C f32 row-major, *err set to
+ * bits 0 or 3); bit 7 (with bit 2): the hi parts of the shared-memory operands
+ * are the raw f32 values, not rounded down to tf32 (the result must equal the
+ * bit-2 result bit for bit if kind::tf32 reads only the top 19 bits).  A, B, C, err are device pointers (C f32 row-major, *err set to
  * 1 if the MMA completion wait gave up).  Requires M = 128, 16 <= N <= 256
  * with N % 16 == 0, K a multiple of 16 (bf16, or A in tensor memory) or 8
  * (tf32), operands that fit in shared memory and at most 512 tensor-memory

@@ -365,7 +365,7 @@ int lola_selftest_umma(int mode, const void* A, const void* B, float* C, int M, 
                        void* stream) {
     if (!A || !B || !C || !err) return fail(LOLA_ERR_INVALID_ARG, "null argument");
     const bool tf32 = mode & 2;
-    if (mode < 0 || mode > 127 || ((mode & 4) && !tf32) || ((mode & 8) && (mode & 16)) ||
+    if (mode < 0 || mode > 255 || ((mode & 4) && !tf32) || ((mode & 128) && !(mode & 4)) || ((mode & 8) && (mode & 16)) ||
         ((mode & 64) && tf32 && (mode & (1 | 8))))
         return fail(LOLA_ERR_INVALID_ARG, "mode=%d", mode);
     if ((mode & 64) && (K % (tf32 ? 32 : 64) || ((mode & 1) && N % 64)))

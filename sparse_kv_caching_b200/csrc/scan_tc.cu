@@ -507,31 +507,42 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
             umma::cp_async_commit();
             if (compute) {
                 const int j8 = tid % J8, rr = tid / J8;
-                float cs[8];
+                // every row's loads in flight before the first split
+                float xs[RPT][8];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) cs[i] = 0.f;
-#pragma unroll 2
                 for (int u = 0; u < RPT; ++u) {
                     const int k = rr * RPT + u;
-                    if (k >= nk) break;
-                    uint32_t w0[4] = {0u, 0u, 0u, 0u}, w1[4] = {0u, 0u, 0u, 0u}, w2[4] = {0u, 0u, 0u, 0u};
                     if (k < nff) {
                         const int e = fold_e[f0 + k];
                         const float* src = pair_ref<TIn>(a, st, b, g, cand_pos[e], e).phik + 8 * j8;
                         const float4 xa = *reinterpret_cast<const float4*>(src);
                         const float4 xb4 = *reinterpret_cast<const float4*>(src + 4);
-                        const float xs[8] = {xa.x, xa.y, xa.z, xa.w, xb4.x, xb4.y, xb4.z, xb4.w};
+                        xs[u][0] = xa.x; xs[u][1] = xa.y; xs[u][2] = xa.z; xs[u][3] = xa.w;
+                        xs[u][4] = xb4.x; xs[u][5] = xb4.y; xs[u][6] = xb4.z; xs[u][7] = xb4.w;
+                    } else {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) cs[i] += xs[i];
+                        for (int i = 0; i < 8; ++i) xs[u][i] = 0.f;
+                    }
+                }
+                float cs[8];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint16_t p0, p1, p2, q0, q1, q2;
-                            split3_bf16(xs[2 * q], p0, p1, p2);
-                            split3_bf16(xs[2 * q + 1], q0, q1, q2);
-                            w0[q] = (uint32_t)p0 | ((uint32_t)q0 << 16);
-                            w1[q] = (uint32_t)p1 | ((uint32_t)q1 << 16);
-                            w2[q] = (uint32_t)p2 | ((uint32_t)q2 << 16);
-                        }
+                for (int i = 0; i < 8; ++i) cs[i] = 0.f;
+#pragma unroll
+                for (int u = 0; u < RPT; ++u) {
+                    const int k = rr * RPT + u;
+                    if (k >= nk) break;
+                    // zero rows (k >= nff) split into zero parts
+                    uint32_t w0[4], w1[4], w2[4];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) cs[i] += xs[u][i];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint16_t p0, p1, p2, q0, q1, q2;
+                        split3_bf16(xs[u][2 * q], p0, p1, p2);
+                        split3_bf16(xs[u][2 * q + 1], q0, q1, q2);
+                        w0[q] = (uint32_t)p0 | ((uint32_t)q0 << 16);
+                        w1[q] = (uint32_t)p1 | ((uint32_t)q1 << 16);
+                        w2[q] = (uint32_t)p2 | ((uint32_t)q2 << 16);
                     }
                     const int off = j8 * (FKB * 16) + k * 16;
                     *reinterpret_cast<uint4*>(fb + off) = make_uint4(w0[0], w0[1], w0[2], w0[3]);

@@ -11,7 +11,9 @@
 // bounded-wait failure path: *err is set, C is filled with NaN, the kernel
 // frees its tensor memory and returns); bit 6 = operands in the 128-byte
 // swizzled layout (128-byte rows, 8-row atoms) instead of chunk-major (tf32:
-// K-major operands only).
+// K-major operands only); bit 7 = with bit 2, the hi parts in shared memory are
+// the raw f32 values (not rounded down to tf32 first), to check that kind::tf32
+// reads only their top 19 bits.
 #include "device_common.cuh"
 #include "umma.cuh"
 
@@ -76,6 +78,7 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
     const bool bmn = a.mode & 1, tf32 = a.mode & 2, x3 = (a.mode & 4) && tf32;
     const bool amn = a.mode & 8, ats = a.mode & 16, expire = a.mode & 32;
     const bool sw = a.mode & 64;
+    const bool rawhi = (a.mode & 128) && x3;                  // hi parts as raw f32
     const int M = a.M, N = a.N, K = a.K;
     const int es = tf32 ? 4 : 2;
     const size_t szA = (size_t)M * K * es, szB = (size_t)N * K * es;
@@ -90,16 +93,16 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
         const float* B = (const float*)a.B;
         if (sw) {    // K-major operands only
             if (!ats) {
-                fill_sw128<float>(sA, A, M, K, false, x3);
+                fill_sw128<float>(sA, A, M, K, false, x3 && !rawhi);
                 if (x3) fill_sw128<float>(sA2, A, M, K, true, false);
             }
-            fill_sw128<float>(sB, B, N, K, false, x3);
+            fill_sw128<float>(sB, B, N, K, false, x3 && !rawhi);
             if (x3) fill_sw128<float>(sB2, B, N, K, true, false);
         } else if (amn) {   // A given as [K][M]: rows = K, chunks along M
             fill_chunk_major<float>(sA, A, K, M, false, x3);
             if (x3) fill_chunk_major<float>(sA2, A, K, M, true, false);
         } else if (!ats) {
-            fill_chunk_major<float>(sA, A, M, K, false, x3);
+            fill_chunk_major<float>(sA, A, M, K, false, x3 && !rawhi);
             if (x3) fill_chunk_major<float>(sA2, A, M, K, true, false);
         }
         if (sw) {
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(128, 1) umma_selftest_kernel(SelftestArgs a) {
             fill_chunk_major<float>(sB, B, K, N, false, x3);
             if (x3) fill_chunk_major<float>(sB2, B, K, N, true, false);
         } else {
-            fill_chunk_major<float>(sB, B, N, K, false, x3);
+            fill_chunk_major<float>(sB, B, N, K, false, x3 && !rawhi);
             if (x3) fill_chunk_major<float>(sB2, B, N, K, true, false);
         }
     } else if (sw) {

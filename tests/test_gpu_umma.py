@@ -86,6 +86,17 @@ def test_tf32_swizzled(mode, N, K):
     assert (C - ref).abs().max() / ref.abs().max() < tol
 
 
+# kind::tf32 reads the top 19 bits of an f32 operand: 3xTF32 with the hi parts
+# passed raw equals 3xTF32 with them rounded down first, bit for bit (the
+# chain's SRE hands its raw phi tile to the tensor cores as the hi part)
+@pytest.mark.parametrize("mode", [6, 22, 70, 86])
+@pytest.mark.parametrize("N,K", [(64, 128), (128, 64)])
+def test_tf32_reads_the_top_19_bits(mode, N, K):
+    C0, _ = _run(mode, N, K, seed=3)
+    C1, _ = _run(mode | 128, N, K, seed=3)
+    assert torch.equal(C0, C1)
+
+
 # tf32 operands are used K-major only (the MN-major tf32 form is not used by
 # the library and is not tested).
 @pytest.mark.parametrize("mode", [2])
