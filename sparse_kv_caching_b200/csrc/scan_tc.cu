@@ -20,7 +20,8 @@
 //     among the compute warps, mbarriers between them and the issuing warp).
 //     For a tile of 64 candidates, P^T = H^T Phi^T is three tf32 MMAs
 //     with A = H_hi / H_lo read from tensor memory and B = Phi_hi / Phi_lo
-//     (the candidates' phi rows, split the same way) in shared memory, in the
+//     (the candidates' phi rows as loaded, which the tensor cores read to tf32,
+//     and their remainders) in shared memory, in the
 //     128-byte swizzled layout (each 128-byte piece of a phi row is one
 //     shared-memory row, so a warp's copies touch few lines and rows):
 //     P = H_hi Phi_hi + H_lo Phi_hi + H_hi Phi_lo, f32-accurate products
@@ -306,8 +307,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
         }
         umma::cp_async_commit();
     };
-    // tf32 split of raw[i % 3] in place (Phi_hi) and into lo[i % 2] (Phi_lo); partial
-    // den_e = phi_e . s over a quarter of the chunks (thread (r, q): chunks q, q+4, ...)
+    // tf32 split: the raw tile in raw[i % 3] serves as Phi_hi as it is (kind::tf32 reads the
+    // top 19 bits of each f32), Phi_lo = phi - hi goes to lo[i % 2]; partial den_e = phi_e . s
+    // over a quarter of the chunks (thread (r, q): chunks q, q+4, ...)
     auto prep = [&](int i) {
         float* phi = reinterpret_cast<float*>(raw_tile(i % 3));
         float* plo = reinterpret_cast<float*>(lo_tile(i & 1));
@@ -316,13 +318,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
         float d0 = 0.f, d1 = 0.f;
         for (int jc = q; jc < D / 4; jc += kTcCompute / TN) {
             const int off = ((jc >> 3) * (TN * 128) + (int)umma::sw128_off(r, jc & 7)) / 4;
-            float4* p = reinterpret_cast<float4*>(phi + off);
-            const float4 x = *p;
+            const float4 x = *reinterpret_cast<const float4*>(phi + off);
             const float4 s4 = *reinterpret_cast<const float4*>(ss + 4 * jc);
             d0 = fmaf(x.x, s4.x, d0); d1 = fmaf(x.y, s4.y, d1);
             d0 = fmaf(x.z, s4.z, d0); d1 = fmaf(x.w, s4.w, d1);
             const float4 h = make_float4(umma::tf32_hi(x.x), umma::tf32_hi(x.y), umma::tf32_hi(x.z), umma::tf32_hi(x.w));
-            *p = h;
             *reinterpret_cast<float4*>(plo + off) = make_float4(x.x - h.x, x.y - h.y, x.z - h.z, x.w - h.w);
         }
         dp[q * TN + r] = d0 + d1;
