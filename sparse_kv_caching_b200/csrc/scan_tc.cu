@@ -14,10 +14,11 @@
 //   * H^T lives in tensor memory for the whole launch: lane c holds column c
 //     of H (rows c >= d are zero), one f32 per TMEM column j < D.  Beside it
 //     the launch keeps H_hi = H rounded down to tf32 and H_lo = H - H_hi.
-//   * SRE, warp-specialised: the compute warps copy a tile's phi rows, split
-//     them and hand the tile to a ninth warp that issues its products, then
-//     take the scores of the previous tile while those run (named barriers
-//     among the compute warps, mbarriers between them and the issuing warp).
+//   * SRE, warp-specialised: a loader warp copies each tile's phi rows (three
+//     tiles ahead), the compute warps split them and hand the tile to an
+//     issuing warp, then take the scores of the previous tile while its
+//     products run (named barriers among the compute warps, mbarriers between
+//     the roles).
 //     For a tile of 64 candidates, P^T = H^T Phi^T is three tf32 MMAs
 //     with A = H_hi / H_lo read from tensor memory and B = Phi_hi / Phi_lo
 //     (the candidates' phi rows as loaded, which the tensor cores read to tf32,
@@ -49,7 +50,8 @@ namespace lola {
 
 constexpr int kTcCompute = 256;  // warps 0-7: loads, tf32 split, epilogue, selection, fold
 constexpr int kTcMmaWarp = 8;    // warp 8: issues the SRE products
-constexpr int kTcThreads = kTcCompute + 32;
+constexpr int kTcLoadWarp = 9;   // warp 9: copies the SRE tiles' phi rows
+constexpr int kTcThreads = kTcCompute + 64;
 constexpr uint32_t kTcComputeBar = 1;   // named barrier of the compute warps
 constexpr int kTcTN = 64;        // candidates per SRE tile (N of the SRE product)
 constexpr int kTcFK = 64;        // folded pairs per fold product (K), f32 inputs
@@ -108,7 +110,7 @@ __host__ __device__ inline TcOffsets tc_offsets(int D, int DV, int esize, int la
     o.tmp = take(32 * 4, 16);
     o.part = take(4 * TN * 4, 16);
     o.ss = take(D * 4, 16);
-    o.mbar = take(8 * 8, 8);
+    o.mbar = take(16 * 8, 8);
     o.tptr = take(16, 16);
     o.total = p;
     return o;
@@ -171,13 +173,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     float* part = reinterpret_cast<float*>(smem + o.part);
     float* ss = reinterpret_cast<float*>(smem + o.ss);
     // [0], [1]: SRE products of tiles i % 2 done; [2]: fold products done; [3], [4]: tile i % 2
-    // split and ready for its products
+    // split and ready for its products; [5 + i % 3]: tile i's phi rows and value pointers in;
+    // [8 + i % 3]: tile i's products done (its raw buffer free again)
     uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + o.mbar);
     uint32_t* tptr = reinterpret_cast<uint32_t*>(smem + o.tptr);
 
     if (warp == 0) umma::tmem_alloc(tptr, TCOLS);
     if (tid == 0) {
         for (int i = 0; i < 5; ++i) umma::mbar_init(&mbar[i], 1);
+        for (int i = 5; i < 8; ++i) umma::mbar_init(&mbar[i], 33);   // 32 copy arrivals + the pointers
+        for (int i = 8; i < 11; ++i) umma::mbar_init(&mbar[i], 1);
         umma::fence_mbar_init();
     }
     const size_t snaps = (size_t)dm.nc_max + 1;
@@ -279,33 +284,48 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     const TIn** vptr = reinterpret_cast<const TIn**>(smem + o.vptr);
     auto raw_tile = [&](int s3) { return smem + o.raw + s3 * (TN * D * 4); };
     auto lo_tile = [&](int lb) { return smem + o.lo + lb * (TN * D * 4); };
-    // cp.async the phi rows of tile t (slot i of this CTA's tiles) into raw[i % 3]; rows
-    // past n are zero; the value-row pointers go to vptr[i % 4].  Always commits a group.
-    static_assert(kTcCompute == 4 * TN, "four compute threads per candidate row");
-    auto issue_loads = [&](int t, int i, int n) {
-        if (t >= 0) {
-            // thread 4 r + q looks up row r of the tile (warp w: rows 8 w .. 8 w + 7); the warp
-            // then copies its eight rows with eight lanes per 128-byte piece (one global line,
-            // one shared row), the row's address taken from the lane that looked it up
-            uint8_t* base = raw_tile(i % 3);
-            const int r = tid / 4, e = t * TN + r;
-            unsigned long long src = 0ull;
-            // rows past n: zero phi, and the value row of candidate 0 (a valid address, so
-            // that the value loads need no test; those scores are never stored)
-            const PairRef<TIn> pr = pair_ref<TIn>(a, st, b, g, cand_pos[e < n ? e : 0], e < n ? e : 0);
-            if (e < n) src = reinterpret_cast<unsigned long long>(pr.phik);
-            if ((tid & 3) == 0) vptr[(i % 4) * TN + r] = pr.v;
-            const int c = lane & 7;
+    // The loader warp: the phi rows of tile t (slot i of this CTA's tiles) into raw[i % 3]
+    // (rows past n zero-filled), the value-row pointers into vptr[i % 4] (rows past n: the
+    // value row of candidate 0, a valid address, so that the value loads need no test; those
+    // scores are never stored).  Lane l looks up rows l and l + 32; eight lanes copy each
+    // 128-byte piece of a row (one global line, one shared row).  Every lane's copies arrive
+    // on mbar[5 + i % 3] as they land, lane 0 once more after the pointers.
+    auto load_tile = [&](int t, int i, int n) {
+        uint8_t* base = raw_tile(i % 3);
+        const int e0 = t * TN + lane, e1 = e0 + 32;
+        const PairRef<TIn> p0 = pair_ref<TIn>(a, st, b, g, cand_pos[e0 < n ? e0 : 0], e0 < n ? e0 : 0);
+        const PairRef<TIn> p1 = pair_ref<TIn>(a, st, b, g, cand_pos[e1 < n ? e1 : 0], e1 < n ? e1 : 0);
+        const unsigned long long s0 = e0 < n ? reinterpret_cast<unsigned long long>(p0.phik) : 0ull;
+        const unsigned long long s1 = e1 < n ? reinterpret_cast<unsigned long long>(p1.phik) : 0ull;
+        vptr[(i % 4) * TN + lane] = p0.v;
+        vptr[(i % 4) * TN + 32 + lane] = p1.v;
+        const int c = lane & 7;
+        const float* dummy = a.sp.H;                          // placeholder source of zero fills
+#pragma unroll 4
+        for (int rg = 0; rg < TN / 4; ++rg) {
+            const int row = 4 * rg + (lane >> 3);
+            const unsigned long long p = __shfl_sync(0xffffffffu, rg < 8 ? s0 : s1, row & 31);
 #pragma unroll
-            for (int u = 0; u < D / 16; ++u) {                // D / 4 chunks x 8 rows / 32 lanes
-                const int rr = 4 * (u & 1) + (lane >> 3), kb = u >> 1, row = 8 * warp + rr;
-                const unsigned long long p = __shfl_sync(0xffffffffu, src, 4 * rr);
+            for (int kb = 0; kb < D / 32; ++kb) {
                 uint8_t* dst = base + kb * (TN * 128) + umma::sw128_off(row, c);
-                if (p != 0ull) umma::cp_async16(dst, reinterpret_cast<const float*>(p) + 32 * kb + 4 * c);
-                else st_shared_zero16(dst);
+                umma::cp_async16_zfill(dst, p != 0ull ? reinterpret_cast<const float*>(p) + 32 * kb + 4 * c : dummy,
+                                       p != 0ull);
             }
         }
-        umma::cp_async_commit();
+        umma::cp_async_arrive_noinc(&mbar[5 + i % 3]);
+        __syncwarp();
+        if (lane == 0) umma::mbar_arrive(&mbar[5 + i % 3]);
+    };
+    // the compute warps' wait for tile i's rows (uniform outcome among them)
+    auto wait_landed = [&](int i) {
+        const int lb = 5 + i % 3;
+        bool ok = true;
+        if (!failed) ok = umma::mbar_wait(&mbar[lb], (phases >> lb) & 1u);
+        phases ^= 1u << lb;
+        if (umma::named_sync_or(kTcComputeBar, kTcCompute, !ok)) {
+            if (!failed && a.err && tid == 0) atomicOr(a.err, 1);
+            failed = true;
+        }
     };
     // tf32 split: the raw tile in raw[i % 3] serves as Phi_hi as it is (kind::tf32 reads the
     // top 19 bits of each f32), Phi_lo = phi - hi goes to lo[i % 2]; partial den_e = phi_e . s
@@ -351,6 +371,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
             umma::mma_tf32_ts(dP, tmem + cHhi + ks * 8, bl0 + step, id, 1u);
         }
         umma::commit(&mbar[pb]);
+        umma::commit(&mbar[8 + i % 3]);
     };
     // score_e of tile t (slot i) -> out[e]: squared residual over this quarter's 32
     // columns (values v from registers, loaded before the MMA wait), summed across the
@@ -400,11 +421,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
         float* out = NCL > 1 ? xsc + xb * NM : score;
         auto tile_of = [&](int i) { return i < mt ? rank + i * NCL : -1; };
         if (mt > 0 && compute) {
-            issue_loads(tile_of(0), 0, n);
-            issue_loads(tile_of(1), 1, n);
-            issue_loads(tile_of(2), 2, n);
-            umma::cp_async_wait<2>();
-            umma::named_sync(kTcComputeBar, kTcCompute);
+            wait_landed(0);
             // split tile i and hand it to the issuing warp (mbar[3 + i % 2])
             auto prep_and_pass = [&](int i) {
                 prep(i);
@@ -429,15 +446,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
             for (int i = 0; i < mt; ++i) {
                 const int t = tile_of(i);
                 if (i + 1 < mt) {
-                    umma::cp_async_wait<1>();                 // tile i + 1 has landed (i + 2 may be in flight)
-                    umma::named_sync(kTcComputeBar, kTcCompute);
+                    wait_landed(i + 1);
                     // lo[(i + 1) % 2] was last read by the products of tile i - 1, waited for
                     prep_and_pass(i + 1);
                     den_final(i + 1);
                     load_values(i + 1, vnext);
                 }
-                wait_mma_c(i & 1);                            // tile i's products; raw[i % 3] is free
-                issue_loads(tile_of(i + 3), i + 3, n);
+                wait_mma_c(i & 1);                            // tile i's products
                 epilogue(t, i, n, out, vcur);
                 umma::fence_before_sync();
 #pragma unroll
@@ -458,6 +473,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
                 umma::fence_after_sync();
                 if (lane == 0 && !failed) issue_sre_mma(i);
                 __syncwarp();
+            }
+        } else if (mt > 0 && warp == kTcLoadWarp) {
+            // tile i's rows once the products of tile i - 3 (same raw buffer) are done; every
+            // tile's completion is waited for once, the last three after the last copy
+            for (int i = 0; i < mt + 3; ++i) {
+                if (i >= 3) {
+                    const int fb = 8 + (i - 3) % 3;
+                    bool ok = true;
+                    if (lane == 0 && !failed) ok = umma::mbar_wait(&mbar[fb], (phases >> fb) & 1u);
+                    phases ^= 1u << fb;
+                    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                    if (!ok) failed = true;                   // made uniform after the block
+                }
+                if (i < mt) load_tile(tile_of(i), i, n);
             }
         }
         if (__syncthreads_or(failed ? 1 : 0)) {

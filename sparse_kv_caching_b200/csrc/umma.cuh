@@ -229,6 +229,11 @@ __device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gme
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                  :: "r"(smem_addr(smem_dst)), "l"(gmem_src), "r"(valid ? 16u : 0u) : "memory");
 }
+// Arrive on an mbarrier once every cp.async this thread issued so far has landed
+// (the arrival counts toward the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* mbar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_addr(mbar)) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
