@@ -283,24 +283,55 @@ __device__ inline int select_place_cta(const float* score, const int* cand_pos, 
         for (int e = tid; e < n; e += NT) keep[e] = 0;
         __syncthreads();
     }
-    // freed slots in slot order (member e sits in slot e)
-    for (int j = tid; j < lam; j += NT) flags[j] = (j >= n_g || keep[j] == 0) ? 1 : 0;
-    __syncthreads();
-    block_exscan(flags, ranks, lam, tmp);
-    for (int j = tid; j < lam; j += NT) if (flags[j]) free_slots[ranks[j]] = j;
-    __syncthreads();
-    // kept newcomers, in position order, take them in order
-    for (int i = tid; i < n_l; i += NT) flags[i] = keep[n_g + i];
-    __syncthreads();
-    block_exscan(flags, ranks, n_l, tmp);
-    for (int i = tid; i < n_l; i += NT) if (flags[i]) slot_pos[free_slots[ranks[i]]] = l_lo + i;
-    __syncthreads();
-    // the folded set S = E \ G_new, in candidate order
-    for (int e = tid; e < n; e += NT) flags[e] = keep[e] ? 0 : 1;
-    __syncthreads();
-    const int nf = block_exscan(flags, ranks, n, tmp);
-    for (int e = tid; e < n; e += NT) if (flags[e]) fold_e[ranks[e]] = e;
-    __syncthreads();
+    int nf = 0;
+    // One block-wide exclusive scan of three packed counts (21 bits each) over x in
+    // [0, max(lam, n)): freed slots in slot order (member e sits in slot e), kept newcomers
+    // in position order, folded candidates in candidate order.  hist (free after the radix
+    // passes) holds the per-warp sums.
+    {
+        auto fa = [&](int x) -> unsigned long long { return (x < lam && (x >= n_g || keep[x] == 0)) ? 1ull : 0ull; };
+        auto fb = [&](int x) -> unsigned long long { return (x < n_l && keep[n_g + x]) ? 1ull : 0ull; };
+        auto fc = [&](int x) -> unsigned long long { return (x < n && keep[x] == 0) ? 1ull : 0ull; };
+        auto fl = [&](int x) { return fa(x) | (fb(x) << 21) | (fc(x) << 42); };
+        constexpr unsigned long long F = (1ull << 21) - 1;
+        unsigned long long* wsum = reinterpret_cast<unsigned long long*>(hist);
+        const int X = max(lam, n), per = (X + NT - 1) / NT;
+        const int lo = min(X, tid * per), hi = min(X, lo + per);
+        const int warp = tid >> 5, NW = NT / 32;
+        unsigned long long sum = 0ull;
+        for (int x = lo; x < hi; ++x) sum += fl(x);
+        unsigned long long incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) wsum[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            unsigned long long w = lane < NW ? wsum[lane] : 0ull;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const unsigned long long y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            if (lane < NW) wsum[lane] = w;
+        }
+        __syncthreads();
+        unsigned long long base = (warp ? wsum[warp - 1] : 0ull) + incl - sum;
+        for (int x = lo; x < hi; ++x) {
+            const unsigned long long f = fl(x);
+            if (f & F) free_slots[(int)(base & F)] = x;
+            if ((f >> 21) & F) ranks[x] = (int)((base >> 21) & F);
+            if (f >> 42) fold_e[(int)(base >> 42)] = x;
+            base += f;
+        }
+        nf = (int)(wsum[NW - 1] >> 42);
+        __syncthreads();
+        // kept newcomers take the freed slots in order
+        for (int i = tid; i < n_l; i += NT) if (keep[n_g + i]) slot_pos[free_slots[ranks[i]]] = l_lo + i;
+        __syncthreads();
+    }
     return nf;
 }
 
