@@ -60,7 +60,8 @@ constexpr int kTcMinSmem = 170 * 1024;   // one chain CTA per SM: its tensor mem
 
 struct TcOffsets {               // byte offsets in dynamic shared memory
     int raw, lo, dpart, inv, vptr;   // SRE ring: raw[3] phi tiles, lo[2], den partials[3], 1/den[3], value rows[4]
-    int fa, fb, fphi, fv, fpsum;     // fold operands, staged rows, column partial sums (alias the SRE ring)
+    int fa, fb, fphi, fv, fpsum, fptr;   // fold operands, staged rows, column partial sums, row addresses
+                                         // (alias the SRE ring)
     int score, xsc, cand_pos, keep, eq_list, fold_e, flags, ranks, slot_pos, free_slots, hist, tmp, part, ss, mbar,
         tptr;
     int total;
@@ -84,12 +85,13 @@ __host__ __device__ inline TcOffsets tc_offsets(int D, int DV, int esize, int la
         o.fb = take(3 * FK * D * 2, 128);
         o.fphi = take(FK * D * 4, 128);
         o.fv = take(FK * DV * esize, 128);
-        o.fpsum = 0;
+        o.fpsum = o.fptr = 0;
     } else {
         o.fa = take(kTcFKB * 128 * 2, 128);
         o.fb = take(3 * kTcFKB * D * 2, 128);
         o.fphi = o.fv = 0;
         o.fpsum = take(8 * 256 * 4, 16);
+        o.fptr = take(2 * kTcFKB * 8, 16);            // phi and value row addresses of the folded rows
     }
     p = ring > p ? ring : p;
     o.dpart = take(3 * 4 * TN * 4, 16);
@@ -521,14 +523,23 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
         uint8_t* fa = smem + o.fa;
         uint8_t* fb = smem + o.fb;
         float* psum = reinterpret_cast<float*>(smem + o.fpsum);
+        // each folded row's phi and value addresses, looked up once
+        const float** prow = reinterpret_cast<const float**>(smem + o.fptr);
+        const TIn** vrow = reinterpret_cast<const TIn**>(smem + o.fptr + FKB * 8);
         for (int f0 = 0; f0 < nf; f0 += FKB) {
             const int nff = min(FKB, nf - f0), nk = (nff + 15) & ~15;
+            for (int k = tid; k < nff; k += NT) {
+                const int e = fold_e[f0 + k];
+                const PairRef<TIn> pr = pair_ref<TIn>(a, st, b, g, cand_pos[e], e);
+                prow[k] = pr.phik;
+                vrow[k] = pr.v;
+            }
+            __syncthreads();
             for (int idx = tid; idx < nk * (M / 8); idx += NT) {
                 const int k = idx / (M / 8), c8 = idx % (M / 8);
                 uint8_t* dst = fa + c8 * (FKB * 16) + k * 16;
                 if (k < nff && 8 * c8 < DV) {
-                    const int e = fold_e[f0 + k];
-                    umma::cp_async16(dst, pair_ref<TIn>(a, st, b, g, cand_pos[e], e).v + 8 * c8);
+                    umma::cp_async16(dst, vrow[k] + 8 * c8);
                 } else {
                     st_shared_zero16(dst);
                 }
@@ -542,8 +553,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
                 for (int u = 0; u < RPT; ++u) {
                     const int k = rr * RPT + u;
                     if (k < nff) {
-                        const int e = fold_e[f0 + k];
-                        const float* src = pair_ref<TIn>(a, st, b, g, cand_pos[e], e).phik + 8 * j8;
+                        const float* src = prow[k] + 8 * j8;
                         const float4 xa = *reinterpret_cast<const float4*>(src);
                         const float4 xb4 = *reinterpret_cast<const float4*>(src + 4);
                         xs[u][0] = xa.x; xs[u][1] = xa.y; xs[u][2] = xa.z; xs[u][3] = xa.w;
