@@ -10,9 +10,9 @@
 // runs one 128-row tile per CTA).  Roles:
 //   warps 0-3 / 4-7  softmax and epilogue of tile A / B (thread r owns row r)
 //   warps 8-9        gather K and V rows of each 64-key tile with cp.async
-//                    into a 4-stage ring (row addresses looked up once per key
-//                    and shared by shuffles, the block's cache positions staged
-//                    in the prologue); tile A's softmax warps turn V into f16
+//                    into a 5-stage ring (row addresses looked up once per key
+//                    and shared by shuffles, each key's cache position read
+//                    one tile ahead); tile A's softmax warps turn V into f16
 //                    in place once their weights are stored
 // K and V tiles sit in the 128-byte swizzled layout: each 128-byte half of a
 // key row is one contiguous shared-memory row (its 16-byte chunks permuted), so
@@ -38,7 +38,7 @@ namespace lola {
 
 template <int DIM, int DH>
 struct WsShape {
-    static constexpr int ROWS = 128, KT = 64, D = 2 * DH, NCH = DIM / 8, NST = 4;
+    static constexpr int ROWS = 128, KT = 64, D = 2 * DH, NCH = DIM / 8, NST = 5;
     static constexpr int NT = 352;                              // 11 warps
     // query tiles per CTA: two 128-row tiles share every gathered key tile for d = 128;
     // one for d = 64 (with two tiles at d = 64 the second tile's scores came out wrong
@@ -48,9 +48,9 @@ struct WsShape {
     static constexpr int KVB = KT * DIM * 2;                    // one K or V tile
     static constexpr int Q = 0;                                 // [2 tiles]
     static constexpr int KV = Q + NTILE * QB;                   // [NST][K, V]
-    static constexpr int MBAR = KV + NST * 2 * KVB;             // 17 barriers
+    static constexpr int MBAR = KV + NST * 2 * KVB;             // 19 barriers
     static constexpr int FLAG = MBAR + 24 * 8;                  // abort flag, tmem pointer
-    static constexpr int CPOS = FLAG + 16;                      // cache positions of the block [lambda] int
+    static constexpr int END = FLAG + 16;
     static constexpr int KPOS = MBAR;                           // (end of the prologue aliases)
     // prologue aliases (the KV and P regions are free until the roles start)
     static constexpr int HT = KV;                               // H_c^T, [D/32][DIM x 32] f32
@@ -66,9 +66,9 @@ struct WsShape {
     static_assert(DIM <= (int)OT && TS + 4 * KT <= 512, "tensor memory");
 };
 
-// barrier indices (four ring stages): K and V landed, stage free; S ready (two buffers
+// barrier indices (five ring stages): K and V landed, stage free; S ready (two buffers
 // per query tile), P ready (for tile A: V in f16 too), P V done (per query tile); prologue
-enum : int { kKvFull = 0, kKvFree = 4, kSFull = 8, kPFull = 12, kPvDone = 14, kPro = 16 };
+enum : int { kKvFull = 0, kKvFree = 5, kSFull = 10, kPFull = 14, kPvDone = 16, kPro = 18 };
 
 // Bounded mbarrier wait that also gives up once another thread of the CTA has
 // raised the abort flag; returns false if it gave up (and raises the flag).
@@ -136,8 +136,8 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
 
     uint8_t* sQ = smem + Sh::Q;
     uint8_t* sKV = smem + Sh::KV;
-    static_assert(NST == 4, "barrier indices assume four stages");
-    int* cpos_s = reinterpret_cast<int*>(smem + Sh::CPOS);
+    static_assert(NST == 5, "barrier indices assume five stages");
+    const int* cpos = a.snap_pos + ((size_t)st * snaps + c) * dm.lam;   // cache positions of the block
     uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + Sh::MBAR);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Sh::FLAG);
     uint32_t* tptr = reinterpret_cast<uint32_t*>(smem + Sh::FLAG + 8);
@@ -167,10 +167,6 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
         } else {
             ws_st4(dst, 0u, 0u, 0u, 0u);
         }
-    }
-    {
-        const int* cpos = a.snap_pos + ((size_t)st * snaps + c) * dm.lam;
-        for (int i = tid; i < n_g; i += NT) cpos_s[i] = cpos[i];
     }
     const float* Hc = a.snap_H + ((size_t)st * snaps + c) * D * DIM;     // H_c^T [DIM][D]
     const float* sc_g = a.snap_s + ((size_t)st * snaps + c) * D;
@@ -284,8 +280,12 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             umma::fence_async_smem();
             umma::mbar_arrive(&mbar[kKvFull + s]);
         };
+        // the cache position of this lane's key, loaded one tile ahead
+        int pos_c = kb + lane < n_g ? cpos[kb + lane] : 0;
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % NST;
+            const int gk_next = (j + 1) * KT + kb + lane;
+            const int pos_n = gk_next < n_g ? cpos[gk_next] : 0;
             if (j >= NST) {
                 bool ok = true;
                 if (lane == 0 && !dead) ok = ws_wait(&mbar[kKvFree + s], ((j / NST) - 1) & 1, abort_flag);
@@ -298,13 +298,14 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             {
                 const int gk = j * KT + kb + lane;
                 if (gk < N && !dead) {
-                    const int pos = gk < n_g ? cpos_s[gk] : (gk < n_g + n_w ? w_lo + (gk - n_g) : t0 + (gk - n_g - n_w));
+                    const int pos = gk < n_g ? pos_c : (gk < n_g + n_w ? w_lo + (gk - n_g) : t0 + (gk - n_g - n_w));
                     const PairRef<bf16> pr = pair_ref<bf16>(a, st, b, g, pos, gk < n_g ? gk : 0);
                     kr = reinterpret_cast<unsigned long long>(pr.k);
                     dv = reinterpret_cast<unsigned long long>(pr.v) - kr;
                     valid = true;
                 }
             }
+            pos_c = pos_n;
             uint8_t* sK = sKV + s * 2 * Sh::KVB;
             uint8_t* sV = sK + Sh::KVB;
             // one 16-byte chunk of K and of V per lane and pass: eight lanes per half row,
@@ -535,7 +536,7 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
 template <int DIM, int DH>
 static cudaError_t launch_ws_t(const PrefillArgs& a, cudaStream_t s) {
     using Sh = WsShape<DIM, DH>;
-    const int bytes = Sh::CPOS + ((a.dm.lam * 4 + 15) & ~15) + 1024;   // + alignment slack
+    const int bytes = Sh::END + 1024;                                  // + alignment slack
     if (bytes > 227 * 1024) return cudaErrorNotSupported;
     cudaError_t e = cudaFuncSetAttribute(output_ws_kernel<DIM, DH>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
