@@ -56,8 +56,9 @@ struct WsShape {
     static constexpr int HT = KV;                               // H_c^T, [D/32][DIM x 32] f32
     static constexpr int HTC = DIM * 32 * 4;
     static constexpr int W = HT + (D / 32) * HTC;               // W [DIM][DH] bf16, MN-major B
-    static constexpr int PHI = W + DIM * DH * 2;                // [2 tiles][128 x 32] f32
-    static constexpr int SC = PHI + NTILE * ROWS * 32 * 4;      // s_c [D] f32
+    static constexpr int PHIS = NTILE * ROWS * 32 * 4;          // one 32-column piece of phi(q), both tiles
+    static constexpr int PHI = W + DIM * DH * 2;                // [2 pieces][2 tiles][128 x 32] f32
+    static constexpr int SC = PHI + 2 * PHIS;                   // s_c [D] f32
     static_assert(SC + D * 4 <= KPOS, "prologue buffers must fit in the KV and P regions");
     // tensor-memory columns
     // O of tile t at column t * OT (each output tile on a 128-column boundary), the four
@@ -178,13 +179,16 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             umma::cp_async16(smem + Sh::W + n8 * DIM * 16 + k * 16, Wg + (size_t)k * DH + 8 * n8);
         }
         for (int idx = tid; idx < D / 4; idx += NT) umma::cp_async16(s_c + 4 * idx, sc_g + 4 * idx);
+    }
+    umma::cp_async_commit();                                   // group: Q, W, s_c
+    if (has_lin) {
         for (int idx = tid; idx < (D / 32) * DIM * 8; idx += NT) {
             const int cc = idx % DIM, jq = (idx / DIM) % 8, ch = idx / (DIM * 8);
             umma::cp_async16(smem + Sh::HT + ch * Sh::HTC + jq * DIM * 16 + cc * 16, Hc + (size_t)cc * D + 32 * ch + 4 * jq);
         }
     }
-    umma::cp_async_commit();
-    umma::cp_async_wait<0>();
+    umma::cp_async_commit();                                   // group: H_c^T (needed after phi(q))
+    umma::cp_async_wait<1>();
     umma::fence_async_smem();
     umma::fence_before_sync();
     __syncthreads();
@@ -196,7 +200,6 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
     const int R = rfirst + wg * ROWS + r;
     const bool row_ok = wg < 2 && R < rows_total;
     const int qpos = t0 + (row_ok ? R % dm.C : 0);
-    const int h = g * dm.Gq + (row_ok ? R / dm.C : 0);
     const bool mma_thread = warp == 10 && lane == 0;
     bool dead = false;
     float l = 0.f;
@@ -216,33 +219,42 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
         dead |= !ws_wait(&mbar[kPro], pro_phase, abort_flag);
         pro_phase ^= 1;
         umma::fence_after_sync();
+        // phi(q) = [softmax(z), softmax(-z)] with z in the log2 domain (exp2 on the XU; the
+        // feature map of the queries reaches y only, within its tolerance)
+        constexpr float kLog2e = 1.4426950408889634f;
         float z[DH];
         float mx = -INFINITY, mn = INFINITY, isp = 0.f, isn = 0.f;
         if (wg < (twoB ? 2 : 1)) {
             ws_tmem_ld<DH>(tmem + lane_off + Sh::TS + 2 * wg * KT, z);
 #pragma unroll
-            for (int i = 0; i < DH; ++i) { mx = fmaxf(mx, z[i]); mn = fminf(mn, z[i]); }
+            for (int i = 0; i < DH; ++i) { z[i] *= kLog2e; mx = fmaxf(mx, z[i]); mn = fminf(mn, z[i]); }
             float sp = 0.f, sn = 0.f;
 #pragma unroll
-            for (int i = 0; i < DH; ++i) { sp += expf(z[i] - mx); sn += expf(mn - z[i]); }
+            for (int i = 0; i < DH; ++i) { sp += ws_ex2(z[i] - mx); sn += ws_ex2(mn - z[i]); }
             isp = 1.f / sp;
             isn = 1.f / sn;
         }
+        umma::cp_async_wait<0>();                              // H_c^T
+        umma::fence_async_smem();
+        // two 32-column pieces of phi(q) per round: store them, then their products
 #pragma unroll
-        for (int jc = 0; jc < D; jc += 32) {
+        for (int j0 = 0; j0 < D; j0 += 64) {
             if (wg < (twoB ? 2 : 1)) {
-                uint8_t* sPhi = smem + Sh::PHI + wg * ROWS * 32 * 4;
 #pragma unroll
-                for (int jq = 0; jq < 8; ++jq) {
-                    float f[4];
+                for (int q = 0; q < 2; ++q) {
+                    uint8_t* sPhi = smem + Sh::PHI + q * Sh::PHIS + wg * ROWS * 32 * 4;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int j = jc + 4 * jq + u;
-                        f[u] = j < DH ? expf(z[j] - mx) * isp : expf(mn - z[j - DH]) * isn;
-                        l = fmaf(f[u], s_c[j], l);
+                    for (int jq = 0; jq < 8; ++jq) {
+                        float f[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int j = j0 + 32 * q + 4 * jq + u;
+                            f[u] = j < DH ? ws_ex2(z[j] - mx) * isp : ws_ex2(mn - z[j - DH]) * isn;
+                            l = fmaf(f[u], s_c[j], l);
+                        }
+                        ws_st4(sPhi + jq * ROWS * 16 + r * 16, __float_as_uint(f[0]), __float_as_uint(f[1]),
+                               __float_as_uint(f[2]), __float_as_uint(f[3]));
                     }
-                    ws_st4(sPhi + jq * ROWS * 16 + r * 16, __float_as_uint(f[0]), __float_as_uint(f[1]),
-                           __float_as_uint(f[2]), __float_as_uint(f[3]));
                 }
             }
             umma::fence_async_smem();
@@ -251,14 +263,18 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             umma::fence_after_sync();
             if (mma_thread && !dead) {
                 const uint32_t id = umma::idesc(umma::kTF32, ROWS, DIM, false, false);
-                const uint8_t* sHt = smem + Sh::HT + (jc / 32) * Sh::HTC;
-                for (int t = 0; t < (twoB ? 2 : 1); ++t)
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma::mma_tf32(tmem + Sh::TO + t * Sh::OT,
-                                       umma::sdesc(umma::smem_addr(smem + Sh::PHI + t * ROWS * 32 * 4) + ks * 2 * ROWS * 16,
-                                                   ROWS * 16, 128),
-                                       umma::sdesc(umma::smem_addr(sHt) + ks * 2 * DIM * 16, DIM * 16, 128), id,
-                                       (jc > 0 || ks > 0) ? 1u : 0u);
+                for (int q = 0; q < 2; ++q) {
+                    const int jc = j0 + 32 * q;
+                    const uint8_t* sHt = smem + Sh::HT + (jc / 32) * Sh::HTC;
+                    for (int t = 0; t < (twoB ? 2 : 1); ++t)
+                        for (int ks = 0; ks < 4; ++ks)
+                            umma::mma_tf32(tmem + Sh::TO + t * Sh::OT,
+                                           umma::sdesc(umma::smem_addr(smem + Sh::PHI + q * Sh::PHIS + t * ROWS * 32 * 4) +
+                                                           ks * 2 * ROWS * 16,
+                                                       ROWS * 16, 128),
+                                           umma::sdesc(umma::smem_addr(sHt) + ks * 2 * DIM * 16, DIM * 16, 128), id,
+                                           (jc > 0 || ks > 0) ? 1u : 0u);
+                }
                 umma::commit(&mbar[kPro]);
             }
             dead |= !ws_wait(&mbar[kPro], pro_phase, abort_flag);
@@ -507,22 +523,35 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             umma::fence_before_sync();
             umma::mbar_arrive(&mbar[kPFull + t]);
         }
-        // ---- epilogue: y = O / l ----
+        // ---- epilogue: y = O / l, staged in the (now free) K/V ring so that whole rows of y
+        // go out in single store instructions ----
         bool ok = !dead && ntiles > 0;
         if (ok) ok = ws_wait(&mbar[kPvDone + t], (ntiles - 1) & 1, abort_flag);
+        if (ok && twoB) ok = ws_wait(&mbar[kPvDone + 1 - t], (ntiles - 1) & 1, abort_flag);   // ring unread
         dead |= !__all_sync(0xffffffffu, ok);
         umma::fence_after_sync();
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        float* yrow = a.y + (((size_t)b * a.T + (qpos - a.t_start)) * dm.Hq + h) * DIM;
+        constexpr int RS = DIM * 4 + 16;                          // padded row: conflict-free staging
+        static_assert(2 * ROWS * RS <= NST * 2 * Sh::KVB, "staging fits in the ring");
+        uint8_t* srow = sKV + (t * ROWS + r) * RS;
 #pragma unroll
         for (int c0 = 0; c0 < DIM; c0 += 64) {
             float r64[64];
             ws_tmem_ld<64>(tmem + lane_off + Sh::TO + t * Sh::OT + c0, r64);
-            if (row_ok && !dead) {
 #pragma unroll
-                for (int i = 0; i < 64; i += 4)
-                    *reinterpret_cast<float4*>(yrow + c0 + i) =
-                        make_float4(r64[i] * inv, r64[i + 1] * inv, r64[i + 2] * inv, r64[i + 3] * inv);
+            for (int i = 0; i < 64; i += 4)
+                ws_st4(srow + (c0 + i) * 4, __float_as_uint(r64[i] * inv), __float_as_uint(r64[i + 1] * inv),
+                       __float_as_uint(r64[i + 2] * inv), __float_as_uint(r64[i + 3] * inv));
+        }
+        const int NR = (twoB ? 2 : 1) * ROWS;                     // rows of this CTA's epilogue threads
+        umma::named_sync(1, NR);
+        constexpr int F4 = DIM / 4;                               // 16-byte pieces of a row
+        for (int idx = tid; idx < NR * F4; idx += NR) {
+            const int row = idx / F4, c4 = idx % F4, Rr = rfirst + row;
+            if (Rr < rows_total && !dead) {
+                const int hr = Rr / dm.C, ir = Rr % dm.C;
+                float* dst = a.y + (((size_t)b * a.T + (t0 + ir - a.t_start)) * dm.Hq + g * dm.Gq + hr) * DIM + 4 * c4;
+                *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(sKV + row * RS + 16 * c4);
             }
         }
     }
