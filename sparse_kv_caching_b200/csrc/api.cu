@@ -59,10 +59,11 @@ thread_local std::string g_err;
 constexpr int kSplitMinChunks = 32;   // calls with fewer chunks run in one segment
 // Relative chunk counts of the chain segments.  The output of segment i runs
 // beside the chain of segment i+1; only the last segment's output is exposed,
-// so the last segment is the shortest (2:2:2:1 measured 0.7 % faster than
-// four equal segments on the 8B-shaped 4096-token prefill; 1:1:1:1, 3:3:3:1,
-// 4:4:4:4:1 and 3:3:3:2:1 were tried).
-constexpr int kSegWeights[] = {2, 2, 2, 1};
+// so the last segment is the shortest.  2:2:2:2:1 measured 1.6 % faster than
+// 2:2:2:1 on the 8B-shaped 16384-token prefill (3 % on the 1B-shaped 32768-token
+// one, 1.3 % slower on the 4096-token one); 3:3:3:1, 1:2:2:2:2:1, 1:1:2:2:2:1
+// and 1:2:3:3:2:1 were slower there.
+constexpr int kSegWeights[] = {2, 2, 2, 2, 1};
 constexpr int kSplitSegments = sizeof(kSegWeights) / sizeof(kSegWeights[0]);
 constexpr int kHostSegments = 4;      // host-buffer prefill: copies overlap compute per segment
 std::atomic<long long> g_launches{0};
