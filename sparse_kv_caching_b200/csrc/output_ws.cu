@@ -156,15 +156,17 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
         umma::fence_mbar_init();
     }
 
-    // ---- prologue: queries of both tiles (row-chunk mapping: 8 rows x 4 chunks per warp) ----
+    // ---- prologue: queries of both tiles, 128-byte swizzled (block kb holds dims
+    // 64 kb .. 64 kb + 63 of every row; eight lanes copy one 128-byte piece) ----
     for (int idx = tid; idx < NTILE * ROWS * NCH; idx += NT) {
-        const int t = idx / (ROWS * NCH), li = idx % (ROWS * NCH);
-        const int r = (li & 7) + 8 * (li / (8 * NCH)), j = (li >> 3) % NCH;
-        uint8_t* dst = sQ + t * Sh::QB + j * ROWS * 16 + r * 16;
+        const int c = idx & 7, kb = (idx >> 3) % (DIM / 64), rt = (idx >> 3) / (DIM / 64);
+        const int r = rt % ROWS, t = rt / ROWS;
+        uint8_t* dst = sQ + t * Sh::QB + kb * (ROWS * 128) + umma::sw128_off(r, c);
         const int R = rfirst + t * ROWS + r;
         if (R < rows_total) {
             const int hr = g * dm.Gq + R / dm.C, ir = R % dm.C;
-            umma::cp_async16(dst, (const bf16*)a.q + (((size_t)b * a.T + (t0 + ir - a.t_start)) * dm.Hq + hr) * DIM + 8 * j);
+            umma::cp_async16(dst, (const bf16*)a.q + (((size_t)b * a.T + (t0 + ir - a.t_start)) * dm.Hq + hr) * DIM +
+                                      64 * kb + 8 * c);
         } else {
             ws_st4(dst, 0u, 0u, 0u, 0u);
         }
@@ -182,9 +184,11 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
     }
     umma::cp_async_commit();                                   // group: Q, W, s_c
     if (has_lin) {
+        // H_c^T piece ch (its columns 32 ch .. 32 ch + 31) as a K-major tf32 operand, 128-byte
+        // swizzled: row cc of the piece is 128 contiguous bytes of H_c^T row cc
         for (int idx = tid; idx < (D / 32) * DIM * 8; idx += NT) {
-            const int cc = idx % DIM, jq = (idx / DIM) % 8, ch = idx / (DIM * 8);
-            umma::cp_async16(smem + Sh::HT + ch * Sh::HTC + jq * DIM * 16 + cc * 16, Hc + (size_t)cc * D + 32 * ch + 4 * jq);
+            const int c = idx & 7, cc = (idx >> 3) % DIM, ch = (idx >> 3) / DIM;
+            umma::cp_async16(smem + Sh::HT + ch * Sh::HTC + umma::sw128_off(cc, c), Hc + (size_t)cc * D + 32 * ch + 4 * c);
         }
     }
     umma::cp_async_commit();                                   // group: H_c^T (needed after phi(q))
@@ -212,7 +216,8 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             for (int t = 0; t < (twoB ? 2 : 1); ++t)
                 for (int ks = 0; ks < DIM / 16; ++ks)
                     umma::mma_bf16(tmem + Sh::TS + 2 * t * KT,
-                                   umma::sdesc(umma::smem_addr(sQ + t * Sh::QB) + ks * 2 * ROWS * 16, ROWS * 16, 128),
+                                   umma::sdesc_sw128(umma::smem_addr(sQ + t * Sh::QB) + (ks >> 2) * ROWS * 128 + (ks & 3) * 32,
+                                                     16, 1024),
                                    umma::sdesc(umma::smem_addr(smem + Sh::W) + ks * 16 * 16, 128, DIM * 16), id, ks > 0);
             umma::commit(&mbar[kPro]);
         }
@@ -272,7 +277,7 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                                            umma::sdesc(umma::smem_addr(smem + Sh::PHI + q * Sh::PHIS + t * ROWS * 32 * 4) +
                                                            ks * 2 * ROWS * 16,
                                                        ROWS * 16, 128),
-                                           umma::sdesc(umma::smem_addr(sHt) + ks * 2 * DIM * 16, DIM * 16, 128), id,
+                                           umma::sdesc_sw128(umma::smem_addr(sHt) + ks * 32, 16, 1024), id,
                                            (jc > 0 || ks > 0) ? 1u : 0u);
                 }
                 umma::commit(&mbar[kPro]);
@@ -356,13 +361,12 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
             const uint32_t idS = umma::idesc(umma::kBF16, ROWS, KT, false, false);
             const uint32_t idO = umma::idesc(umma::kF16, ROWS, DIM, false, true);   // A = P in tensor memory
             const int ntl = twoB ? 2 : 1;
-            // operand descriptors built once (the address field counts 16-byte units).  Q
-            // (chunk-major, K-major): a K step moves the start by two 16-byte chunks of the
-            // tile's rows.  K (swizzled, K-major): 32 bytes inside a 128-byte half row, the next
-            // half KT rows further.  V (swizzled, MN-major): 16 key rows of 128 bytes.  P (tensor
+            // operand descriptors built once (the address field counts 16-byte units).  Q and K
+            // (swizzled, K-major): a K step moves the start by 32 bytes inside a 128-byte half
+            // row, the next half ROWS (KT) rows further.  V (swizzled, MN-major): 16 key rows of 128 bytes.  P (tensor
             // memory, two f16 per column): 8 columns.
-            const uint64_t dQ0 = umma::sdesc(umma::smem_addr(sQ), ROWS * 16, 128);
-            const uint64_t dQ1 = umma::sdesc(umma::smem_addr(sQ + (NTILE - 1) * Sh::QB), ROWS * 16, 128);
+            const uint64_t dQ0 = umma::sdesc_sw128(umma::smem_addr(sQ), 16, 1024);
+            const uint64_t dQ1 = umma::sdesc_sw128(umma::smem_addr(sQ + (NTILE - 1) * Sh::QB), 16, 1024);
             // stage s sits 2 KVB bytes after stage s - 1
             const uint64_t dK0 = umma::sdesc_sw128(umma::smem_addr(sKV), 16, 1024);
             const uint64_t dV0 = umma::sdesc_sw128(umma::smem_addr(sKV + Sh::KVB), KT * 128, 1024);
@@ -372,13 +376,13 @@ __global__ void __launch_bounds__(352, 1) output_ws_kernel(const __grid_constant
                 const uint32_t d0 = tmem + Sh::TS + (j & 1) * KT;
 #pragma unroll
                 for (int ks = 0; ks < DIM / 16; ++ks)
-                    umma::mma_bf16(d0, dQ0 + (uint64_t)(ks * 2 * ROWS), bk + (uint64_t)((ks >> 2) * KT * 8 + (ks & 3) * 2),
-                                   idS, ks > 0 ? 1u : 0u);
+                    umma::mma_bf16(d0, dQ0 + (uint64_t)((ks >> 2) * ROWS * 8 + (ks & 3) * 2),
+                                   bk + (uint64_t)((ks >> 2) * KT * 8 + (ks & 3) * 2), idS, ks > 0 ? 1u : 0u);
                 umma::commit(&mbar[kSFull + (j & 1)]);
                 if (ntl > 1) {
 #pragma unroll
                     for (int ks = 0; ks < DIM / 16; ++ks)
-                        umma::mma_bf16(d0 + 2 * KT, dQ1 + (uint64_t)(ks * 2 * ROWS),
+                        umma::mma_bf16(d0 + 2 * KT, dQ1 + (uint64_t)((ks >> 2) * ROWS * 8 + (ks & 3) * 2),
                                        bk + (uint64_t)((ks >> 2) * KT * 8 + (ks & 3) * 2), idS, ks > 0 ? 1u : 0u);
                     umma::commit(&mbar[kSFull + 2 + (j & 1)]);
                 }
