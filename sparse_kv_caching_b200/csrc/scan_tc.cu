@@ -87,8 +87,8 @@ __host__ __device__ inline TcOffsets tc_offsets(int D, int DV, int esize, int la
         o.fv = take(FK * DV * esize, 128);
         o.fpsum = o.fptr = 0;
     } else {
-        o.fa = take(kTcFKB * 128 * 2, 128);
-        o.fb = take(3 * kTcFKB * D * 2, 128);
+        o.fa = take(kTcFKB * 128 * 2, 1024);          // 128-byte swizzled operands
+        o.fb = take(3 * kTcFKB * D * 2, 1024);
         o.fphi = o.fv = 0;
         o.fpsum = take(8 * 256 * 4, 16);
         o.fptr = take(2 * kTcFKB * 8, 16);            // phi and value row addresses of the folded rows
@@ -516,7 +516,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
     // the A operand (bf16 is exact: one part); thread (j8, rr) of the compute warps reads
     // columns 8 j8 .. 8 j8 + 7 of rows rr RPT .. rr RPT + RPT - 1 of phi from global memory,
     // splits them into the three B parts and keeps the column sums of its rows; s then adds
-    // the row ranges' sums in range order.
+    // the row ranges' sums in range order.  Both operands are MN-major and 128-byte swizzled:
+    // folded row k of block mb holds its columns 64 mb .. 64 mb + 63 as one 128-byte row.
     auto fold_b16 = [&](int nf) {
         constexpr int FKB = kTcFKB, J8 = D / 8, RR = kTcCompute / J8, RPT = FKB / RR;
         static_assert(RR * J8 == kTcCompute && RPT * RR == FKB, "fold tiling");
@@ -537,7 +538,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
             __syncthreads();
             for (int idx = tid; idx < nk * (M / 8); idx += NT) {
                 const int k = idx / (M / 8), c8 = idx % (M / 8);
-                uint8_t* dst = fa + c8 * (FKB * 16) + k * 16;
+                uint8_t* dst = fa + (c8 >> 3) * (FKB * 128) + umma::sw128_off(k, c8 & 7);
                 if (k < nff && 8 * c8 < DV) {
                     umma::cp_async16(dst, vrow[k] + 8 * c8);
                 } else {
@@ -583,7 +584,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
                         w1[q] = (uint32_t)p1 | ((uint32_t)q1 << 16);
                         w2[q] = (uint32_t)p2 | ((uint32_t)q2 << 16);
                     }
-                    const int off = j8 * (FKB * 16) + k * 16;
+                    const int off = (j8 >> 3) * (FKB * 128) + (int)umma::sw128_off(k, j8 & 7);
                     *reinterpret_cast<uint4*>(fb + off) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
                     *reinterpret_cast<uint4*>(fb + FKB * D * 2 + off) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
                     *reinterpret_cast<uint4*>(fb + 2 * FKB * D * 2 + off) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
@@ -606,15 +607,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
                 const uint32_t id = umma::idesc(umma::kBF16, M, D, true, true);
                 const uint32_t A0 = umma::smem_addr(fa), B0 = umma::smem_addr(fb);
                 constexpr uint32_t PB = FKB * D * 2;                      // bytes between phi parts
-                const uint64_t a0 = umma::sdesc(A0, 128, FKB * 16), b0 = umma::sdesc(B0, 128, FKB * 16);
+                // MN-major swizzled: lbo = the stride between 64-column blocks, sbo = 8 rows
+                const uint64_t a0 = umma::sdesc_sw128(A0, FKB * 128, 1024), b0 = umma::sdesc_sw128(B0, FKB * 128, 1024);
 #pragma unroll
                 for (int ks = 0; ks < FKB / 16; ++ks) {
                     if (ks * 16 >= nk) break;
-                    // a K step of 16 moves the start by 256 bytes; the phi parts are PB bytes apart
-                    const uint64_t da = a0 + (uint64_t)((ks * 256) >> 4);
-                    umma::mma_bf16(tmem + cH, da, b0 + (uint64_t)((ks * 256) >> 4), id, 1u);
-                    umma::mma_bf16(tmem + cH, da, b0 + (uint64_t)((PB + ks * 256) >> 4), id, 1u);
-                    umma::mma_bf16(tmem + cH, da, b0 + (uint64_t)((2 * PB + ks * 256) >> 4), id, 1u);
+                    // a K step of 16 rows moves the start by 2048 bytes; the phi parts are PB bytes apart
+                    const uint64_t da = a0 + (uint64_t)((ks * 2048) >> 4);
+                    umma::mma_bf16(tmem + cH, da, b0 + (uint64_t)((ks * 2048) >> 4), id, 1u);
+                    umma::mma_bf16(tmem + cH, da, b0 + (uint64_t)((PB + ks * 2048) >> 4), id, 1u);
+                    umma::mma_bf16(tmem + cH, da, b0 + (uint64_t)((2 * PB + ks * 2048) >> 4), id, 1u);
                 }
                 umma::commit(&mbar[2]);
             }
