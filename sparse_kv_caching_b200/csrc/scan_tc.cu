@@ -228,19 +228,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) scan_tc_kernel(const __grid_con
 
     // H_{c}^T, slot positions and s_c into the snapshots of block c (rows of H^T and
     // slot ranges split over the cluster, s by rank 0)
+    // (rows of H_c^T go out whole: staged in the SRE ring, which is free between blocks,
+    // with a padded row so that the staging stores do not collide)
     auto publish = [&](int c) {
         float* sH = a.snap_H + ((size_t)st * snaps + c) * D * DV;
-        const bool mine = crow < DV && (NCL == 1 || crow / (DV / NCL) == rank);
-        if (compute) {
+        constexpr int RSB = D * 4 + 16;
+        uint8_t* stage = smem + o.raw;
+        if (compute && crow < DV) {
             float x[D / 2];
 #pragma unroll
             for (int j0 = 0; j0 < D / 2; j0 += 16)
                 umma::tmem_ld16(tmem + lane_off + cH + half * (D / 2) + j0, *reinterpret_cast<float(*)[16]>(x + j0));
             umma::tmem_wait_ld();
-            if (mine) {
-                float4* dst = reinterpret_cast<float4*>(sH + (size_t)crow * D + half * (D / 2));
+            uint8_t* row = stage + crow * RSB + half * (D / 2) * 4;
 #pragma unroll
-                for (int u = 0; u < D / 8; ++u) dst[u] = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+            for (int u = 0; u < D / 8; ++u)
+                *reinterpret_cast<float4*>(row + 16 * u) = make_float4(x[4 * u], x[4 * u + 1], x[4 * u + 2], x[4 * u + 3]);
+        }
+        __syncthreads();
+        {
+            // this CTA's share of the rows (split over the cluster), one 16-byte piece per thread
+            constexpr int F4 = D / 4, NR = DV / NCL;
+            const int r0 = rank * NR;
+            for (int idx = tid; idx < NR * F4; idx += NT) {
+                const int rr = r0 + idx / F4, c4 = idx % F4;
+                *reinterpret_cast<float4*>(sH + (size_t)rr * D + 4 * c4) =
+                    *reinterpret_cast<const float4*>(stage + rr * RSB + 16 * c4);
             }
         }
         int* sp_ = a.snap_pos + ((size_t)st * snaps + c) * lam;
