@@ -26,10 +26,10 @@
 namespace lola {
 
 constexpr int kDecThreads = 256;
-constexpr int kDecSlotBatch = 8;  // slot rows per warp in flight while scoring
+constexpr int kDecSlotBatch = 4;  // value rows per warp in flight in P V
 
 struct DecOffsets {
-    int Hs, ss, Ws, qs, phq, kn, vn, phk, phl, Pl, vf, phf, red, kp, sc, wm, R, part, total;
+    int ss, L, Ws, qs, phq, kn, vn, phk, phl, Pl, vf, phf, red, kp, sc, wm, R, part, total;
 };
 
 __host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int lam, int eta, int esize) {
@@ -37,8 +37,8 @@ __host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int l
     DecOffsets o;
     int p = 0;
     auto take = [&](int n) { int r = p; p += (n + 3) & ~3; return r; };
-    o.Hs = take(D * DIM);
     o.ss = take(D);
+    o.L = take(Gq * DIM);                  // phi(q)^T H per head
     o.Ws = 0;                             // set below: W (raw, <= 4 B per element) aliases R/part
     o.qs = take(Gq * DIM);
     o.phq = take(Gq * D);
@@ -53,8 +53,10 @@ __host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int l
     o.kp = take(4 * NK);                   // key and value row pointers (64-bit each)
     o.sc = take(max(Gq * NK, lam + 1));    // slot scores (update phase)
     o.wm = take(NW * 8 * 2);               // per-warp softmax max and sum per head
-    // the read-phase partial sums [NW][Gq][DIM] alias the z scratch and the staged W
-    o.R = take(max(NW * Gq * DIM, (DIM * DH * esize + 3) / 4 + (Gq + 1) * DH));
+    // the read-phase partial sums [NW][Gq][DIM] and the H-pass partial sums
+    // [NT / DIM][Gq + 1][DIM] alias the z scratch and the staged W
+    o.R = take(max(max(NW * Gq * DIM, kDecThreads / DIM * (Gq + 1) * DIM),
+                   (DIM * DH * esize + 3) / 4 + (Gq + 1) * DH));
     o.part = o.R;
     o.Ws = o.R + (Gq + 1) * DH;           // after the z scratch rows
     o.total = p;
@@ -70,6 +72,23 @@ __device__ __forceinline__ float quad_sum(float x) {
     x += __shfl_xor_sync(0xffffffffu, x, 1);
     x += __shfl_xor_sync(0xffffffffu, x, 2);
     return x;
+}
+// An octet of 8 lanes handles one row in the residual update: lane o takes the
+// 4-element chunks o, o + 8, o + 16, ..., so element u of lane o is row[oidx(o, u)].
+__device__ __forceinline__ int oidx(int o, int u) { return ((u >> 2) * 8 + o) * 4 + (u & 3); }
+__device__ __forceinline__ float oct_sum(float x) {
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    return x;
+}
+template <int N, typename T>
+__device__ __forceinline__ void load_oct(const T* row, int o, float (&out)[N / 8]) {
+#pragma unroll
+    for (int i = 0; i < N / 32; ++i) {
+        const float4 f = load4(row + (8 * i + o) * 4);
+        out[4 * i] = f.x; out[4 * i + 1] = f.y; out[4 * i + 2] = f.z; out[4 * i + 3] = f.w;
+    }
 }
 template <int N>
 __device__ __forceinline__ void load_quarter(const float* row, int q, float (&out)[N / 4]) {
@@ -89,7 +108,7 @@ __device__ __forceinline__ void load_quarter(const __nv_bfloat16* row, int q, fl
 }
 
 template <int DIM, int DH, typename TIn>
-__global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int D = 2 * DH, NT = kDecThreads, NW = NT / 32, CPL = DIM / 32;
     extern __shared__ __align__(16) float smem[];
     const Dims& dm = a.dm;
@@ -97,8 +116,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     const int st = blockIdx.x, b = st / dm.Hkv, g = st % dm.Hkv;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const DecOffsets o = dec_offsets(DIM, DH, Gq, lam, eta, (int)sizeof(TIn));
-    float* Hs = smem + o.Hs;
     float* ss = smem + o.ss;
+    float* Lq = smem + o.L;
     float* qs = smem + o.qs;
     float* phq = smem + o.phq;
     float* kn = smem + o.kn;
@@ -118,9 +137,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     float* Hg = a.sp.H + (size_t)st * D * DIM;
     float* sg = a.sp.s + (size_t)st * D;
     const TIn* Wg = (const TIn*)a.sp.W + (size_t)g * DIM * DH;
-    // H, s and W with asynchronous copies: every chunk in flight at once
+    // s and W with asynchronous copies (H stays in global memory: one pass reads
+    // it for the products below, the fold updates it in place)
     TIn* Wsm = reinterpret_cast<TIn*>(Ws);
-    for (int i = tid; i < D * DIM / 4; i += NT) umma::cp_async16(Hs + 4 * i, Hg + 4 * i);
     for (int i = tid; i < D / 4; i += NT) umma::cp_async16(ss + 4 * i, sg + 4 * i);
     constexpr int WCH = DIM * DH * (int)sizeof(TIn) / 16;
     for (int i = tid; i < WCH; i += NT)
@@ -200,6 +219,47 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
         for (int u = 0; u < DH / 32; ++u) { out[lane + 32 * u] = ep[u] / sp; out[DH + lane + 32 * u] = en[u] / sn; }
     }
     __syncthreads();
+
+    // ---- one pass over H ([D][DIM] in global memory): Lq[hh][cc] = phi(q_hh)^T H[:, cc]
+    // for the read and Pl[cc] = H[:, cc] . phi_l for the update; NT / DIM threads per
+    // column, each over a contiguous share of the rows, then their sums in share order ----
+    auto h_pass = [&](const bool wantL, const bool wantP) {
+        constexpr int NSP = NT / DIM, RPS = D / NSP, HB = 8;
+        const int cc = tid % DIM, sp = tid / DIM;
+        float acc[9];
+#pragma unroll
+        for (int k = 0; k < 9; ++k) acc[k] = 0.f;
+        const float* hcol = Hg + (size_t)sp * RPS * DIM + cc;
+        for (int j0 = 0; j0 < RPS; j0 += HB) {
+            float h[HB];
+#pragma unroll
+            for (int u = 0; u < HB; ++u) h[u] = hcol[(size_t)(j0 + u) * DIM];   // the batch's loads first
+#pragma unroll
+            for (int u = 0; u < HB; ++u) {
+                const int j = sp * RPS + j0 + u;
+                if (wantL) {
+#pragma unroll
+                    for (int hh = 0; hh < 8; ++hh)
+                        if (hh < Gq) acc[hh] = fmaf(phq[hh * D + j], h[u], acc[hh]);
+                }
+                if (wantP) acc[8] = fmaf(phl[j], h[u], acc[8]);
+            }
+        }
+        float* hp = smem + o.R;                                     // [NSP][Gq + 1][DIM]
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh)
+            if (hh < Gq) hp[(sp * (Gq + 1) + hh) * DIM + cc] = acc[hh];
+        hp[(sp * (Gq + 1) + Gq) * DIM + cc] = acc[8];
+        __syncthreads();
+        for (int idx = tid; idx < (Gq + 1) * DIM; idx += NT) {
+            float x = 0.f;
+            for (int k = 0; k < NSP; ++k) x += hp[k * (Gq + 1) * DIM + idx];
+            const int hh = idx / DIM;
+            if (hh < Gq) { if (wantL) Lq[idx] = x; }
+            else if (wantP) Pl[idx - Gq * DIM] = x;
+        }
+        __syncthreads();
+    };
 
     // ---- read: scores (a quad per key), softmax per head, P V (lane owns columns) ----
     // Eq. 14 over the NK keys of kp and, unless hidden, the state (H, s) in shared memory
@@ -300,9 +360,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
             const int hh = idx / DIM, cc = idx % DIM;
             float A = 0.f;
             for (int w = 0; w < NW; ++w) A += part[(w * Gq + hh) * DIM + cc];
-            float L = 0.f;
-            if (!hide_state)
-                for (int j = 0; j < D; ++j) L = fmaf(phq[hh * D + j], Hs[j * DIM + cc], L);
+            const float L = hide_state ? 0.f : Lq[idx];
             const float em = expf(-red[hh]);
             a.y[((size_t)b * dm.Hq + (size_t)g * Gq + hh) * DIM + cc] = (A + em * L) / (red[8 + hh] + em * red[16 + hh]);
         }
@@ -314,13 +372,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
         if (leaving) {
             const size_t wsl = wbase + rs;
             const TIn* vl = (const TIn*)a.sp.win_v + wsl * DIM;
-            // P_l = H^T phi_l, den_l = phi_l . s, R_l = P_l - den_l v_l (pre-fold state; SRE only)
+            // P_l = H^T phi_l (the H pass), den_l = phi_l . s, R_l = P_l - den_l v_l
+            // (pre-fold state; SRE only)
             if (!a.scorer) {
-                for (int cc = tid; cc < DIM; cc += NT) {
-                    float x = 0.f;
-                    for (int j = 0; j < D; ++j) x = fmaf(phl[j], Hs[j * DIM + cc], x);
-                    Pl[cc] = x;
-                }
                 if (warp == 0) {
                     float x = 0.f;
                     for (int j = lane; j < D; j += 32) x = fmaf(phl[j], ss[j], x);
@@ -403,44 +457,65 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                 for (int i = tid; i < D; i += NT) phf[i] = f < lam ? a.sp.cache_phik[(cbase + f) * D + i] : phl[i];
                 for (int i = tid; i < DIM; i += NT) vf[i] = to_f32(f < lam ? ((const TIn*)a.sp.cache_v)[(cbase + f) * DIM + i] : vl[i]);
                 __syncthreads();
-                // fold (Eqs. 12-13): H += phi_f v_f^T, s += phi_f
-                for (int i = tid; i < D * DIM; i += NT) Hs[i] = fmaf(phf[i / DIM], vf[i % DIM], Hs[i]);
+                // fold (Eqs. 12-13): H += phi_f v_f^T in place (8 float4 loads in flight
+                // per thread), s += phi_f
+                {
+                    constexpr int NV = D * DIM / 4 / NT, FB = NV < 8 ? NV : 8;
+                    static_assert(NV * NT * 4 == D * DIM, "whole float4 rounds");
+                    float4* H4 = reinterpret_cast<float4*>(Hg);
+#pragma unroll 1
+                    for (int v0 = 0; v0 < NV; v0 += FB) {
+                        float4 h[FB];
+#pragma unroll
+                        for (int u = 0; u < FB; ++u) h[u] = H4[(v0 + u) * NT + tid];
+#pragma unroll
+                        for (int u = 0; u < FB; ++u) {
+                            const int i = 4 * ((v0 + u) * NT + tid), j = i / DIM, c = i % DIM;
+                            const float p = phf[j];
+                            h[u].x = fmaf(p, vf[c], h[u].x);
+                            h[u].y = fmaf(p, vf[c + 1], h[u].y);
+                            h[u].z = fmaf(p, vf[c + 2], h[u].z);
+                            h[u].w = fmaf(p, vf[c + 3], h[u].w);
+                            H4[(v0 + u) * NT + tid] = h[u];
+                        }
+                    }
+                }
                 for (int i = tid; i < D; i += NT) ss[i] += phf[i];
                 // residuals of every remaining member follow the rank-1 change (SRE only)
-                // a quad per member: k_e = phi_e . phi_f, R_e += k_e (v_f - v_e), den_e += k_e
+                // an octet per member: k_e = phi_e . phi_f, R_e += k_e (v_f - v_e), den_e += k_e
                 if (!a.scorer) {
-                    constexpr int PQ = D / 4, RQ = DIM / 4;
-                    const int q4 = lane & 3, rq = lane >> 2;
-                    for (int e0 = warp * 8; e0 <= lam; e0 += NW * 8) {
-                        const int e = e0 + rq;
+                    constexpr int PO = D / 8, RO = DIM / 8;
+                    const int o8 = lane & 7, ro = lane >> 3;
+                    for (int e0 = warp * 4; e0 <= lam; e0 += NW * 4) {
+                        const int e = e0 + ro;
                         const bool act = e <= lam && e != f;
-                        float pv[PQ], vv[RQ], r0[RQ];
+                        float pv[PO], vv[RO], r0[RO];
                         float d0 = 0.f;
                         if (act) {
-                            load_quarter<D>(e < lam ? a.sp.cache_phik + (cbase + e) * D : phl, q4, pv);
-                            load_quarter<DIM>(e < lam ? (const TIn*)a.sp.cache_v + (cbase + e) * DIM : vl, q4, vv);
+                            load_oct<D>(e < lam ? a.sp.cache_phik + (cbase + e) * D : phl, o8, pv);
+                            load_oct<DIM>(e < lam ? (const TIn*)a.sp.cache_v + (cbase + e) * DIM : vl, o8, vv);
                             if (e < lam) {
-                                load_quarter<DIM>(Rg + (size_t)e * DIM, q4, r0);
+                                load_oct<DIM>(Rg + (size_t)e * DIM, o8, r0);
                                 d0 = deng[e];
                             } else {
 #pragma unroll
-                                for (int u = 0; u < RQ; ++u) r0[u] = Pl[qidx(q4, u)] - den_l * vv[u];
+                                for (int u = 0; u < RO; ++u) r0[u] = Pl[oidx(o8, u)] - den_l * vv[u];
                                 d0 = den_l;
                             }
                         }
                         float kap = 0.f;
                         if (act) {
 #pragma unroll
-                            for (int u = 0; u < PQ; ++u) kap = fmaf(pv[u], phf[qidx(q4, u)], kap);
+                            for (int u = 0; u < PO; ++u) kap = fmaf(pv[u], phf[oidx(o8, u)], kap);
                         }
-                        kap = quad_sum(kap);
+                        kap = oct_sum(kap);
                         float q = 0.f, vq = 0.f;
+                        const int dst = e < lam ? e : f;   // its own slot, or f's slot for the newcomer l
                         if (act) {
-                            const int dst = e < lam ? e : f;   // its own slot, or f's slot for the newcomer l
                             float* rw = Rg + (size_t)dst * DIM;
 #pragma unroll
-                            for (int u = 0; u < RQ; u += 4) {
-                                const int c0 = qidx(q4, u);                       // 4 consecutive columns
+                            for (int u = 0; u < RO; u += 4) {
+                                const int c0 = oidx(o8, u);                       // 4 consecutive columns
                                 const float4 r4 = make_float4(
                                     fmaf(kap, vf[c0] - vv[u], r0[u]), fmaf(kap, vf[c0 + 1] - vv[u + 1], r0[u + 1]),
                                     fmaf(kap, vf[c0 + 2] - vv[u + 2], r0[u + 2]), fmaf(kap, vf[c0 + 3] - vv[u + 3], r0[u + 3]));
@@ -449,12 +524,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                                 q = fmaf(r4.z, r4.z, q); q = fmaf(r4.w, r4.w, q);
                             }
 #pragma unroll
-                            for (int u = 0; u < RQ; ++u) vq = fmaf(vv[u], vv[u], vq);
+                            for (int u = 0; u < RO; ++u) vq = fmaf(vv[u], vv[u], vq);
                         }
-                        q = quad_sum(q);
-                        vq = quad_sum(vq);
-                        if (act && q4 == 0) {
-                            const int dst = e < lam ? e : f;
+                        q = oct_sum(q);
+                        vq = oct_sum(vq);
+                        if (act && o8 == 0) {
                             const float dn = d0 + kap;
                             deng[dst] = dn;
                             a.sp.cache_sc[cbase + dst] = dn > 0.f ? q / (dn * dn) : vq;   // SRE against the new state
@@ -474,8 +548,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
                     }
                 }
                 __syncthreads();
-                for (int i = tid; i < D * DIM / 4; i += NT)
-                    reinterpret_cast<float4*>(Hg)[i] = reinterpret_cast<const float4*>(Hs)[i];
                 for (int i = tid; i < D; i += NT) sg[i] = ss[i];
             }
         }
@@ -492,10 +564,13 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
         }
     };
 
+    const bool needP = leaving && !a.scorer;                      // H^T phi_l for the update
     if (!a.update_first) {
+        if (!hide_state || needP) h_pass(!hide_state, needP);
         read_phase(NK, rg0, rlo0);
         update_phase();
     } else {
+        if (needP) h_pass(false, true);
         // the token equations read literally: update, then read the new memories
         // (cache slots [0, min(lambda, t + 1 - eta)), window [t + 1 - eta, t), the token)
         update_phase();
@@ -503,6 +578,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
         const int rg1 = hide_sparse ? 0 : min(lam, max(0, t + 1 - eta)), rlo1 = max(0, t + 1 - eta);
         const int nk = fill_kp(rg1, rlo1);
         __syncthreads();
+        if (!hide_state) h_pass(true, false);                     // the folded state
         read_phase(nk, rg1, rlo1);
     }
 }
