@@ -26,10 +26,10 @@
 namespace lola {
 
 constexpr int kDecThreads = 256;
-constexpr int kDecSlotBatch = 4;  // value rows per warp in flight in P V
+constexpr int kDecSlotBatch = 8;  // value rows per warp in flight in P V
 
 struct DecOffsets {
-    int ss, L, Ws, qs, phq, kn, vn, phk, phl, Pl, vf, phf, red, kp, sc, wm, R, part, total;
+    int ss, L, hp, Ws, qs, phq, kn, vn, phk, phl, Pl, vf, phf, red, kp, sc, wm, R, part, total;
 };
 
 __host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int lam, int eta, int esize) {
@@ -39,6 +39,7 @@ __host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int l
     auto take = [&](int n) { int r = p; p += (n + 3) & ~3; return r; };
     o.ss = take(D);
     o.L = take(Gq * DIM);                  // phi(q)^T H per head
+    o.hp = take(kDecThreads / DIM * (Gq + 1) * DIM);   // the H pass's partial sums
     o.Ws = 0;                             // set below: W (raw, <= 4 B per element) aliases R/part
     o.qs = take(Gq * DIM);
     o.phq = take(Gq * D);
@@ -53,10 +54,8 @@ __host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int l
     o.kp = take(4 * NK);                   // key and value row pointers (64-bit each)
     o.sc = take(max(Gq * NK, lam + 1));    // slot scores (update phase)
     o.wm = take(NW * 8 * 2);               // per-warp softmax max and sum per head
-    // the read-phase partial sums [NW][Gq][DIM] and the H-pass partial sums
-    // [NT / DIM][Gq + 1][DIM] alias the z scratch and the staged W
-    o.R = take(max(max(NW * Gq * DIM, kDecThreads / DIM * (Gq + 1) * DIM),
-                   (DIM * DH * esize + 3) / 4 + (Gq + 1) * DH));
+    // the read-phase partial sums [NW][Gq][DIM] alias the z scratch and the staged W
+    o.R = take(max(NW * Gq * DIM, (DIM * DH * esize + 3) / 4 + (Gq + 1) * DH));
     o.part = o.R;
     o.Ws = o.R + (Gq + 1) * DH;           // after the z scratch rows
     o.total = p;
@@ -73,6 +72,20 @@ __device__ __forceinline__ float quad_sum(float x) {
     x += __shfl_xor_sync(0xffffffffu, x, 2);
     return x;
 }
+// Rows kept as raw 32-bit words until their values are used (a bf16 word holds
+// two elements, the lower address in the low half).
+template <int NWD>
+__device__ __forceinline__ void load_words(const void* p, unsigned* w) {
+    if constexpr (NWD == 4) { const uint4 v = *reinterpret_cast<const uint4*>(p); w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w; }
+    else if constexpr (NWD == 2) { const uint2 v = *reinterpret_cast<const uint2*>(p); w[0] = v.x; w[1] = v.y; }
+    else { static_assert(NWD == 1, "1, 2 or 4 words"); w[0] = *reinterpret_cast<const unsigned*>(p); }
+}
+template <typename T> __device__ __forceinline__ float word_elem(unsigned w, int h);
+template <> __device__ __forceinline__ float word_elem<float>(unsigned w, int) { return __uint_as_float(w); }
+template <> __device__ __forceinline__ float word_elem<__nv_bfloat16>(unsigned w, int h) {
+    return __uint_as_float(h ? (w & 0xffff0000u) : (w << 16));
+}
+
 // An octet of 8 lanes handles one row in the residual update: lane o takes the
 // 4-element chunks o, o + 8, o + 16, ..., so element u of lane o is row[oidx(o, u)].
 __device__ __forceinline__ int oidx(int o, int u) { return ((u >> 2) * 8 + o) * 4 + (u & 3); }
@@ -107,7 +120,8 @@ __device__ __forceinline__ void load_quarter(const __nv_bfloat16* row, int q, fl
     }
 }
 
-template <int DIM, int DH, typename TIn>
+// GQM bounds the query heads per kv head (Gq <= GQM): per-head registers are sized by it.
+template <int DIM, int DH, int GQM, typename TIn>
 __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int D = 2 * DH, NT = kDecThreads, NW = NT / 32, CPL = DIM / 32;
     extern __shared__ __align__(16) float smem[];
@@ -226,9 +240,9 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
     auto h_pass = [&](const bool wantL, const bool wantP) {
         constexpr int NSP = NT / DIM, RPS = D / NSP, HB = 8;
         const int cc = tid % DIM, sp = tid / DIM;
-        float acc[9];
+        float acc[GQM + 1];
 #pragma unroll
-        for (int k = 0; k < 9; ++k) acc[k] = 0.f;
+        for (int k = 0; k <= GQM; ++k) acc[k] = 0.f;
         const float* hcol = Hg + (size_t)sp * RPS * DIM + cc;
         for (int j0 = 0; j0 < RPS; j0 += HB) {
             float h[HB];
@@ -239,17 +253,17 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
                 const int j = sp * RPS + j0 + u;
                 if (wantL) {
 #pragma unroll
-                    for (int hh = 0; hh < 8; ++hh)
+                    for (int hh = 0; hh < GQM; ++hh)
                         if (hh < Gq) acc[hh] = fmaf(phq[hh * D + j], h[u], acc[hh]);
                 }
-                if (wantP) acc[8] = fmaf(phl[j], h[u], acc[8]);
+                if (wantP) acc[GQM] = fmaf(phl[j], h[u], acc[GQM]);
             }
         }
-        float* hp = smem + o.R;                                     // [NSP][Gq + 1][DIM]
+        float* hp = smem + o.hp;                                    // [NSP][Gq + 1][DIM]
 #pragma unroll
-        for (int hh = 0; hh < 8; ++hh)
+        for (int hh = 0; hh < GQM; ++hh)
             if (hh < Gq) hp[(sp * (Gq + 1) + hh) * DIM + cc] = acc[hh];
-        hp[(sp * (Gq + 1) + Gq) * DIM + cc] = acc[8];
+        hp[(sp * (Gq + 1) + Gq) * DIM + cc] = acc[GQM];
         __syncthreads();
         for (int idx = tid; idx < (Gq + 1) * DIM; idx += NT) {
             float x = 0.f;
@@ -263,24 +277,44 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
 
     // ---- read: scores (a quad per key), softmax per head, P V (lane owns columns) ----
     // Eq. 14 over the NK keys of kp and, unless hidden, the state (H, s) in shared memory
-    auto read_phase = [&](const int NK, const int rg, const int rlo) {
-        constexpr int KQ = DIM / 4;                                  // key elements per quad lane
+    auto read_phase = [&](const int NK, const int rg, const int rlo, const bool wantP) {
+        // a quad of lanes per key, KPQ keys per quad; lane q4 takes the 16-byte chunks
+        // q4, q4 + 4, ... of the row, kept as raw words
+        constexpr int CH = 16 / (int)sizeof(TIn), NCH = DIM / CH / 4, KW = NCH * 4, EPW = 4 / (int)sizeof(TIn);
+        constexpr int KPQ = sizeof(TIn) == 2 ? 2 : 1;
         const int q4 = lane & 3, rq = lane >> 2;                     // lane in quad, quad in warp
         const float scale = 1.0f / sqrtf((float)DIM);
-        for (int i0 = warp * 8; i0 < NK; i0 += NW * 8) {
-            const int i = i0 + rq;
-            float kk[KQ];
-            if (i < NK) load_quarter<DIM>(kp[2 * i], q4, kk);
+        for (int i0 = warp * 8 * KPQ; i0 < NK; i0 += NW * 8 * KPQ) {
+            unsigned kw[KPQ][KW];
 #pragma unroll
-            for (int hh = 0; hh < 8; ++hh) {
+            for (int kq = 0; kq < KPQ; ++kq) {
+                const int i = i0 + kq * 8 + rq;
+                if (i < NK)
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c) load_words<4>(kp[2 * i] + (c * 4 + q4) * CH, &kw[kq][4 * c]);
+            }
+#pragma unroll
+            for (int hh = 0; hh < GQM; ++hh) {
                 if (hh < Gq) {
-                    float sdot = 0.f;
-                    if (i < NK) {
+                    float sd[KPQ];
 #pragma unroll
-                        for (int u = 0; u < KQ; ++u) sdot = fmaf(qs[hh * DIM + qidx(q4, u)], kk[u], sdot);
+                    for (int kq = 0; kq < KPQ; ++kq) sd[kq] = 0.f;
+#pragma unroll
+                    for (int c = 0; c < NCH; ++c)
+#pragma unroll
+                        for (int w = 0; w < 4; ++w)
+#pragma unroll
+                            for (int h = 0; h < EPW; ++h) {
+                                const float qv = qs[hh * DIM + (c * 4 + q4) * CH + w * EPW + h];
+#pragma unroll
+                                for (int kq = 0; kq < KPQ; ++kq) sd[kq] = fmaf(qv, word_elem<TIn>(kw[kq][4 * c + w], h), sd[kq]);
+                            }
+#pragma unroll
+                    for (int kq = 0; kq < KPQ; ++kq) {
+                        const float x = quad_sum(sd[kq]);
+                        const int i = i0 + kq * 8 + rq;
+                        if (i < NK && q4 == 0) sc[hh * NK + i] = x * scale;
                     }
-                    sdot = quad_sum(sdot);
-                    if (i < NK && q4 == 0) sc[hh * NK + i] = sdot * scale;
                 }
             }
         }
@@ -320,42 +354,43 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
             if (lane == 0) { red[hh] = mx; red[8 + hh] = sum; red[16 + hh] = dl; }
         }
         __syncthreads();
-        float accp[8][CPL];
+        float accp[GQM][CPL];
 #pragma unroll
-        for (int hh = 0; hh < 8; ++hh)
+        for (int hh = 0; hh < GQM; ++hh)
 #pragma unroll
             for (int u = 0; u < CPL; ++u) accp[hh][u] = 0.f;
+        constexpr int PVW = CPL * (int)sizeof(TIn) / 4;              // words of a lane's columns
         for (int i0 = warp; i0 < NK; i0 += NW * kDecSlotBatch) {
-            float vv[kDecSlotBatch][CPL];
+            unsigned vw[kDecSlotBatch][PVW];
 #pragma unroll
             for (int bb = 0; bb < kDecSlotBatch; ++bb) {             // issue the batch's loads first
                 const int i = i0 + bb * NW;
-                if (i < NK) {
-                    const TIn* vr = kp[2 * i + 1] + lane * CPL;
-                    if constexpr (CPL == 4) { const float4 v4 = load4(vr); vv[bb][0] = v4.x; vv[bb][1] = v4.y; vv[bb][2] = v4.z; vv[bb][3] = v4.w; }
-                    else { const float2 v2 = load2(vr); vv[bb][0] = v2.x; vv[bb][1] = v2.y; }
-                }
+                if (i < NK) load_words<PVW>(kp[2 * i + 1] + lane * CPL, vw[bb]);
             }
 #pragma unroll
             for (int bb = 0; bb < kDecSlotBatch; ++bb) {
                 const int i = i0 + bb * NW;
                 if (i >= NK) break;
 #pragma unroll
-                for (int hh = 0; hh < 8; ++hh) {
+                for (int hh = 0; hh < GQM; ++hh) {
                     if (hh < Gq) {
                         const float p = sc[hh * NK + i];
 #pragma unroll
-                        for (int u = 0; u < CPL; ++u) accp[hh][u] = fmaf(p, vv[bb][u], accp[hh][u]);
+                        for (int u = 0; u < CPL; ++u)
+                            accp[hh][u] = fmaf(p, word_elem<TIn>(vw[bb][u / EPW], u % EPW), accp[hh][u]);
                     }
                 }
             }
         }
 #pragma unroll
-        for (int hh = 0; hh < 8; ++hh)
+        for (int hh = 0; hh < GQM; ++hh)
             if (hh < Gq)
 #pragma unroll
                 for (int u = 0; u < CPL; ++u) part[(warp * Gq + hh) * DIM + lane * CPL + u] = accp[hh][u];
         __syncthreads();
+        // phi(q)^T H for the output and, read first, H^T phi_l for the update: H is read
+        // here, close to the fold, so that the fold finds it in L2
+        if (!hide_state || wantP) h_pass(!hide_state, wantP);
         for (int idx = tid; idx < Gq * DIM; idx += NT) {
             const int hh = idx / DIM, cc = idx % DIM;
             float A = 0.f;
@@ -566,8 +601,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
 
     const bool needP = leaving && !a.scorer;                      // H^T phi_l for the update
     if (!a.update_first) {
-        if (!hide_state || needP) h_pass(!hide_state, needP);
-        read_phase(NK, rg0, rlo0);
+        read_phase(NK, rg0, rlo0, needP);
         update_phase();
     } else {
         if (needP) h_pass(false, true);
@@ -578,8 +612,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
         const int rg1 = hide_sparse ? 0 : min(lam, max(0, t + 1 - eta)), rlo1 = max(0, t + 1 - eta);
         const int nk = fill_kp(rg1, rlo1);
         __syncthreads();
-        if (!hide_state) h_pass(true, false);                     // the folded state
-        read_phase(nk, rg1, rlo1);
+        read_phase(nk, rg1, rlo1, false);                         // over the folded state
     }
 }
 
@@ -636,15 +669,20 @@ __global__ void __launch_bounds__(256) residual_init_kernel(const __grid_constan
     }
 }
 
-template <int DIM, int DH, typename TIn>
-static cudaError_t launch_dec_t(const DecodeArgs& a0, cudaStream_t s) {
-    const DecodeArgs& a = a0;
+template <int DIM, int DH, int GQM, typename TIn>
+static cudaError_t launch_dec_g(const DecodeArgs& a, cudaStream_t s) {
     const size_t bytes = (size_t)dec_offsets(DIM, DH, a.dm.Gq, a.dm.lam, a.dm.eta, (int)sizeof(TIn)).total * 4;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<DIM, DH, TIn>,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<DIM, DH, GQM, TIn>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
-    decode_kernel<DIM, DH, TIn><<<a.dm.S, kDecThreads, bytes, s>>>(a);
+    decode_kernel<DIM, DH, GQM, TIn><<<a.dm.S, kDecThreads, bytes, s>>>(a);
     return cudaGetLastError();
+}
+
+template <int DIM, int DH, typename TIn>
+static cudaError_t launch_dec_t(const DecodeArgs& a, cudaStream_t s) {
+    if (a.dm.Gq < 1 || a.dm.Gq > 8) return cudaErrorInvalidValue;
+    return a.dm.Gq <= 4 ? launch_dec_g<DIM, DH, 4, TIn>(a, s) : launch_dec_g<DIM, DH, 8, TIn>(a, s);
 }
 
 template <int DIM, int DH, typename TIn>
