@@ -29,7 +29,7 @@ constexpr int kDecThreads = 256;
 constexpr int kDecSlotBatch = 8;  // value rows per warp in flight in P V
 
 struct DecOffsets {
-    int ss, L, hp, Ws, qs, phq, kn, vn, phk, phl, Pl, vf, phf, red, kp, sc, wm, R, part, total;
+    int ss, L, hp, Ws, qs, phq, kn, vn, phk, phl, Pl, vf, phf, red, kp, sc, R, part, total;
 };
 
 __host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int lam, int eta, int esize) {
@@ -53,7 +53,6 @@ __host__ __device__ inline DecOffsets dec_offsets(int DIM, int DH, int Gq, int l
     o.red = take(128);
     o.kp = take(4 * NK);                   // key and value row pointers (64-bit each)
     o.sc = take(max(Gq * NK, lam + 1));    // slot scores (update phase)
-    o.wm = take(NW * 8 * 2);               // per-warp softmax max and sum per head
     // the read-phase partial sums [NW][Gq][DIM] alias the z scratch and the staged W
     o.R = take(max(NW * Gq * DIM, (DIM * DH * esize + 3) / 4 + (Gq + 1) * DH));
     o.part = o.R;
@@ -144,7 +143,6 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
     float* red = smem + o.red;
     const TIn** kp = reinterpret_cast<const TIn**>(smem + o.kp);
     float* sc = smem + o.sc;
-    float* wm = smem + o.wm;
     float* Ws = smem + o.Ws;
     float* part = smem + o.part;
 
@@ -277,7 +275,9 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
 
     // ---- read: scores (a quad per key), softmax per head, P V (lane owns columns) ----
     // Eq. 14 over the NK keys of kp and, unless hidden, the state (H, s) in shared memory
-    auto read_phase = [&](const int NK, const int rg, const int rlo, const bool wantP) {
+    // hL / hP: run the H pass after P V for phi(q)^T H / H^T phi_l; dlReady: phi(q) . s
+    // is already in red[16 + hh] (taken before a fold that precedes the read)
+    auto read_phase = [&](const int NK, const int rg, const int rlo, const bool hL, const bool hP, const bool dlReady) {
         // a quad of lanes per key, KPQ keys per quad; lane q4 takes the 16-byte chunks
         // q4, q4 + 4, ... of the row, kept as raw words
         constexpr int CH = 16 / (int)sizeof(TIn), NCH = DIM / CH / 4, KW = NCH * 4, EPW = 4 / (int)sizeof(TIn);
@@ -347,11 +347,14 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
             float sum = 0.f;
             for (int i = lane; i < NK; i += 32) { const float e = expf(sc[hh * NK + i] - mx); sc[hh * NK + i] = e; sum += e; }
             sum = warp_sum(sum);
-            float dl = 0.f;
-            if (!hide_state)
-                for (int j = lane; j < D; j += 32) dl = fmaf(phq[hh * D + j], ss[j], dl);
-            dl = warp_sum(dl);
-            if (lane == 0) { red[hh] = mx; red[8 + hh] = sum; red[16 + hh] = dl; }
+            if (!dlReady) {
+                float dl = 0.f;
+                if (!hide_state)
+                    for (int j = lane; j < D; j += 32) dl = fmaf(phq[hh * D + j], ss[j], dl);
+                dl = warp_sum(dl);
+                if (lane == 0) red[16 + hh] = dl;
+            }
+            if (lane == 0) { red[hh] = mx; red[8 + hh] = sum; }
         }
         __syncthreads();
         float accp[GQM][CPL];
@@ -390,7 +393,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
         __syncthreads();
         // phi(q)^T H for the output and, read first, H^T phi_l for the update: H is read
         // here, close to the fold, so that the fold finds it in L2
-        if (!hide_state || wantP) h_pass(!hide_state, wantP);
+        if (hL || hP) h_pass(hL, hP);
         for (int idx = tid; idx < Gq * DIM; idx += NT) {
             const int hh = idx / DIM, cc = idx % DIM;
             float A = 0.f;
@@ -402,8 +405,95 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
         __syncthreads();
     };
 
+    int f_fold = lam;                                             // the folded candidate
+    float den_fold = 0.f;                                         // phi_l . s before the fold
+    // the remaining members' residuals follow the rank-1 fold of f (SRE only), then l
+    // takes the folded member's slot
+    auto members_and_slot = [&](const int f, const float den_l) {
+        const size_t wsl = wbase + rs;
+        const TIn* vl = (const TIn*)a.sp.win_v + wsl * DIM;
+        float* Rg = a.sp.cache_R + cbase * DIM;
+        float* deng = a.sp.cache_den + cbase;
+        // an octet per member: k_e = phi_e . phi_f, R_e += k_e (v_f - v_e), den_e += k_e
+        if (!a.scorer) {
+            constexpr int PO = D / 8, RO = DIM / 8;
+            const int o8 = lane & 7, ro = lane >> 3;
+            for (int e0 = warp * 4; e0 <= lam; e0 += NW * 4) {
+                const int e = e0 + ro;
+                const bool act = e <= lam && e != f;
+                float pv[PO], vv[RO], r0[RO];
+                float d0 = 0.f;
+                if (act) {
+                    load_oct<D>(e < lam ? a.sp.cache_phik + (cbase + e) * D : phl, o8, pv);
+                    load_oct<DIM>(e < lam ? (const TIn*)a.sp.cache_v + (cbase + e) * DIM : vl, o8, vv);
+                    if (e < lam) {
+                        load_oct<DIM>(Rg + (size_t)e * DIM, o8, r0);
+                        d0 = deng[e];
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < RO; ++u) r0[u] = Pl[oidx(o8, u)] - den_l * vv[u];
+                        d0 = den_l;
+                    }
+                }
+                float kap = 0.f;
+                if (act) {
+#pragma unroll
+                    for (int u = 0; u < PO; ++u) kap = fmaf(pv[u], phf[oidx(o8, u)], kap);
+                }
+                kap = oct_sum(kap);
+                float q = 0.f, vq = 0.f;
+                const int dst = e < lam ? e : f;   // its own slot, or f's slot for the newcomer l
+                if (act) {
+                    float* rw = Rg + (size_t)dst * DIM;
+#pragma unroll
+                    for (int u = 0; u < RO; u += 4) {
+                        const int c0 = oidx(o8, u);                       // 4 consecutive columns
+                        const float4 r4 = make_float4(
+                            fmaf(kap, vf[c0] - vv[u], r0[u]), fmaf(kap, vf[c0 + 1] - vv[u + 1], r0[u + 1]),
+                            fmaf(kap, vf[c0 + 2] - vv[u + 2], r0[u + 2]), fmaf(kap, vf[c0 + 3] - vv[u + 3], r0[u + 3]));
+                        *reinterpret_cast<float4*>(rw + c0) = r4;
+                        q = fmaf(r4.x, r4.x, q); q = fmaf(r4.y, r4.y, q);
+                        q = fmaf(r4.z, r4.z, q); q = fmaf(r4.w, r4.w, q);
+                    }
+#pragma unroll
+                    for (int u = 0; u < RO; ++u) vq = fmaf(vv[u], vv[u], vq);
+                }
+                q = oct_sum(q);
+                vq = oct_sum(vq);
+                if (act && o8 == 0) {
+                    const float dn = d0 + kap;
+                    deng[dst] = dn;
+                    a.sp.cache_sc[cbase + dst] = dn > 0.f ? q / (dn * dn) : vq;   // SRE against the new state
+                }
+            }
+        }
+        if (f < lam) {                                            // l takes the folded member's slot
+            const size_t cs = cbase + f;
+            for (int i = tid; i < DIM; i += NT) {
+                ((TIn*)a.sp.cache_k)[cs * DIM + i] = ((const TIn*)a.sp.win_k)[wsl * DIM + i];
+                ((TIn*)a.sp.cache_v)[cs * DIM + i] = vl[i];
+            }
+            for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
+            if (tid == 0) {
+                a.sp.cache_pos[cs] = lpos;
+                if (a.scorer) a.sp.cache_sc[cs] = sc[lam];
+            }
+        }
+    };
+    // the new token enters the window ring (after every read of the leaving slot)
+    auto ring_write = [&]() {
+        __syncthreads();
+        const size_t ws = wbase + (size_t)(t % eta);
+        for (int i = tid; i < DIM; i += NT) {
+            ((TIn*)a.sp.win_k)[ws * DIM + i] = kg[i];
+            ((TIn*)a.sp.win_v)[ws * DIM + i] = vg[i];
+        }
+        for (int i = tid; i < D; i += NT) a.sp.win_phik[ws * D + i] = phk[i];
+        if (a.scorer && !a.update_first && tid == 0) a.sp.win_sc[ws] = red[48];
+    };
+
     // ---- update (Eqs. 11-13 with one leaving pair l = t - eta) ----
-    auto update_phase = [&]() {
+    auto update_phase = [&](const bool tail) {
         if (leaving) {
             const size_t wsl = wbase + rs;
             const TIn* vl = (const TIn*)a.sp.win_v + wsl * DIM;
@@ -488,6 +578,8 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
                     if (cand_key(e) == bb) *fsel = e;
                 __syncthreads();
                 const int f = *fsel;
+                f_fold = f;
+                den_fold = den_l;
                 // stage the folded pair
                 for (int i = tid; i < D; i += NT) phf[i] = f < lam ? a.sp.cache_phik[(cbase + f) * D + i] : phl[i];
                 for (int i = tid; i < DIM; i += NT) vf[i] = to_f32(f < lam ? ((const TIn*)a.sp.cache_v)[(cbase + f) * DIM + i] : vl[i]);
@@ -517,102 +609,46 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
                 }
                 for (int i = tid; i < D; i += NT) ss[i] += phf[i];
                 // residuals of every remaining member follow the rank-1 change (SRE only)
-                // an octet per member: k_e = phi_e . phi_f, R_e += k_e (v_f - v_e), den_e += k_e
-                if (!a.scorer) {
-                    constexpr int PO = D / 8, RO = DIM / 8;
-                    const int o8 = lane & 7, ro = lane >> 3;
-                    for (int e0 = warp * 4; e0 <= lam; e0 += NW * 4) {
-                        const int e = e0 + ro;
-                        const bool act = e <= lam && e != f;
-                        float pv[PO], vv[RO], r0[RO];
-                        float d0 = 0.f;
-                        if (act) {
-                            load_oct<D>(e < lam ? a.sp.cache_phik + (cbase + e) * D : phl, o8, pv);
-                            load_oct<DIM>(e < lam ? (const TIn*)a.sp.cache_v + (cbase + e) * DIM : vl, o8, vv);
-                            if (e < lam) {
-                                load_oct<DIM>(Rg + (size_t)e * DIM, o8, r0);
-                                d0 = deng[e];
-                            } else {
-#pragma unroll
-                                for (int u = 0; u < RO; ++u) r0[u] = Pl[oidx(o8, u)] - den_l * vv[u];
-                                d0 = den_l;
-                            }
-                        }
-                        float kap = 0.f;
-                        if (act) {
-#pragma unroll
-                            for (int u = 0; u < PO; ++u) kap = fmaf(pv[u], phf[oidx(o8, u)], kap);
-                        }
-                        kap = oct_sum(kap);
-                        float q = 0.f, vq = 0.f;
-                        const int dst = e < lam ? e : f;   // its own slot, or f's slot for the newcomer l
-                        if (act) {
-                            float* rw = Rg + (size_t)dst * DIM;
-#pragma unroll
-                            for (int u = 0; u < RO; u += 4) {
-                                const int c0 = oidx(o8, u);                       // 4 consecutive columns
-                                const float4 r4 = make_float4(
-                                    fmaf(kap, vf[c0] - vv[u], r0[u]), fmaf(kap, vf[c0 + 1] - vv[u + 1], r0[u + 1]),
-                                    fmaf(kap, vf[c0 + 2] - vv[u + 2], r0[u + 2]), fmaf(kap, vf[c0 + 3] - vv[u + 3], r0[u + 3]));
-                                *reinterpret_cast<float4*>(rw + c0) = r4;
-                                q = fmaf(r4.x, r4.x, q); q = fmaf(r4.y, r4.y, q);
-                                q = fmaf(r4.z, r4.z, q); q = fmaf(r4.w, r4.w, q);
-                            }
-#pragma unroll
-                            for (int u = 0; u < RO; ++u) vq = fmaf(vv[u], vv[u], vq);
-                        }
-                        q = oct_sum(q);
-                        vq = oct_sum(vq);
-                        if (act && o8 == 0) {
-                            const float dn = d0 + kap;
-                            deng[dst] = dn;
-                            a.sp.cache_sc[cbase + dst] = dn > 0.f ? q / (dn * dn) : vq;   // SRE against the new state
-                        }
-                    }
-                }
-                if (f < lam) {                                            // l takes the folded member's slot
-                    const size_t cs = cbase + f;
-                    for (int i = tid; i < DIM; i += NT) {
-                        ((TIn*)a.sp.cache_k)[cs * DIM + i] = ((const TIn*)a.sp.win_k)[wsl * DIM + i];
-                        ((TIn*)a.sp.cache_v)[cs * DIM + i] = vl[i];
-                    }
-                    for (int i = tid; i < D; i += NT) a.sp.cache_phik[cs * D + i] = phl[i];
-                    if (tid == 0) {
-                        a.sp.cache_pos[cs] = lpos;
-                        if (a.scorer) a.sp.cache_sc[cs] = sc[lam];
-                    }
-                }
                 __syncthreads();
                 for (int i = tid; i < D; i += NT) sg[i] = ss[i];
+                if (tail) members_and_slot(f, den_l);
             }
         }
-        __syncthreads();
-        // the new token enters the window ring
-        {
-            const size_t ws = wbase + (size_t)(t % eta);
-            for (int i = tid; i < DIM; i += NT) {
-                ((TIn*)a.sp.win_k)[ws * DIM + i] = kg[i];
-                ((TIn*)a.sp.win_v)[ws * DIM + i] = vg[i];
-            }
-            for (int i = tid; i < D; i += NT) a.sp.win_phik[ws * D + i] = phk[i];
-            if (a.scorer && !a.update_first && tid == 0) a.sp.win_sc[ws] = red[48];
-        }
+        if (tail) ring_write();
     };
 
     const bool needP = leaving && !a.scorer;                      // H^T phi_l for the update
-    if (!a.update_first) {
-        read_phase(NK, rg0, rlo0, needP);
-        update_phase();
+    if (!a.update_first && !a.scorer) {
+        // SRE rule, read first.  The read sees the memories entering the step, so its
+        // products over (H, s) are taken first; then the fold, the read itself, and the
+        // members' residuals right after P V, while their value rows are still in L2.
+        // l's slot and the ring slot are written last, after every read of them.
+        if (!hide_state || needP) h_pass(!hide_state, needP);
+        for (int hh = warp; hh < Gq; hh += NW) {
+            float dl = 0.f;
+            if (!hide_state)
+                for (int j = lane; j < D; j += 32) dl = fmaf(phq[hh * D + j], ss[j], dl);
+            dl = warp_sum(dl);
+            if (lane == 0) red[16 + hh] = dl;
+        }
+        __syncthreads();
+        update_phase(false);
+        read_phase(NK, rg0, rlo0, false, false, true);
+        if (leaving && n_g == lam) members_and_slot(f_fold, den_fold);
+        ring_write();
+    } else if (!a.update_first) {
+        read_phase(NK, rg0, rlo0, !hide_state, needP, false);
+        update_phase(true);
     } else {
         if (needP) h_pass(false, true);
         // the token equations read literally: update, then read the new memories
         // (cache slots [0, min(lambda, t + 1 - eta)), window [t + 1 - eta, t), the token)
-        update_phase();
+        update_phase(true);
         __syncthreads();
         const int rg1 = hide_sparse ? 0 : min(lam, max(0, t + 1 - eta)), rlo1 = max(0, t + 1 - eta);
         const int nk = fill_kp(rg1, rlo1);
         __syncthreads();
-        read_phase(nk, rg1, rlo1, false);                         // over the folded state
+        read_phase(nk, rg1, rlo1, !hide_state, false, false);     // over the folded state
     }
 }
 
