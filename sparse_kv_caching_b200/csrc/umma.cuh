@@ -235,11 +235,6 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* mbar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_addr(mbar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-// Bulk prefetch of a contiguous global range into L2 (a hint; no data moves into
-// the SM).  The address is 16-byte aligned and the size a multiple of 16 bytes.
-__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
 
