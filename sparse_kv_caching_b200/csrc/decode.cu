@@ -20,6 +20,15 @@
 // residual_init_kernel computes them exactly from (H, s) after a prefill.  The
 // pass that updates R_e also stores each member's SRE against the new state,
 // so the next step's scoring reads one float per member instead of R.
+//
+// Layout: one CTA of 256 threads per stream, 64 registers and about 44 KB of
+// shared memory, so that four CTAs share an SM and every stream of a decode
+// batch of 512 streams is resident at once.  H stays in global memory: one
+// streaming pass reads it for phi(q)^T H and H^T phi_l, and the fold updates it
+// in place while it is still in L2.  Under the SRE rule with the read first the
+// step runs: the products over the entering (H, s), the selection and fold, the
+// read, the residual update right after P V (the members' value rows still in
+// L2), and last the writes of l's slot and of the ring slot.
 #include "device_common.cuh"
 #include "umma.cuh"
 
@@ -274,7 +283,8 @@ __global__ void __launch_bounds__(kDecThreads, 4) decode_kernel(const __grid_con
     };
 
     // ---- read: scores (a quad per key), softmax per head, P V (lane owns columns) ----
-    // Eq. 14 over the NK keys of kp and, unless hidden, the state (H, s) in shared memory
+    // Eq. 14 over the NK keys of kp and, unless hidden, the state (H, s): phi(q)^T H from
+    // the H pass (Lq), phi(q) . s from s in shared memory
     // hL / hP: run the H pass after P V for phi(q)^T H / H^T phi_l; dlReady: phi(q) . s
     // is already in red[16 + hh] (taken before a fold that precedes the read)
     auto read_phase = [&](const int NK, const int rg, const int rlo, const bool hL, const bool hP, const bool dlReady) {
