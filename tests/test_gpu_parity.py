@@ -194,6 +194,14 @@ def test_decode_small():
     _decode_check(w, 512, 160, [(0, 0), (1, 1)])
 
 
+@pytest.mark.parametrize("base,Hq,Hkv", [(4, 16, 2), (1, 4, 2)])
+def test_decode_head_groups(base, Hq, Hkv):
+    """Decode after a prefill that fills the cache, with 8 query heads per kv head
+    (bf16, d 128) and with 2 (f32, d 64): both per-head register bounds of the kernel."""
+    w = P.small_workload(base, B=1, Hkv=Hkv, Hq=Hq, T=384, eta=64, lam=48, chunk=64, decode_steps=96)
+    _decode_check(w, 384, 96, [(0, 0), (0, Hkv - 1)])
+
+
 def test_decode_from_empty_state_equals_oracle():
     """Decode from t = 0 (window filling, cache filling, then scoring) is a prefill with C = 1."""
     w = P.small_workload(1, T=64, eta=16, lam=12, chunk=64, decode_steps=200)
